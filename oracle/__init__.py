@@ -1,0 +1,247 @@
+"""Python face of the plain CPU oracle (numpy in, numpy out).
+
+TEST INFRASTRUCTURE ONLY: imported by the tests, by ``__graft_entry__.smoke()``
+and by the benchmark's CPU-baseline / reference leg, never by the product
+package. It shares no code with the CUDA path. Arithmetic lives in
+``oracle.cpp``; this module only marshals arguments.
+
+bf16 tensors are passed as their raw uint16 bit patterns.
+"""
+import ctypes as C
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = C.CDLL(path)
+        u8p, u16p, f32p, f64p = (C.POINTER(C.c_uint8), C.POINTER(C.c_uint16),
+                                  C.POINTER(C.c_float), C.POINTER(C.c_double))
+        i64 = C.c_int64
+        L.oracle_set_threads.argtypes = [C.c_int]
+        L.oracle_get_threads.restype = C.c_int
+        L.oracle_e4m3_decode.argtypes = [C.c_uint8]
+        L.oracle_e4m3_decode.restype = C.c_double
+        L.oracle_e2m1_decode.argtypes = [C.c_uint8]
+        L.oracle_e2m1_decode.restype = C.c_double
+        L.oracle_e4m3_encode.argtypes = [C.c_float]
+        L.oracle_e4m3_encode.restype = C.c_uint8
+        L.oracle_e2m1_encode.argtypes = [C.c_float]
+        L.oracle_e2m1_encode.restype = C.c_uint8
+        L.oracle_e4m3_encode_array.argtypes = [f32p, i64, u8p]
+        L.oracle_e2m1_encode_array.argtypes = [f32p, i64, u8p]
+        L.oracle_e4m3_encode_bits_range.argtypes = [C.c_uint32, i64, u8p]
+        L.oracle_e2m1_encode_bits_range.argtypes = [C.c_uint32, i64, u8p]
+        L.oracle_bf16_from_double.argtypes = [C.c_double]
+        L.oracle_bf16_from_double.restype = C.c_uint16
+        L.oracle_bf16_from_double_array.argtypes = [f64p, i64, u16p]
+        L.oracle_nvfp4_global_scale.argtypes = [u16p, i64]
+        L.oracle_nvfp4_global_scale.restype = C.c_float
+        L.oracle_nvfp4_quantize.argtypes = [u16p, i64, i64, C.c_float, u8p, u8p]
+        L.oracle_nvfp4_quantize.restype = C.c_int
+        L.oracle_nvfp4_dequantize.argtypes = [u8p, u8p, i64, i64, f64p]
+        L.oracle_nvfp4_dequantize.restype = C.c_int
+        L.oracle_nvfp4_linear.argtypes = [u8p, u8p, i64, i64, u8p, u8p, i64, C.c_float,
+                                          C.c_float, f32p, u16p, f64p, f64p]
+        L.oracle_nvfp4_linear.restype = C.c_int
+        L.oracle_nvfp4_linear_unquantized_act.argtypes = [u16p, i64, i64, u8p, u8p, i64,
+                                                          C.c_float, f32p, f64p]
+        L.oracle_nvfp4_linear_unquantized_act.restype = C.c_int
+        L.oracle_fp8r_quantize_rows.argtypes = [u16p, i64, i64, u8p, f32p]
+        L.oracle_fp8r_quantize_rows.restype = C.c_int
+        L.oracle_fp8r_linear.argtypes = [u8p, f32p, i64, i64, u8p, f32p, i64, f32p,
+                                         u16p, f64p, f64p]
+        L.oracle_fp8r_linear.restype = C.c_int
+        _lib = L
+    return _lib
+
+
+def _p(a, ctype):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle inputs must be C-contiguous"
+    return a.ctypes.data_as(C.POINTER(ctype))
+
+
+def _bits16(x):
+    """bf16 data as a contiguous uint16 numpy array (accepts torch bf16 or uint16)."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            return x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(x, dtype=np.uint16)
+
+
+def set_threads(n: int) -> None:
+    lib().oracle_set_threads(int(n))
+
+
+def get_threads() -> int:
+    return int(lib().oracle_get_threads())
+
+
+def e4m3_decode(code: int) -> float:
+    return float(lib().oracle_e4m3_decode(code & 0xFF))
+
+
+def e2m1_decode(nibble: int) -> float:
+    return float(lib().oracle_e2m1_decode(nibble & 0xF))
+
+
+def e4m3_encode(v) -> np.ndarray:
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    out = np.empty(v.shape, np.uint8)
+    lib().oracle_e4m3_encode_array(_p(v, C.c_float), v.size, _p(out, C.c_uint8))
+    return out
+
+
+def e2m1_encode(v) -> np.ndarray:
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    out = np.empty(v.shape, np.uint8)
+    lib().oracle_e2m1_encode_array(_p(v, C.c_float), v.size, _p(out, C.c_uint8))
+    return out
+
+
+def e4m3_encode_bits_range(first: int, count: int) -> np.ndarray:
+    out = np.empty(count, np.uint8)
+    lib().oracle_e4m3_encode_bits_range(first, count, _p(out, C.c_uint8))
+    return out
+
+
+def e2m1_encode_bits_range(first: int, count: int) -> np.ndarray:
+    out = np.empty(count, np.uint8)
+    lib().oracle_e2m1_encode_bits_range(first, count, _p(out, C.c_uint8))
+    return out
+
+
+def bf16_from_double(v) -> np.ndarray:
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    out = np.empty(v.shape, np.uint16)
+    lib().oracle_bf16_from_double_array(_p(v, C.c_double), v.size, _p(out, C.c_uint16))
+    return out
+
+
+def nvfp4_global_scale(x) -> float:
+    """Calibration rule of the workloads: amax / (6 * 448), fp32."""
+    xb = _bits16(x)
+    return float(lib().oracle_nvfp4_global_scale(_p(xb, C.c_uint16), xb.size))
+
+
+def nvfp4_quantize(x, g: float):
+    """bf16 [R, K] -> (codes uint8 [R, K/2], block scales uint8 [R, K/16])."""
+    xb = _bits16(x)
+    R, K = xb.shape
+    q = np.empty((R, K // 2), np.uint8)
+    s = np.empty((R, K // 16), np.uint8)
+    rc = lib().oracle_nvfp4_quantize(_p(xb, C.c_uint16), R, K, np.float32(g),
+                                     _p(q, C.c_uint8), _p(s, C.c_uint8))
+    if rc != 0:
+        raise ValueError(f"oracle_nvfp4_quantize: bad shape {xb.shape}")
+    return q, s
+
+
+def nvfp4_dequantize(q, s) -> np.ndarray:
+    q = np.ascontiguousarray(q, np.uint8)
+    s = np.ascontiguousarray(s, np.uint8)
+    R, K = q.shape[0], q.shape[1] * 2
+    out = np.empty((R, K), np.float64)
+    lib().oracle_nvfp4_dequantize(_p(q, C.c_uint8), _p(s, C.c_uint8), R, K, _p(out, C.c_double))
+    return out
+
+
+def nvfp4_linear(xq, xs, wq, ws, input_scale, weight_scale_2, bias=None):
+    """Returns (y bf16 bits uint16 [M,N], y fp64 [M,N], tolerance scale T fp64 [M,N])."""
+    xq = np.ascontiguousarray(xq, np.uint8)
+    xs = np.ascontiguousarray(xs, np.uint8)
+    wq = np.ascontiguousarray(wq, np.uint8)
+    ws = np.ascontiguousarray(ws, np.uint8)
+    M, K = xq.shape[0], xq.shape[1] * 2
+    N = wq.shape[0]
+    assert wq.shape[1] * 2 == K and xs.shape == (M, K // 16) and ws.shape == (N, K // 16)
+    b = None if bias is None else np.ascontiguousarray(bias, np.float32)
+    y = np.empty((M, N), np.uint16)
+    y64 = np.empty((M, N), np.float64)
+    T = np.empty((M, N), np.float64)
+    rc = lib().oracle_nvfp4_linear(_p(xq, C.c_uint8), _p(xs, C.c_uint8), M, K,
+                                   _p(wq, C.c_uint8), _p(ws, C.c_uint8), N,
+                                   np.float32(input_scale), np.float32(weight_scale_2),
+                                   _p(b, C.c_float), _p(y, C.c_uint16), _p(y64, C.c_double),
+                                   _p(T, C.c_double))
+    if rc != 0:
+        raise ValueError("oracle_nvfp4_linear: bad shape")
+    return y, y64, T
+
+
+def nvfp4_linear_unquantized_act(x, wq, ws, weight_scale_2, bias=None):
+    xb = _bits16(x)
+    wq = np.ascontiguousarray(wq, np.uint8)
+    ws = np.ascontiguousarray(ws, np.uint8)
+    M, K = xb.shape
+    N = wq.shape[0]
+    b = None if bias is None else np.ascontiguousarray(bias, np.float32)
+    y64 = np.empty((M, N), np.float64)
+    rc = lib().oracle_nvfp4_linear_unquantized_act(_p(xb, C.c_uint16), M, K, _p(wq, C.c_uint8),
+                                                   _p(ws, C.c_uint8), N,
+                                                   np.float32(weight_scale_2), _p(b, C.c_float),
+                                                   _p(y64, C.c_double))
+    if rc != 0:
+        raise ValueError("bad shape")
+    return y64
+
+
+def fp8r_quantize_rows(x):
+    """bf16 [R, K] -> (E4M3 codes uint8 [R, K], fp32 row scales [R])."""
+    xb = _bits16(x)
+    R, K = xb.shape
+    q = np.empty((R, K), np.uint8)
+    s = np.empty((R,), np.float32)
+    rc = lib().oracle_fp8r_quantize_rows(_p(xb, C.c_uint16), R, K, _p(q, C.c_uint8),
+                                         _p(s, C.c_float))
+    if rc != 0:
+        raise ValueError("bad shape")
+    return q, s
+
+
+def fp8r_linear(xq, xs, wq, ws, bias=None):
+    """Returns (y bf16 bits uint16 [M,N], y fp64, tolerance scale T)."""
+    xq = np.ascontiguousarray(xq, np.uint8)
+    xs = np.ascontiguousarray(xs, np.float32)
+    wq = np.ascontiguousarray(wq, np.uint8)
+    ws = np.ascontiguousarray(ws, np.float32)
+    M, K = xq.shape
+    N = wq.shape[0]
+    b = None if bias is None else np.ascontiguousarray(bias, np.float32)
+    y = np.empty((M, N), np.uint16)
+    y64 = np.empty((M, N), np.float64)
+    T = np.empty((M, N), np.float64)
+    rc = lib().oracle_fp8r_linear(_p(xq, C.c_uint8), _p(xs, C.c_float), M, K, _p(wq, C.c_uint8),
+                                  _p(ws, C.c_float), N, _p(b, C.c_float), _p(y, C.c_uint16),
+                                  _p(y64, C.c_double), _p(T, C.c_double))
+    if rc != 0:
+        raise ValueError("bad shape")
+    return y, y64, T
+
+
+def bf16_ulp(v) -> np.ndarray:
+    """Spacing of bf16 values at |v|: 2^(floor(log2|v|) - 7) for normal |v|,
+    2^-133 for zero and subnormals."""
+    a = np.abs(np.asarray(v, np.float64))
+    out = np.full(a.shape, 2.0 ** -133)
+    normal = a >= 2.0 ** -126
+    e = np.floor(np.log2(a[normal]))
+    out[normal] = np.ldexp(1.0, (e - 7).astype(np.int64))
+    return out
+
+
+def bf16_bits_to_f64(bits) -> np.ndarray:
+    b = np.ascontiguousarray(bits, np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
