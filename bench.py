@@ -1,0 +1,504 @@
+"""Benchmark of the NVFP4 W4A4 linear (run-time activation quantization + block-
+scaled FP4 GEMM) on the MLP up-projection of a diffusion transformer:
+M = 4096 tokens (64 x 64 latent patches of a 1024 x 1024 image), K = 3072,
+N = 12288, bf16 in / bf16 out, synthetic seeded inputs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one nvfp4_linear call (prologue kernel + GEMM kernel). Each timed step
+is bracketed by CUDA events on the launching stream; a 256 MB buffer is written
+between steps (outside the events) so every step starts with a cold L2. Several
+GPUs run independent replicas (weak scaling; the layer has no exchange step);
+the time is the max over ranks.
+
+Prints one JSON line (rank 0). Extra keys: roofline of the GEMM kernel,
+cpu_baseline (the CPU oracle on a bounded sample), e2e (host buffers, copies
+inside the timed region), clocks sampled during the timed region, and the other
+layer shapes under "variants".
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 W4A4 linear TFLOPS (quant+GEMM) M4096 K3072 N12288; % dense FP4 peak"
+UNIT = "TFLOP/s"
+WORKLOAD = dict(M=4096, K=3072, N=12288)
+NOMINAL_FP4_OVER_BF16 = 4.0      # dense FP4 : dense bf16 tensor rate (9 : 2.25 PFLOP/s)
+NOMINAL_FP8_OVER_BF16 = 2.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- distributed
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def reduce_max(value: float, device=None) -> float:
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def aggregate(local_ms: float, units_per_rank: float, world: int, device=None):
+    """Whole-job throughput: all ranks' units over the slowest rank's time."""
+    ms = reduce_max(local_ms, device)
+    return ms, units_per_rank * world / (ms / 1e3)
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = [
+        ("gpu_idle", 0x1), ("applications_clocks_setting", 0x2), ("sw_power_cap", 0x4),
+        ("hw_slowdown", 0x8), ("sync_boost", 0x10), ("sw_thermal_slowdown", 0x20),
+        ("hw_thermal_slowdown", 0x40), ("hw_power_brake_slowdown", 0x80),
+        ("display_clock_setting", 0x100),
+    ]
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.idx = device_index
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self.ok = False
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self._physical_index())
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+            return self
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
+        return self
+
+    def _physical_index(self):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        if vis:
+            parts = [p for p in vis.split(",") if p.strip()]
+            if self.idx < len(parts) and parts[self.idx].strip().isdigit():
+                return int(parts[self.idx])
+        return self.idx
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        names = [n for n, bit in self.REASONS if self.reasons & bit]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- workloads
+
+def nvfp4_flops(M, K, N):
+    return 2.0 * M * K * N
+
+
+def nvfp4_alg_bytes(M, K, N, bias=False):
+    """Algorithmic bytes of one fused NVFP4 linear: read X (bf16), W codes and
+    scales, bias; write Y (bf16)."""
+    return 2 * M * K + N * K // 2 + N * K // 16 + 2 * M * N + (4 * N if bias else 0)
+
+
+class Nvfp4Layer:
+    """Device-resident NVFP4 layer: W quantized on the GPU (same kernel as the
+    activations), input_scale calibrated on the GPU (amax / 2688)."""
+
+    def __init__(self, M, K, N, bias, device, seed=0):
+        import torch
+        import fp8_rowwise_quantized_b200 as q
+        from synthetic import make_linear_inputs
+        inp = make_linear_inputs(M, K, N, seed=seed, with_bias=bias)
+        self.M, self.K, self.N = M, K, N
+        self.x_host = inp.x
+        self.x = inp.x.to(device)
+        w = inp.w.to(device)
+        self.wq, self.ws, self.gw = q.prepare_nvfp4_weight(w)
+        del w
+        self.gx = q.nvfp4_global_scale(self.x)
+        self.bias = None if inp.bias is None else inp.bias.to(device)
+        self.y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        self.work = torch.empty(q.nvfp4_linear_workspace_size(M, K, N), dtype=torch.uint8,
+                                device=device)
+        self.q = q
+
+    def step(self):
+        self.q.nvfp4_linear(self.x, self.wq, self.ws, self.gw, self.gx, bias=self.bias, y=self.y,
+                            workspace=self.work)
+
+    def prologue(self):
+        self.q.nvfp4_linear_prologue(self.x, self.ws, self.gx, self.work)
+
+    def gemm(self):
+        self.q.nvfp4_linear_gemm(self.M, self.wq, self.gw, self.gx, self.work, bias=self.bias,
+                                 y=self.y)
+
+
+class Fp8rLayer:
+    def __init__(self, M, K, N, bias, device, seed=0):
+        import torch
+        import fp8_rowwise_quantized_b200 as q
+        from synthetic import make_linear_inputs
+        inp = make_linear_inputs(M, K, N, seed=seed, with_bias=bias)
+        self.M, self.K, self.N = M, K, N
+        self.x = inp.x.to(device)
+        self.wq, self.wsc = q.prepare_fp8r_weight(inp.w.to(device))
+        self.bias = None if inp.bias is None else inp.bias.to(device)
+        self.y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        self.work = torch.empty(q.fp8r_linear_workspace_size(M, K, N), dtype=torch.uint8,
+                                device=device)
+        self.xq, self.xs = q.fp8r_quantize_rows(self.x)
+        self.q = q
+
+    def step(self):
+        self.q.fp8r_linear(self.x, self.wq, self.wsc, bias=self.bias, y=self.y,
+                           workspace=self.work)
+
+    def gemm(self):
+        self.q.fp8r_linear_gemm(self.xq, self.xs, self.wq, self.wsc, bias=self.bias, y=self.y)
+
+
+def time_events(fn, steps, warmup, flush, stream):
+    """Mean device time (ms) of fn over `steps` calls, each bracketed by CUDA events
+    on `stream`, with an L2 flush (outside the events) before every call."""
+    import torch
+    for _ in range(warmup):
+        flush()
+        fn()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for i in range(steps):
+        flush()
+        starts[i].record(stream)
+        fn()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    times = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    return statistics.fmean(times), times
+
+
+def traffic_from_profiles(kernel_key: str):
+    """Per-launch DRAM bytes of a kernel from the committed ncu summary, or None
+    when the kernel source changed since the capture."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[kernel_key]
+    except (OSError, ValueError, KeyError):
+        return None
+    src_hash = source_hash(rec.get("sources", []))
+    if src_hash != rec.get("source_sha1"):
+        return None
+    return rec.get("bytes_per_launch")
+
+
+def source_hash(files):
+    h = hashlib.sha1()
+    for rel in files:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def cpu_oracle_sample(M, K, N, target_s=12.0, min_rows=4):
+    """Time the oracle (as it stands) on a bounded row sample of the workload:
+    activation quantization of the sampled rows + fp64 contraction against the
+    whole weight. Returns (TFLOP/s, threads, rows, seconds)."""
+    import numpy as np
+    import oracle
+    from synthetic import make_linear_inputs
+    inp = make_linear_inputs(M, K, N, seed=0)
+    gw = oracle.nvfp4_global_scale(inp.w)
+    wq, ws = oracle.nvfp4_quantize(inp.w, gw)
+    gx = oracle.nvfp4_global_scale(inp.x)
+    x = inp.x
+
+    def run(rows):
+        t0 = time.perf_counter()
+        xq, xs = oracle.nvfp4_quantize(x[:rows], gx)
+        oracle.nvfp4_linear(xq, xs, wq, ws, gx, gw)
+        return time.perf_counter() - t0
+
+    rows = min_rows
+    t = run(rows)
+    if t < target_s / 4:
+        rows = int(min(M, max(rows, rows * (target_s / max(t, 1e-3)) * 0.9)))
+        t = run(rows)
+    tflops = nvfp4_flops(rows, K, N) / t / 1e12
+    return tflops, oracle.get_threads(), rows, t
+
+
+# ----------------------------------------------------------------------------- arms
+
+def run_reference(args):
+    """The CPU oracle as the reference arm: each step is a bounded row sample of
+    the workload, timed on the host cores."""
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    import numpy as np
+    from synthetic import make_linear_inputs
+    M, K, N = WORKLOAD["M"], WORKLOAD["K"], WORKLOAD["N"]
+    inp = make_linear_inputs(M, K, N, seed=0)
+    gw = oracle.nvfp4_global_scale(inp.w)
+    wq, ws = oracle.nvfp4_quantize(inp.w, gw)
+    gx = oracle.nvfp4_global_scale(inp.x)
+    # size one step so that warmup + steps take about two minutes in total
+    t0 = time.perf_counter()
+    xq, xs = oracle.nvfp4_quantize(inp.x[:4], gx)
+    oracle.nvfp4_linear(xq, xs, wq, ws, gx, gw)
+    t4 = time.perf_counter() - t0
+    per_step = 120.0 / max(1, args.steps + args.warmup)
+    rows = int(max(1, min(M, 4 * per_step / max(t4, 1e-3))))
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        xq, xs = oracle.nvfp4_quantize(inp.x[:rows], gx)
+        oracle.nvfp4_linear(xq, xs, wq, ws, gx, gw)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+    sec = statistics.fmean(times)
+    value = nvfp4_flops(rows, K, N) / sec / 1e12
+    sample = f"{rows} of {M} activation rows per step (all N={N}, K={K}); quantize + fp64 contraction"
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": "nvfp4_mlp_up M4096 K3072 N12288", **WORKLOAD},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.get_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(device)
+    import fp8_rowwise_quantized_b200 as q
+    peaks, peak_src = load_peaks()
+    M, K, N = WORKLOAD["M"], WORKLOAD["K"], WORKLOAD["N"]
+
+    layer = Nvfp4Layer(M, K, N, bias=False, device=device)
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def flush():
+        flush_buf.fill_(1)
+
+    # --------------------------------------------------- headline: timed steps
+    for _ in range(args.warmup):
+        flush()
+        layer.step()
+    torch.cuda.synchronize()
+    barrier(device)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush()
+            starts[i].record(stream)
+            layer.step()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    barrier(device)
+    torch.cuda.synchronize()
+    local_ms = statistics.fmean(s.elapsed_time(e) for s, e in zip(starts, ends))
+    flops = nvfp4_flops(M, K, N)
+    ms, value_flops = aggregate(local_ms, flops, world, device)
+    value = value_flops / 1e12
+    status = q.read_device_status()
+
+    # --------------------------------------------------- roofline of the GEMM kernel
+    fp4_peak = peaks["bf16_tflops"] * NOMINAL_FP4_OVER_BF16
+    roof_steps = max(20, min(args.steps, 200))
+    layer.prologue()
+    gemm_ms, _ = time_events(layer.gemm, roof_steps, 3, flush, stream)
+    prol_ms, _ = time_events(layer.prologue, roof_steps, 3, flush, stream)
+    gemm_tflops = flops / (gemm_ms / 1e3) / 1e12
+    prologue_bytes = 2 * M * K + M * K // 2 + M * K // 16 + 2 * (N * K // 16)
+    roofline = {
+        "kernel": "qgemm_kernel<FP4, BN=192> (tcgen05 block-scaled FP4 GEMM)",
+        "bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
+        "frac": gemm_tflops / fp4_peak,
+        "traffic": traffic_from_profiles("nvfp4_gemm_mlp_up"),
+        "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {NOMINAL_FP4_OVER_BF16} "
+                       "(nominal dense FP4:bf16 ratio)",
+        "gemm_us": gemm_ms * 1e3,
+        "prologue_us": prol_ms * 1e3,
+        "prologue_gbs": prologue_bytes / (prol_ms / 1e3) / 1e9,
+        "prologue_hbm_frac": prologue_bytes / (prol_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+        "frac_of_nominal_9pf": gemm_tflops / 9000.0,
+        "step_frac_of_fp4_peak": value / world / fp4_peak,
+    }
+
+    # --------------------------------------------------- e2e through the public API
+    e2e = None
+    if not args.no_e2e:
+        x_pin = layer.x_host.pin_memory()
+        y_pin = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+        x_dev = torch.empty_like(layer.x)
+
+        def e2e_step():
+            x_dev.copy_(x_pin, non_blocking=True)
+            q.nvfp4_linear(x_dev, layer.wq, layer.ws, layer.gw, layer.gx, y=layer.y,
+                           workspace=layer.work)
+            y_pin.copy_(layer.y, non_blocking=True)
+
+        e_steps = max(10, min(args.steps, 50))
+        e_ms, _ = time_events(e2e_step, e_steps, 3, flush, stream)
+        e_ms, e_val = aggregate(e_ms, flops, world, device)
+        e2e = {"value": e_val / 1e12, "unit": UNIT, "h2d_bytes_per_step": 2 * M * K,
+               "d2h_bytes_per_step": 2 * M * N, "ms_per_step": e_ms}
+
+    # --------------------------------------------------- other layer shapes
+    variants = {}
+    if not args.no_variants:
+        v_steps = max(10, min(args.steps, 100))
+        for name, (kind, Mv, Kv, Nv, bias) in {
+            "fp8r_4096x3072x3072": ("fp8r", 4096, 3072, 3072, False),
+            "nvfp4_attn_proj_4096x3072x3072_bias": ("nvfp4", 4096, 3072, 3072, True),
+            "nvfp4_attn_qkv_4096x3072x9216_bias": ("nvfp4", 4096, 3072, 9216, True),
+            "nvfp4_mlp_down_4096x12288x3072": ("nvfp4", 4096, 12288, 3072, False),
+        }.items():
+            L = (Fp8rLayer if kind == "fp8r" else Nvfp4Layer)(Mv, Kv, Nv, bias, device)
+            vms, _ = time_events(L.step, v_steps, 3, flush, stream)
+            gms, _ = time_events(L.gemm, v_steps, 3, flush, stream)
+            fl = nvfp4_flops(Mv, Kv, Nv)
+            pk = peaks["bf16_tflops"] * (NOMINAL_FP8_OVER_BF16 if kind == "fp8r" else NOMINAL_FP4_OVER_BF16)
+            variants[name] = {"us": vms * 1e3, "tflops": fl / (vms / 1e3) / 1e12,
+                              "gemm_us": gms * 1e3, "gemm_tflops": fl / (gms / 1e3) / 1e12,
+                              "gemm_frac_of_peak": fl / (gms / 1e3) / 1e12 / pk}
+            del L
+        torch.cuda.empty_cache()
+
+    # --------------------------------------------------- CPU oracle baseline (rank 0, N=1)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tfl, cores, rows, sec = cpu_oracle_sample(M, K, N)
+        cpu = {"value": tfl, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{rows} of {M} activation rows, all N={N}, K={K} (quantize + fp64 "
+                         f"contraction), {sec:.1f} s"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e2m1xe2m1->f32 (bf16 in/out)", "data": "synthetic",
+        "config": {"workload": "nvfp4_mlp_up M4096 K3072 N12288", **WORKLOAD,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "flushed (256 MB write) before every step, outside the events"},
+        "frac_of_fp4_peak": value / world / fp4_peak,
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "clocks": clk.summary(),
+        "gpu_launches": 2 * args.steps,
+        "device_status": status,
+        "variants": variants,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        barrier(device)
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-variants", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

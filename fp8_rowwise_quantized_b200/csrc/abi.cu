@@ -1,0 +1,336 @@
+// C ABI of the quantized linear (declared in include/qlinear.h): argument
+// validation, workspace carving, device checks, the device status word and the
+// error text. Every step of the computation runs in the kernels of quantize.cu
+// and gemm.cu; this file only checks arguments and launches them.
+#include <cuda_runtime.h>
+#include <atomic>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/qlinear.h"
+#include "internal.h"
+#include "layout.cuh"
+
+namespace {
+
+// Status word written by kernels whose bounded waits expire (one per device).
+__device__ int g_device_status;
+
+thread_local char g_last_error[256] = "";
+std::atomic<int> g_inject_fault{0};
+std::atomic<int> g_timeout_ms{2000};
+
+int record(cudaError_t e, const char* where) {
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%s)", where, cudaGetErrorName(e),
+                cudaGetErrorString(e));
+  return QL_ERR_LAUNCH;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Current device must be an sm_100 part; returns QL_OK or an error code.
+int check_device(int* dev_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return record(e, "cudaGetDevice");
+  static int cc_cache[64] = {};  // 0 = unknown, else major*10+minor
+  int cc = dev < 64 ? cc_cache[dev] : 0;
+  if (cc == 0) {
+    int major = 0, minor = 0;
+    e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e != cudaSuccess) return record(e, "cudaDeviceGetAttribute");
+    e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (e != cudaSuccess) return record(e, "cudaDeviceGetAttribute");
+    cc = major * 10 + minor;
+    if (dev < 64) cc_cache[dev] = cc;
+  }
+  if (cc != 100) {
+    std::snprintf(g_last_error, sizeof(g_last_error),
+                  "device %d has compute capability %d.%d; this library runs on sm_100 only", dev,
+                  cc / 10, cc % 10);
+    return QL_ERR_DEVICE;
+  }
+  if (dev_out) *dev_out = dev;
+  return QL_OK;
+}
+
+int* status_ptr(int dev) {
+  static int* cache[64] = {};
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 64 && cache[dev]) return cache[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+  if (dev < 64) cache[dev] = static_cast<int*>(p);
+  return static_cast<int*>(p);
+}
+
+int fail_shape(const char* what) {
+  std::snprintf(g_last_error, sizeof(g_last_error), "shape: %s", what);
+  return QL_ERR_SHAPE;
+}
+
+uint64_t timeout_ns() { return static_cast<uint64_t>(g_timeout_ms.load()) * 1000000ull; }
+
+bool nvfp4_shape_ok(int64_t M, int64_t K, int64_t N) {
+  return M >= 1 && N >= 1 && K >= 32 && K % 32 == 0 && M <= (1ll << 30) && N <= (1ll << 30) &&
+         K <= (1ll << 30);
+}
+
+bool fp8r_shape_ok(int64_t M, int64_t K, int64_t N) {
+  return M >= 1 && N >= 1 && K >= 16 && K % 16 == 0 && M <= (1ll << 30) && N <= (1ll << 30) &&
+         K <= (1ll << 30);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ql_status_string(int status) {
+  switch (status) {
+    case QL_OK: return "ok";
+    case QL_ERR_INVALID_ARG: return "invalid argument (null pointer or non-positive size)";
+    case QL_ERR_SHAPE: return "unsupported shape";
+    case QL_ERR_ALIGN: return "base pointer not 16-byte aligned";
+    case QL_ERR_DEVICE: return "device is not sm_100";
+    case QL_ERR_WORKSPACE: return "workspace missing or too small";
+    case QL_ERR_LAUNCH: return "CUDA launch or runtime error";
+    case QL_ERR_TIMEOUT: return "a kernel's bounded wait expired";
+  }
+  return "unknown status";
+}
+
+const char* ql_last_error_message(void) { return g_last_error; }
+
+void ql_set_fault_injection(int enable, int timeout_ms) {
+  g_inject_fault.store(enable ? 1 : 0);
+  g_timeout_ms.store(timeout_ms > 0 ? timeout_ms : 2000);
+}
+
+int ql_read_device_status(int* status) {
+  if (!status) return QL_ERR_INVALID_ARG;
+  int dev = 0;
+  int rc = check_device(&dev);
+  if (rc != QL_OK) return rc;
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int));
+  if (e != cudaSuccess) return record(e, "cudaMemcpyFromSymbol");
+  const int zero = 0;
+  e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
+  if (e != cudaSuccess) return record(e, "cudaMemcpyToSymbol");
+  *status = v;
+  return QL_OK;
+}
+
+// ------------------------------------------------------------------ NVFP4
+
+int nvfp4_quantize_act(const void* x, int64_t M, int64_t K, const float* input_scale,
+                       uint8_t* xq, uint8_t* xs, ql_stream_t stream) {
+  if (!x || !input_scale || !xq || !xs || M <= 0 || K <= 0) return QL_ERR_INVALID_ARG;
+  if (K % 16 != 0) return fail_shape("K must be a multiple of 16");
+  if (!aligned16(x) || !aligned16(xq)) return QL_ERR_ALIGN;
+  int rc = check_device(nullptr);
+  if (rc != QL_OK) return rc;
+  cudaError_t e = ql::launch_nvfp4_quantize_rowmajor(x, M, K, input_scale, xq, xs,
+                                                     reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QL_OK : record(e, "nvfp4_quantize_act");
+}
+
+size_t nvfp4_linear_workspace_size(int64_t M, int64_t K, int64_t N) {
+  if (!nvfp4_shape_ok(M, K, N)) return 0;
+  return ql::nvfp4_workspace(M, K, N, ql::choose_bn(true, M, N)).total;
+}
+
+int nvfp4_linear_workspace_layout(int64_t M, int64_t K, int64_t N, size_t* codes_offset,
+                                  size_t* act_scales_offset, size_t* weight_scales_offset) {
+  if (!nvfp4_shape_ok(M, K, N)) return QL_ERR_SHAPE;
+  const ql::Nvfp4Workspace L = ql::nvfp4_workspace(M, K, N, ql::choose_bn(true, M, N));
+  if (codes_offset) *codes_offset = L.codes_off;
+  if (act_scales_offset) *act_scales_offset = L.act_sf_off;
+  if (weight_scales_offset) *weight_scales_offset = L.wgt_sf_off;
+  return QL_OK;
+}
+
+int nvfp4_linear_prologue(const void* x, int64_t M, int64_t K, const uint8_t* w_scale, int64_t N,
+                          const float* input_scale, void* workspace, size_t workspace_bytes,
+                          ql_stream_t stream) {
+  if (!x || !w_scale || !input_scale || M <= 0 || N <= 0 || K <= 0) return QL_ERR_INVALID_ARG;
+  if (!nvfp4_shape_ok(M, K, N)) return fail_shape("nvfp4: needs K >= 32 and K % 32 == 0");
+  if (!aligned16(x)) return QL_ERR_ALIGN;
+  const int bn = ql::choose_bn(true, M, N);
+  const ql::Nvfp4Workspace L = ql::nvfp4_workspace(M, K, N, bn);
+  if (!workspace || workspace_bytes < L.total) return QL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return QL_ERR_ALIGN;
+  int rc = check_device(nullptr);
+  if (rc != QL_OK) return rc;
+  cudaError_t e = ql::launch_nvfp4_prologue(x, M, K, w_scale, N, bn, input_scale,
+                                            static_cast<uint8_t*>(workspace),
+                                            reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QL_OK : record(e, "nvfp4_linear_prologue");
+}
+
+static int nvfp4_gemm_impl(int64_t M, int64_t K, const uint8_t* w, int64_t N,
+                           const float* weight_scale_2, const float* input_scale,
+                           const float* bias, void* y, const void* workspace,
+                           size_t workspace_bytes, ql_stream_t stream, bool pdl) {
+  if (!w || !weight_scale_2 || !input_scale || !y || M <= 0 || N <= 0 || K <= 0)
+    return QL_ERR_INVALID_ARG;
+  if (!nvfp4_shape_ok(M, K, N)) return fail_shape("nvfp4: needs K >= 32 and K % 32 == 0");
+  if (!aligned16(w) || !aligned16(y) || (bias && !aligned16(bias))) return QL_ERR_ALIGN;
+  const int bn = ql::choose_bn(true, M, N);
+  const ql::Nvfp4Workspace L = ql::nvfp4_workspace(M, K, N, bn);
+  if (!workspace || workspace_bytes < L.total) return QL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return QL_ERR_ALIGN;
+  int dev = 0;
+  int rc = check_device(&dev);
+  if (rc != QL_OK) return rc;
+  const uint8_t* ws = static_cast<const uint8_t*>(workspace);
+  ql::GemmProblem p{};
+  p.fp4 = true;
+  p.bn = bn;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.a = ws + L.codes_off;
+  p.b = w;
+  p.sfa = ws + L.act_sf_off;
+  p.sfb = ws + L.wgt_sf_off;
+  p.scale_a = input_scale;
+  p.scale_b = weight_scale_2;
+  p.bias = bias;
+  p.y = y;
+  p.status = status_ptr(dev);
+  p.timeout_ns = timeout_ns();
+  p.inject_fault = g_inject_fault.load();
+  p.pdl = pdl;
+  cudaError_t e = ql::launch_gemm(p, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QL_OK : record(e, "nvfp4 gemm launch");
+}
+
+int nvfp4_linear_gemm(int64_t M, int64_t K, const uint8_t* w, int64_t N,
+                      const float* weight_scale_2, const float* input_scale, const float* bias,
+                      void* y, const void* workspace, size_t workspace_bytes, ql_stream_t stream) {
+  return nvfp4_gemm_impl(M, K, w, N, weight_scale_2, input_scale, bias, y, workspace,
+                         workspace_bytes, stream, false);
+}
+
+int nvfp4_linear(const void* x, int64_t M, int64_t K, const uint8_t* w, const uint8_t* w_scale,
+                 int64_t N, const float* weight_scale_2, const float* input_scale,
+                 const float* bias, void* y, void* workspace, size_t workspace_bytes,
+                 ql_stream_t stream) {
+  if (!x || !w || !w_scale || !weight_scale_2 || !input_scale || !y || M <= 0 || N <= 0 || K <= 0)
+    return QL_ERR_INVALID_ARG;
+  if (!nvfp4_shape_ok(M, K, N)) return fail_shape("nvfp4: needs K >= 32 and K % 32 == 0");
+  if (!aligned16(x) || !aligned16(w) || !aligned16(y) || (bias && !aligned16(bias)))
+    return QL_ERR_ALIGN;
+  const ql::Nvfp4Workspace L = ql::nvfp4_workspace(M, K, N, ql::choose_bn(true, M, N));
+  if (!workspace || workspace_bytes < L.total) return QL_ERR_WORKSPACE;
+  int rc = nvfp4_linear_prologue(x, M, K, w_scale, N, input_scale, workspace, workspace_bytes,
+                                 stream);
+  if (rc != QL_OK) return rc;
+  return nvfp4_gemm_impl(M, K, w, N, weight_scale_2, input_scale, bias, y, workspace,
+                         workspace_bytes, stream, true);
+}
+
+int nvfp4_global_scale(const void* x, int64_t n, float* out, ql_stream_t stream) {
+  if (!x || !out || n <= 0) return QL_ERR_INVALID_ARG;
+  int rc = check_device(nullptr);
+  if (rc != QL_OK) return rc;
+  cudaError_t e = ql::launch_global_scale(x, n, out, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QL_OK : record(e, "nvfp4_global_scale");
+}
+
+// ------------------------------------------------------------------ fp8r
+
+int fp8r_quantize_rows(const void* x, int64_t M, int64_t K, uint8_t* xq, float* x_scale,
+                       ql_stream_t stream) {
+  if (!x || !xq || !x_scale || M <= 0 || K <= 0) return QL_ERR_INVALID_ARG;
+  if (K % 8 != 0) return fail_shape("fp8r: K must be a multiple of 8");
+  if (!aligned16(x) || !aligned16(xq)) return QL_ERR_ALIGN;
+  int rc = check_device(nullptr);
+  if (rc != QL_OK) return rc;
+  cudaError_t e = ql::launch_fp8r_quantize_rows(x, M, K, xq, x_scale,
+                                                reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QL_OK : record(e, "fp8r_quantize_rows");
+}
+
+size_t fp8r_linear_workspace_size(int64_t M, int64_t K, int64_t N) {
+  if (!fp8r_shape_ok(M, K, N)) return 0;
+  return ql::align_up(static_cast<size_t>(M) * static_cast<size_t>(K), 1024) +
+         ql::align_up(static_cast<size_t>(M) * 4, 1024);
+}
+
+static int fp8r_gemm_impl(const uint8_t* xq, const float* x_scale, int64_t M, int64_t K,
+                          const uint8_t* w, const float* w_scale, int64_t N, const float* bias,
+                          void* y, ql_stream_t stream, bool pdl) {
+  if (!xq || !x_scale || !w || !w_scale || !y || M <= 0 || N <= 0 || K <= 0)
+    return QL_ERR_INVALID_ARG;
+  if (!fp8r_shape_ok(M, K, N)) return fail_shape("fp8r: needs K >= 16 and K % 16 == 0");
+  if (!aligned16(xq) || !aligned16(w) || !aligned16(y) || !aligned16(w_scale) ||
+      (bias && !aligned16(bias)))
+    return QL_ERR_ALIGN;
+  int dev = 0;
+  int rc = check_device(&dev);
+  if (rc != QL_OK) return rc;
+  ql::GemmProblem p{};
+  p.fp4 = false;
+  p.bn = ql::choose_bn(false, M, N);
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.a = xq;
+  p.b = w;
+  p.scale_a = x_scale;
+  p.scale_b = w_scale;
+  p.bias = bias;
+  p.y = y;
+  p.status = status_ptr(dev);
+  p.timeout_ns = timeout_ns();
+  p.inject_fault = g_inject_fault.load();
+  p.pdl = pdl;
+  cudaError_t e = ql::launch_gemm(p, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QL_OK : record(e, "fp8r gemm launch");
+}
+
+int fp8r_linear_gemm(const uint8_t* xq, const float* x_scale, int64_t M, int64_t K,
+                     const uint8_t* w, const float* w_scale, int64_t N, const float* bias, void* y,
+                     ql_stream_t stream) {
+  return fp8r_gemm_impl(xq, x_scale, M, K, w, w_scale, N, bias, y, stream, false);
+}
+
+int fp8r_linear(const void* x, int64_t M, int64_t K, const uint8_t* w, const float* w_scale,
+                int64_t N, const float* bias, void* y, void* workspace, size_t workspace_bytes,
+                ql_stream_t stream) {
+  if (!x || !w || !w_scale || !y || M <= 0 || N <= 0 || K <= 0) return QL_ERR_INVALID_ARG;
+  if (!fp8r_shape_ok(M, K, N)) return fail_shape("fp8r: needs K >= 16 and K % 16 == 0");
+  const size_t need = fp8r_linear_workspace_size(M, K, N);
+  if (!workspace || workspace_bytes < need) return QL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return QL_ERR_ALIGN;
+  uint8_t* xq = static_cast<uint8_t*>(workspace);
+  float* xs = reinterpret_cast<float*>(xq + ql::align_up(static_cast<size_t>(M) * K, 1024));
+  int rc = fp8r_quantize_rows(x, M, K, xq, xs, stream);
+  if (rc != QL_OK) return rc;
+  return fp8r_gemm_impl(xq, xs, M, K, w, w_scale, N, bias, y, stream, true);
+}
+
+// ------------------------------------------------------------------ diagnostics
+
+int ql_encode_e4m3(const float* in, uint8_t* out, int64_t n, ql_stream_t stream) {
+  if (!in || !out || n <= 0) return QL_ERR_INVALID_ARG;
+  int rc = check_device(nullptr);
+  if (rc != QL_OK) return rc;
+  cudaError_t e = ql::launch_encode(in, out, n, false, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QL_OK : record(e, "ql_encode_e4m3");
+}
+
+int ql_encode_e2m1(const float* in, uint8_t* out, int64_t n, ql_stream_t stream) {
+  if (!in || !out || n <= 0) return QL_ERR_INVALID_ARG;
+  int rc = check_device(nullptr);
+  if (rc != QL_OK) return rc;
+  cudaError_t e = ql::launch_encode(in, out, n, true, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QL_OK : record(e, "ql_encode_e2m1");
+}
+
+}  // extern "C"

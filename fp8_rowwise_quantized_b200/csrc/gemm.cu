@@ -1,0 +1,507 @@
+// Tensor-core GEMMs of the quantized linear (sm_100a, tcgen05):
+//   FP4 = true : Y = bf16(input_scale * weight_scale_2 * sum_k A*SFA * B*SFB + bias),
+//                A, B packed E2M1, SFA/SFB E4M3 per 16 elements (kind::mxf4nvf4);
+//   FP4 = false: Y = bf16(x_scale[m] * w_scale[n] * sum_k A * B + bias),
+//                A, B E4M3 (kind::f8f6f4).
+// The block-scaled FP4 GEMM is the "mm_fp4" step and the FP8 one the "scaled GEMM
+// with row-wise scales" step of the Diffusers page "BFL (fp8r / nvfp4)", section
+// "Kernels", table.
+//
+// Structure: one persistent CTA per SM walks output tiles of 128 x BN.
+//   warp 0     TMA producer: A and B tiles (128-byte swizzle), scale atoms (bulk
+//              copies), into a STAGES-deep shared-memory ring;
+//   warp 1     allocates TMEM and issues the MMAs from one thread: per stage it
+//              copies the scale atoms into TMEM (tcgen05.cp) and issues 4 MMAs of
+//              K = 64 (FP4) or K = 32 (FP8) into a TMEM accumulator;
+//   warps 2-5  epilogue: TMEM -> registers (tcgen05.ld), scale, bias, bf16, store.
+// Accumulators are double-buffered in TMEM when they fit (BN <= 192), so the
+// epilogue of one tile overlaps the main loop of the next.
+// Every wait is bounded by a deadline; on expiry the kernel records
+// QL_ERR_TIMEOUT in the device status word, drains its own copies and MMAs,
+// frees TMEM and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+#include "layout.cuh"
+#include "ptx.cuh"
+
+namespace ql {
+
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kThreads = 192;
+constexpr int kSmemLimit = 232448;  // 227 KB opt-in per block
+constexpr int kTmemCols = 512;
+
+struct GemmArgs {
+  int M, N, K;
+  int tiles_m, tiles_n, num_k_tiles, total_tiles;
+  int64_t kg;               // FP4: 64-element scale groups per row (padded)
+  const uint8_t* sfa;       // FP4: activation scale atoms
+  const uint8_t* sfb;       // FP4: weight scale atoms
+  const float* scale_a;     // FP4: input_scale (scalar)   FP8: x_scale [M]
+  const float* scale_b;     // FP4: weight_scale_2 (scalar) FP8: w_scale [N]
+  const float* bias;        // [N] or null
+  uint16_t* y;              // bf16 [M, N]
+  int* status;              // device status word
+  uint64_t timeout_ns;
+  int inject_fault;
+  int wait_prior_grid;
+};
+
+template <bool FP4, int BN>
+struct Cfg {
+  static constexpr int NA = (BN + 127) / 128;                       // 128-row scale atoms of B
+  static constexpr int A_BYTES = kBM * 128;
+  static constexpr int B_BYTES = BN * 128;
+  static constexpr int SFA_BYTES = FP4 ? 4 * kSfAtomBytes : 0;      // 4 K-groups x 1 atom
+  static constexpr int SFB_BYTES = FP4 ? 4 * NA * kSfAtomBytes : 0; // 4 K-groups x NA atoms
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int RESERVED = 1024 /*alignment*/ + 1024 /*barriers*/;
+  static constexpr int STAGES_FIT = (kSmemLimit - RESERVED) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+  static constexpr int NACC = (2 * BN + 16 + 4 * NA * 4 <= kTmemCols) ? 2 : 1;
+  static constexpr int SFA_COL = NACC * BN;
+  static constexpr int SFB_COL = SFA_COL + 16;
+  static constexpr int SMEM = RESERVED + STAGES * STAGE_BYTES;
+  // instruction descriptor: M = 128, N = BN, K-major A and B, fp32 accumulate;
+  // FP4: E2M1 x E2M1 with UE4M3 scales; FP8: E4M3 x E4M3.
+  static constexpr uint32_t IDESC =
+      FP4 ? ((1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(kBM >> 4) << 24))
+          : ((1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(kBM >> 4) << 24));
+  static_assert(STAGES >= 2, "shared memory too small for two stages");
+  static_assert(SFB_COL + 4 * NA * 4 <= kTmemCols, "TMEM budget");
+  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "tile width");
+};
+
+__device__ __forceinline__ void record_timeout(int* status) {
+  if (status) atomicCAS(status, 0, static_cast<int>(QL_ERR_TIMEOUT_CODE));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&p);
+}
+
+template <bool FP4, int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+             const GemmArgs args) {
+  using C = Cfg<FP4, BN>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* smem_a = smem;
+  uint8_t* smem_b = smem_a + C::STAGES * C::A_BYTES;
+  uint8_t* smem_sfa = smem_b + C::STAGES * C::B_BYTES;
+  uint8_t* smem_sfb = smem_sfa + C::STAGES * C::SFA_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_sfb + C::STAGES * C::SFB_BYTES);
+  uint64_t* full_bar = bars;
+  uint64_t* empty_bar = bars + C::STAGES;
+  uint64_t* tfull_bar = bars + 2 * C::STAGES;
+  uint64_t* tempty_bar = tfull_bar + 2;
+  uint64_t* drain_bar = tempty_bar + 2;
+  uint64_t* never_bar = drain_bar + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(never_bar + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const uint64_t deadline = globaltimer_ns() + args.timeout_ns;
+
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tmap_a);
+    prefetch_tmap(&tmap_b);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull_bar[b], 1);
+      mbar_init(&tempty_bar[b], 4);
+    }
+    mbar_init(drain_bar, 1);
+    mbar_init(never_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  // Everything above overlaps the tail of the previous kernel on the stream;
+  // global inputs are read only after it has completed.
+  if (args.wait_prior_grid) grid_dependency_wait();
+
+  bool run = true;
+  if (args.inject_fault) {
+    run = false;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      if (!mbar_wait_bounded(never_bar, 0, deadline)) record_timeout(args.status);
+    }
+  }
+
+  if (run && warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    int issued = 0;
+    for (int tile = blockIdx.x; ok && tile < args.total_tiles; tile += gridDim.x) {
+      const int m_blk = tile % args.tiles_m;
+      const int n_blk = tile / args.tiles_m;
+      for (int kt = 0; kt < args.num_k_tiles; ++kt) {
+        if (!warp_wait_bounded(&empty_bar[stage], phase ^ 1u, deadline)) {
+          ok = false;
+          break;
+        }
+        if (elect_one()) {
+          mbar_arrive_expect_tx(&full_bar[stage], C::STAGE_BYTES);
+          tma_load_2d(smem_a + stage * C::A_BYTES, &tmap_a, &full_bar[stage], kt * 128,
+                      m_blk * kBM);
+          tma_load_2d(smem_b + stage * C::B_BYTES, &tmap_b, &full_bar[stage], kt * 128,
+                      n_blk * BN);
+          if constexpr (FP4) {
+            const uint8_t* sfa = args.sfa + (static_cast<int64_t>(m_blk) * args.kg + kt * 4) *
+                                                kSfAtomBytes;
+            const uint8_t* sfb = args.sfb + ((static_cast<int64_t>(n_blk) * args.kg + kt * 4) *
+                                             C::NA) * kSfAtomBytes;
+            bulk_load(smem_sfa + stage * C::SFA_BYTES, sfa, C::SFA_BYTES, &full_bar[stage]);
+            bulk_load(smem_sfb + stage * C::SFB_BYTES, sfb, C::SFB_BYTES, &full_bar[stage]);
+          }
+        }
+        __syncwarp();
+        ++issued;
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok) {
+      record_timeout(args.status);
+      *abort_flag = 1;
+      // wait (bounded) for the copies this warp still has in flight
+      const uint64_t drain_deadline = globaltimer_ns() + 100000000ull;
+      const int n = issued < C::STAGES ? issued : C::STAGES;
+      int s = stage;
+      uint32_t p = phase;
+      for (int i = 0; i < n; ++i) {
+        if (--s < 0) {
+          s = C::STAGES - 1;
+          p ^= 1u;
+        }
+        mbar_wait_bounded(&full_bar[s], p, drain_deadline);
+      }
+    }
+  } else if (run && warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    bool issued_any = false;
+    for (int tile = blockIdx.x; ok && tile < args.total_tiles; tile += gridDim.x) {
+      if (!warp_wait_bounded(&tempty_bar[acc], acc_phase ^ 1u, deadline)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+      for (int kt = 0; kt < args.num_k_tiles; ++kt) {
+        if (!warp_wait_bounded(&full_bar[stage], phase, deadline)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (elect_one()) {
+          const uint32_t a_addr = smem_u32(smem_a + stage * C::A_BYTES);
+          const uint32_t b_addr = smem_u32(smem_b + stage * C::B_BYTES);
+          if constexpr (FP4) {
+            const uint32_t sfa_addr = smem_u32(smem_sfa + stage * C::SFA_BYTES);
+            const uint32_t sfb_addr = smem_u32(smem_sfb + stage * C::SFB_BYTES);
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb) {
+              tmem_cp_32x128b_x4(tmem_base + C::SFA_COL + kb * 4,
+                                 smem_desc(sfa_addr + kb * kSfAtomBytes, 0, 128, 0));
+#pragma unroll
+              for (int a = 0; a < C::NA; ++a)
+                tmem_cp_32x128b_x4(tmem_base + C::SFB_COL + (kb * C::NA + a) * 4,
+                                   smem_desc(sfb_addr + (kb * C::NA + a) * kSfAtomBytes, 0, 128, 0));
+            }
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb) {
+              mma_nvf4(d_tmem, smem_desc(a_addr + kb * 32, 16, 1024, 2),
+                       smem_desc(b_addr + kb * 32, 16, 1024, 2), C::IDESC,
+                       tmem_base + C::SFA_COL + kb * 4, tmem_base + C::SFB_COL + kb * C::NA * 4,
+                       (kt | kb) != 0 ? 1u : 0u);
+            }
+          } else {
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb) {
+              mma_f8f6f4(d_tmem, smem_desc(a_addr + kb * 32, 16, 1024, 2),
+                         smem_desc(b_addr + kb * 32, 16, 1024, 2), C::IDESC,
+                         (kt | kb) != 0 ? 1u : 0u);
+            }
+          }
+          tc_commit(&empty_bar[stage]);  // frees the stage once these MMAs have read it
+        }
+        __syncwarp();
+        issued_any = true;
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (elect_one()) tc_commit(&tfull_bar[acc]);  // accumulator ready for the epilogue
+      __syncwarp();
+      if (C::NACC == 2) {
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      } else {
+        acc_phase ^= 1u;
+      }
+    }
+    if (!ok) {
+      record_timeout(args.status);
+      *abort_flag = 1;
+      if (issued_any) {  // wait (bounded) for this thread's MMAs and copies to finish
+        if (elect_one()) tc_commit(drain_bar);
+        __syncwarp();
+        mbar_wait_bounded(drain_bar, 0, globaltimer_ns() + 100000000ull);
+      }
+    }
+  } else if (run) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp % 4;  // TMEM lane quadrant this warp may access
+    const int row_in_tile = q * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    float alpha = 1.0f;
+    if constexpr (FP4) alpha = __fmul_rn(__ldg(args.scale_a), __ldg(args.scale_b));
+    const bool vec_ok = (args.N % 8) == 0;
+    for (int tile = blockIdx.x; tile < args.total_tiles; tile += gridDim.x) {
+      const int m_blk = tile % args.tiles_m;
+      const int n_blk = tile / args.tiles_m;
+      if (!warp_wait_bounded(&tfull_bar[acc], acc_phase, deadline)) {
+        record_timeout(args.status);
+        break;
+      }
+      tc_fence_after();
+      const int m = m_blk * kBM + row_in_tile;
+      float row_scale = 1.0f;
+      if constexpr (!FP4) row_scale = (m < args.M) ? __ldg(args.scale_a + m) : 0.0f;
+      uint16_t* yrow = args.y + static_cast<int64_t>(m) * args.N;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        __syncwarp();  // tcgen05.ld is warp-collective
+        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                               static_cast<uint32_t>(acc * BN + c * 32),
+                           r);
+        tmem_ld_wait();
+        if (c == BN / 32 - 1) {  // all columns read: hand the buffer back early
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty_bar[acc]);
+        }
+        const int n0 = n_blk * BN + c * 32;
+        if (m >= args.M || n0 >= args.N) continue;
+        if (vec_ok && n0 + 32 <= args.N) {
+          float sc[32], bi[32];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float4 b4 = args.bias ? __ldg(reinterpret_cast<const float4*>(args.bias + n0) + i)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+            bi[4 * i] = b4.x;
+            bi[4 * i + 1] = b4.y;
+            bi[4 * i + 2] = b4.z;
+            bi[4 * i + 3] = b4.w;
+            if constexpr (FP4) {
+              sc[4 * i] = sc[4 * i + 1] = sc[4 * i + 2] = sc[4 * i + 3] = alpha;
+            } else {
+              const float4 w4 = __ldg(reinterpret_cast<const float4*>(args.scale_b + n0) + i);
+              sc[4 * i] = __fmul_rn(row_scale, w4.x);
+              sc[4 * i + 1] = __fmul_rn(row_scale, w4.y);
+              sc[4 * i + 2] = __fmul_rn(row_scale, w4.z);
+              sc[4 * i + 3] = __fmul_rn(row_scale, w4.w);
+            }
+          }
+          uint32_t packed[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float v0 = __fmaf_rn(__uint_as_float(r[2 * i]), sc[2 * i], bi[2 * i]);
+            const float v1 = __fmaf_rn(__uint_as_float(r[2 * i + 1]), sc[2 * i + 1], bi[2 * i + 1]);
+            packed[i] = pack_bf16(v0, v1);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(yrow + n0);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int n = n0 + i;
+            if (n < args.N) {
+              const float s = FP4 ? alpha : __fmul_rn(row_scale, __ldg(args.scale_b + n));
+              const float b = args.bias ? __ldg(args.bias + n) : 0.0f;
+              const float v = __fmaf_rn(__uint_as_float(r[i]), s, b);
+              const __nv_bfloat16 h = __float2bfloat16_rn(v);
+              yrow[n] = *reinterpret_cast<const uint16_t*>(&h);
+            }
+          }
+        }
+      }
+      if (C::NACC == 2) {
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      } else {
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Row-major uint8 matrix [rows, cols_bytes] viewed in boxes of [box_rows, 128 bytes]
+// with the 128-byte swizzle that the K-major MMA descriptors expect.
+bool make_tmap(CUtensorMap* map, const void* base, int64_t rows, int64_t cols_bytes, int box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols_bytes), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols_bytes)};
+  const cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool FP4, int BN>
+cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
+  using Cf = Cfg<FP4, BN>;
+  auto kern = qgemm_kernel<FP4, BN>;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static bool attr_set[64] = {};
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 64 && !attr_set[dev]) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
+      if (e != cudaSuccess) return e;
+      attr_set[dev] = true;
+    }
+  }
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+
+  const int64_t k_bytes = FP4 ? p.K / 2 : p.K;
+  CUtensorMap ta, tb;
+  if (!make_tmap(&ta, p.a, p.M, k_bytes, kBM) || !make_tmap(&tb, p.b, p.N, k_bytes, BN))
+    return cudaErrorInvalidValue;
+
+  GemmArgs a{};
+  a.M = static_cast<int>(p.M);
+  a.N = static_cast<int>(p.N);
+  a.K = static_cast<int>(p.K);
+  a.tiles_m = static_cast<int>(ceil_div64(p.M, kBM));
+  a.tiles_n = static_cast<int>(ceil_div64(p.N, BN));
+  a.num_k_tiles = static_cast<int>(ceil_div64(p.K, FP4 ? kKTileFp4 : kKTileFp8));
+  a.total_tiles = a.tiles_m * a.tiles_n;
+  a.kg = sf_kgroups(p.K);
+  a.sfa = p.sfa;
+  a.sfb = p.sfb;
+  a.scale_a = p.scale_a;
+  a.scale_b = p.scale_b;
+  a.bias = p.bias;
+  a.y = static_cast<uint16_t*>(p.y);
+  a.status = p.status;
+  a.timeout_ns = p.timeout_ns;
+  a.inject_fault = p.inject_fault;
+  a.wait_prior_grid = p.pdl ? 1 : 0;
+
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(a.total_tiles < sms ? a.total_tiles : sms));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = Cf::SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = p.pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, a);
+}
+
+}  // namespace
+
+int choose_bn(bool fp4, int64_t M, int64_t N) {
+  (void)fp4;
+  (void)M;
+  if (N % 192 == 0 && N >= 1536) return 192;
+  if (N % 256 == 0 && N >= 4096) return 256;
+  return 128;
+}
+
+cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream) {
+  if (p.fp4) {
+    switch (p.bn) {
+      case 128: return launch_typed<true, 128>(p, stream);
+      case 192: return launch_typed<true, 192>(p, stream);
+      case 256: return launch_typed<true, 256>(p, stream);
+    }
+  } else {
+    switch (p.bn) {
+      case 128: return launch_typed<false, 128>(p, stream);
+      case 192: return launch_typed<false, 192>(p, stream);
+      case 256: return launch_typed<false, 256>(p, stream);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace ql

@@ -1,0 +1,44 @@
+// Host-side declarations shared by the translation units of the library.
+#pragma once
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+namespace ql {
+
+constexpr int QL_ERR_TIMEOUT_CODE = 7;  // same value as QL_ERR_TIMEOUT in qlinear.h
+
+// One GEMM launch (both schemes). a, b: row-major codes [M, K*] and [N, K*]
+// (K* = K/2 bytes for FP4, K bytes for FP8).
+struct GemmProblem {
+  bool fp4;
+  int bn;
+  int64_t M, N, K;
+  const void* a;
+  const void* b;
+  const uint8_t* sfa;    // FP4 only: activation scale atoms
+  const uint8_t* sfb;    // FP4 only: weight scale atoms for tile width bn
+  const float* scale_a;  // FP4: input_scale scalar; FP8: x_scale [M]
+  const float* scale_b;  // FP4: weight_scale_2 scalar; FP8: w_scale [N]
+  const float* bias;     // [N] or null
+  void* y;               // bf16 [M, N]
+  int* status;           // device status word
+  uint64_t timeout_ns;
+  int inject_fault;
+  bool pdl;              // launched right after its producer kernel (programmatic dependency)
+};
+
+int choose_bn(bool fp4, int64_t M, int64_t N);
+cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream);
+
+cudaError_t launch_nvfp4_quantize_rowmajor(const void* x, int64_t M, int64_t K, const float* g,
+                                           uint8_t* xq, uint8_t* xs, cudaStream_t s);
+cudaError_t launch_nvfp4_prologue(const void* x, int64_t M, int64_t K, const uint8_t* w_scale,
+                                  int64_t N, int bn, const float* input_scale, uint8_t* workspace,
+                                  cudaStream_t s);
+cudaError_t launch_fp8r_quantize_rows(const void* x, int64_t M, int64_t K, uint8_t* xq,
+                                      float* x_scale, cudaStream_t s);
+cudaError_t launch_global_scale(const void* x, int64_t n, float* out, cudaStream_t s);
+cudaError_t launch_encode(const float* in, uint8_t* out, int64_t n, bool fp4, cudaStream_t s);
+
+}  // namespace ql

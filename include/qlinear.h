@@ -1,0 +1,195 @@
+/*
+ * qlinear.h - C ABI of the B200 (sm_100a) NVFP4 / FP8-rowwise quantized linear.
+ *
+ * The operation (Diffusers documentation "BFL (fp8r / nvfp4)"):
+ *   - scheme list, `nvfp4` entry: a quantized linear stores a packed E2M1
+ *     `weight` (two values per byte), one E4M3 block scale per 16 elements
+ *     (`weight_scale`), a global fp32 `weight_scale_2` and a calibrated fp32
+ *     activation scale `input_scale`;
+ *   - scheme list, `fp8r` entry: an E4M3 `weight` with one fp32 `weight_scale`
+ *     per row; activations are quantized per row to E4M3 at run time;
+ *   - section "Kernels", table: nvfp4 quantizes the activations at run time and
+ *     runs a block-scaled FP4 GEMM; fp8r runs a GEMM with row-wise scales.
+ * Element formats are the OCP ones: E4M3 "FN" (bias 7, max 448, no inf) and
+ * E2M1 (magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6).
+ *
+ * Arithmetic (the stated reading; the pages print no formula):
+ *   NVFP4 quantize of a bf16 row with global scale g, per 16-element block:
+ *     c = RN32(1 / RN32(6 g)) (once per tensor); s = E4M3(RN32(amax * c));
+ *     d = RN32(decode(s) * g); codes = E2M1(RN32(x * RN32(1/d))), or 0 if d == 0.
+ *     Element 2j in bits 3..0 of byte j, element 2j+1 in bits 7..4.
+ *   NVFP4 linear: Y = bf16( input_scale * weight_scale_2 *
+ *                          sum_k (E2M1(xq) E4M3(xs)) (E2M1(wq) E4M3(ws)) + bias ).
+ *   fp8r quantize of a row: scale = RN32(amax / 448); codes = E4M3(RN32(x * RN32(1/scale))),
+ *     or 0 if scale == 0.
+ *   fp8r linear: Y = bf16( x_scale[m] * w_scale[n] * sum_k E4M3(xq) E4M3(wq) + bias ).
+ *   E4M3 / E2M1 encoding: round to nearest, ties to even, saturating to the
+ *   largest finite value, sign kept.
+ *
+ * Conventions for every entry point:
+ *   - Tensors are row-major and densely packed (leading dimension = row length).
+ *   - All tensor and scale pointers are DEVICE pointers (current device), except
+ *     where a function says otherwise. Scalar scales are device pointers so that
+ *     no host synchronisation is needed and calls can be captured in graphs.
+ *   - Base pointers must be 16-byte aligned (QL_ERR_ALIGN otherwise).
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Calls are
+ *     asynchronous on it; nothing synchronises the host.
+ *   - The caller owns every buffer, including workspaces. The library never
+ *     allocates or frees device memory and keeps no per-call state.
+ *   - Return value: QL_OK (0) or an error code below; errors found on the host
+ *     leave all outputs untouched. QL_ERR_LAUNCH keeps the CUDA error text,
+ *     readable through ql_last_error_message().
+ *   - Only sm_100 devices (B200 class) are accepted (QL_ERR_DEVICE otherwise).
+ *   - NaN or infinite inputs give unspecified codes (never a fault).
+ */
+#ifndef QLINEAR_H
+#define QLINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* ql_stream_t; /* a cudaStream_t */
+
+enum {
+  QL_OK = 0,
+  QL_ERR_INVALID_ARG = 1, /* null pointer, non-positive size */
+  QL_ERR_SHAPE = 2,       /* size constraint violated (see each function) */
+  QL_ERR_ALIGN = 3,       /* a base pointer is not 16-byte aligned */
+  QL_ERR_DEVICE = 4,      /* current device is not sm_100 */
+  QL_ERR_WORKSPACE = 5,   /* workspace missing or smaller than required */
+  QL_ERR_LAUNCH = 6,      /* a CUDA call failed; see ql_last_error_message() */
+  QL_ERR_TIMEOUT = 7      /* a kernel's bounded wait expired (device status word) */
+};
+
+/* ------------------------------------------------------------------------ */
+/* NVFP4                                                                     */
+/* ------------------------------------------------------------------------ */
+
+/* Run-time NVFP4 quantization of activations ("BFL (fp8r / nvfp4)", "Kernels"
+ * table: nvfp4_quantize for activations). The same routine quantizes a weight
+ * offline when given weight_scale_2 as the global scale.
+ *   x           bf16 [M, K]
+ *   input_scale fp32 scalar (device): the calibrated global scale g
+ *   xq          uint8 [M, K/2]  packed E2M1 codes (output)
+ *   xs          uint8 [M, K/16] E4M3 block-scale codes (output)
+ * Requires M >= 1, K >= 16, K % 16 == 0. */
+int nvfp4_quantize_act(const void* x, int64_t M, int64_t K, const float* input_scale,
+                       uint8_t* xq, uint8_t* xs, ql_stream_t stream);
+
+/* Bytes of workspace nvfp4_linear needs for this problem size (0 on bad sizes). */
+size_t nvfp4_linear_workspace_size(int64_t M, int64_t K, int64_t N);
+
+/* NVFP4 W4A4 linear forward: quantizes x at run time with input_scale and
+ * contracts it on the tensor cores against the pre-quantized weight.
+ *   x              bf16 [M, K]
+ *   w              uint8 [N, K/2]  packed E2M1 weight codes
+ *   w_scale        uint8 [N, K/16] E4M3 weight block scales (row-major, as stored
+ *                  in the checkpoint; any hardware layout is produced internally)
+ *   weight_scale_2 fp32 scalar (device)
+ *   input_scale    fp32 scalar (device)
+ *   bias           fp32 [N] or NULL
+ *   y              bf16 [M, N] (output)
+ *   workspace      device buffer of >= nvfp4_linear_workspace_size(M, K, N) bytes;
+ *                  holds the quantized activations and the scale layouts between
+ *                  the two kernels of one call (its contents are internal)
+ * Requires M, N >= 1, K >= 32, K % 32 == 0 (16-byte aligned packed rows). */
+int nvfp4_linear(const void* x, int64_t M, int64_t K,
+                 const uint8_t* w, const uint8_t* w_scale, int64_t N,
+                 const float* weight_scale_2, const float* input_scale,
+                 const float* bias, void* y,
+                 void* workspace, size_t workspace_bytes, ql_stream_t stream);
+
+/* The two halves of nvfp4_linear, for callers that time or schedule them apart.
+ * nvfp4_linear == nvfp4_linear_prologue followed by nvfp4_linear_gemm on the same
+ * stream and workspace. The prologue quantizes x into the workspace and lays out
+ * both scale tensors for the tensor cores; the GEMM reads only the workspace,
+ * w, the scalars and bias. Same argument meaning and requirements as above. */
+int nvfp4_linear_prologue(const void* x, int64_t M, int64_t K,
+                          const uint8_t* w_scale, int64_t N, const float* input_scale,
+                          void* workspace, size_t workspace_bytes, ql_stream_t stream);
+int nvfp4_linear_gemm(int64_t M, int64_t K, const uint8_t* w, int64_t N,
+                      const float* weight_scale_2, const float* input_scale,
+                      const float* bias, void* y,
+                      const void* workspace, size_t workspace_bytes, ql_stream_t stream);
+
+/* Offsets (bytes from the workspace base) of the quantized activations inside an
+ * nvfp4_linear workspace, for diagnostics: codes are row-major uint8 [M, K/2] at
+ * *codes_offset. Returns QL_OK or QL_ERR_SHAPE. */
+int nvfp4_linear_workspace_layout(int64_t M, int64_t K, int64_t N, size_t* codes_offset,
+                                  size_t* act_scales_offset, size_t* weight_scales_offset);
+
+/* Calibration rule used by the workloads: out = RN32(amax(|x|) / (6 * 448)),
+ * the global scale that maps the largest magnitude onto E2M1 6 times E4M3 448.
+ *   x bf16 [n]; out fp32 scalar (device, overwritten). Requires n >= 1. */
+int nvfp4_global_scale(const void* x, int64_t n, float* out, ql_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* fp8r (FP8 row-wise)                                                       */
+/* ------------------------------------------------------------------------ */
+
+/* Per-row E4M3 quantization ("BFL (fp8r / nvfp4)", scheme list, fp8r entry).
+ * Quantizes weights (rows = output channels) and activations (rows = tokens).
+ *   x       bf16 [M, K]
+ *   xq      uint8 [M, K] E4M3 codes (output)
+ *   x_scale fp32 [M] row scales (output)
+ * Requires M >= 1, K >= 8, K % 8 == 0. */
+int fp8r_quantize_rows(const void* x, int64_t M, int64_t K, uint8_t* xq, float* x_scale,
+                       ql_stream_t stream);
+
+/* Bytes of workspace fp8r_linear needs (0 on bad sizes). */
+size_t fp8r_linear_workspace_size(int64_t M, int64_t K, int64_t N);
+
+/* fp8r linear forward: quantizes x per row at run time and runs the E4M3 GEMM with
+ * the row-wise scales ("Kernels" table: a scaled GEMM with row-wise scales).
+ *   x       bf16 [M, K]
+ *   w       uint8 [N, K] E4M3 weight codes
+ *   w_scale fp32 [N] per-row weight scales
+ *   bias    fp32 [N] or NULL
+ *   y       bf16 [M, N] (output)
+ *   workspace >= fp8r_linear_workspace_size(M, K, N) bytes
+ * Requires M, N >= 1, K >= 16, K % 16 == 0. */
+int fp8r_linear(const void* x, int64_t M, int64_t K,
+                const uint8_t* w, const float* w_scale, int64_t N,
+                const float* bias, void* y,
+                void* workspace, size_t workspace_bytes, ql_stream_t stream);
+
+/* The GEMM half of fp8r_linear, from activations already quantized by
+ * fp8r_quantize_rows: xq uint8 [M, K], x_scale fp32 [M]. */
+int fp8r_linear_gemm(const uint8_t* xq, const float* x_scale, int64_t M, int64_t K,
+                     const uint8_t* w, const float* w_scale, int64_t N,
+                     const float* bias, void* y, ql_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Diagnostics and status                                                    */
+/* ------------------------------------------------------------------------ */
+
+/* The hardware element encoders used by the kernels, on an fp32 array:
+ * out[i] = E4M3 code of in[i] (one byte each), or the E2M1 code (low nibble of
+ * each byte). in and out are device pointers; n >= 1. */
+int ql_encode_e4m3(const float* in, uint8_t* out, int64_t n, ql_stream_t stream);
+int ql_encode_e2m1(const float* in, uint8_t* out, int64_t n, ql_stream_t stream);
+
+/* Device status word of the current device: kernels whose bounded waits expire
+ * write QL_ERR_TIMEOUT there (they never hang). Reading synchronises the device.
+ * ql_read_device_status stores the word in *status (host pointer) and clears it. */
+int ql_read_device_status(int* status);
+
+/* Test hook: while set (nonzero), the next GEMM launches start with one wait on a
+ * barrier that nothing completes, so the bounded-wait path runs and reports
+ * QL_ERR_TIMEOUT through the status word. `timeout_ms` bounds every wait of the
+ * GEMM kernels (default 2000 ms; 0 restores the default). Host-side settings. */
+void ql_set_fault_injection(int enable, int timeout_ms);
+
+/* Text of a status code, and of the last CUDA error recorded by this thread. */
+const char* ql_status_string(int status);
+const char* ql_last_error_message(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLINEAR_H */

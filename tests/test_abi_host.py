@@ -1,0 +1,92 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every
+function include/qlinear.h declares, sizes its workspaces, and rejects bad
+arguments with the documented status codes before touching the device."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from fp8_rowwise_quantized_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qlinear.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s+\*?([a-z][a-z0-9_]+)\s*\(",
+                       text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib.load()
+    names = declared_functions()
+    assert len(names) >= 17, names
+    for n in names:
+        assert hasattr(lib, n), f"missing export {n}"
+    assert set(names) == set(_lib.SIGNATURES), set(names) ^ set(_lib.SIGNATURES)
+
+
+def test_status_strings():
+    lib = _lib.load()
+    for code in range(8):
+        s = lib.ql_status_string(code).decode()
+        assert s and s != "unknown status"
+    assert lib.ql_status_string(99).decode() == "unknown status"
+
+
+def test_workspace_sizes():
+    lib = _lib.load()
+    M, K, N = 4096, 3072, 12288
+    ws = lib.nvfp4_linear_workspace_size(M, K, N)
+    # codes M*K/2 + activation scale atoms + weight scale atoms (padded), 1 KB aligned
+    assert ws >= M * K // 2 + M * K // 16 + N * K // 16
+    assert ws < M * K // 2 + 2 * (M * K // 16) + 2 * (N * K // 16) + 8192
+    assert ws % 1024 == 0
+    assert lib.nvfp4_linear_workspace_size(M, 48, N) == 0       # K % 32 != 0
+    assert lib.nvfp4_linear_workspace_size(0, K, N) == 0
+    assert lib.fp8r_linear_workspace_size(4096, 3072, 3072) >= 4096 * 3072 + 4096 * 4
+    assert lib.fp8r_linear_workspace_size(4096, 3000, 3072) == 0  # K % 16 != 0
+    a, b, c = C.c_size_t(), C.c_size_t(), C.c_size_t()
+    assert lib.nvfp4_linear_workspace_layout(M, K, N, C.byref(a), C.byref(b), C.byref(c)) == 0
+    assert a.value == 0 and b.value >= M * K // 2 and c.value > b.value and c.value < ws
+
+
+def test_argument_errors_before_device():
+    lib = _lib.load()
+    fake = 1 << 20          # aligned, never dereferenced: validation fails first
+    odd = fake + 8          # not 16-byte aligned
+    M, K, N = 128, 256, 256
+    ws = lib.nvfp4_linear_workspace_size(M, K, N)
+    # null pointer
+    assert lib.nvfp4_linear(None, M, K, fake, fake, N, fake, fake, None, fake, fake, ws, None) == 1
+    # non-positive size
+    assert lib.nvfp4_linear(fake, 0, K, fake, fake, N, fake, fake, None, fake, fake, ws, None) == 1
+    # K not a multiple of 32
+    assert lib.nvfp4_linear(fake, M, 48, fake, fake, N, fake, fake, None, fake, fake, ws, None) == 2
+    # misaligned output
+    assert lib.nvfp4_linear(fake, M, K, fake, fake, N, fake, fake, None, odd, fake, ws, None) == 3
+    # workspace too small / missing
+    assert lib.nvfp4_linear(fake, M, K, fake, fake, N, fake, fake, None, fake, fake, ws - 1, None) == 5
+    assert lib.nvfp4_linear(fake, M, K, fake, fake, N, fake, fake, None, fake, None, ws, None) == 5
+    assert lib.fp8r_linear(fake, M, 40, fake, fake, N, None, fake, fake, 1 << 30, None) == 2
+    assert lib.fp8r_quantize_rows(fake, M, 12, fake, fake, None) == 2
+    assert lib.nvfp4_quantize_act(fake, M, 24, fake, fake, fake, None) == 2
+    assert lib.nvfp4_quantize_act(odd, M, K, fake, fake, fake, None) == 3
+    assert lib.ql_encode_e4m3(None, fake, 10, None) == 1
+
+
+def test_no_device_reports_error_instead_of_crashing():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    lib = _lib.load()
+    fake = 1 << 20
+    rc = lib.nvfp4_quantize_act(fake, 128, 256, fake, fake, fake, None)
+    assert rc in (4, 6)           # device check or CUDA error, never a crash
+    assert lib.ql_last_error_message().decode()
+    st = C.c_int(-1)
+    assert lib.ql_read_device_status(C.byref(st)) in (4, 6)

@@ -1,0 +1,139 @@
+"""GPU parity of the NVFP4 and fp8r linear layers (tensor-core GEMMs) against the
+fp64 oracle, through the C ABI. Small shapes are compared element by element in
+full (several tiles plus ragged tails in M, N and K; every tile width); the
+full diffusion-transformer sizes are compared on sampled rows, with properties
+that hold at any size checked on the whole output."""
+import numpy as np
+import pytest
+import torch
+
+import fp8_rowwise_quantized_b200 as q
+import oracle
+from gpu_helpers import (Fp8rCase, Nvfp4Case, bf16_bits, check_linear, sample_rows, scalar_dev,
+                         to_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+def nan_output(M, N):
+    # every element must be written: start from NaN and require all finite after
+    return torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+
+
+def run_nvfp4(c: Nvfp4Case, rows=None, workspace=None):
+    d = c.device_args()
+    y = q.nvfp4_linear(d["x"], d["w"], d["w_scale"], d["weight_scale_2"], d["input_scale"],
+                       bias=d["bias"], y=nan_output(c.M, c.N), workspace=workspace)
+    torch.cuda.synchronize()
+    assert bool(torch.isfinite(y).all()), "unwritten or non-finite outputs"
+    y_ref, y64, T = c.reference(rows)
+    yc = y if rows is None else y[torch.from_numpy(rows).cuda()]
+    return y, check_linear(yc, y64, T, f"nvfp4 {c.M}x{c.K}x{c.N}")
+
+
+@pytest.mark.parametrize("M,K,N", [
+    (128, 256, 256),     # the tiny layer: 2 N tiles
+    (1, 32, 8),          # smallest K, one row, narrow N
+    (17, 96, 136),       # ragged everything; K not a multiple of 256
+    (200, 288, 392),     # two M tiles, partial K tile
+    (256, 512, 384),     # tile width 128, three N tiles
+    (130, 1024, 1536),   # tile width 192
+    (300, 768, 4096),    # tile width 256 (single TMEM accumulator)
+    (64, 3072, 200),     # N not a multiple of 8 -> scalar tail stores
+])
+def test_nvfp4_linear_small_full(M, K, N):
+    run_nvfp4(Nvfp4Case(M, K, N, seed=M + N))
+
+
+def test_nvfp4_linear_tiny_with_bias_and_saturation():
+    run_nvfp4(Nvfp4Case(128, 256, 256, seed=0, bias=True))
+    run_nvfp4(Nvfp4Case(128, 256, 256, seed=1, input_scale_div=4.0))
+
+
+@pytest.mark.parametrize("name,M,K,N,bias", [
+    ("attn_proj", 4096, 3072, 3072, True),
+    ("attn_qkv", 4096, 3072, 9216, True),
+    ("mlp_up", 4096, 3072, 12288, False),
+])
+def test_nvfp4_linear_dit_sizes_sampled(name, M, K, N, bias):
+    c = Nvfp4Case(M, K, N, seed=0, bias=bias)
+    rows = sample_rows(M, 20, seed=1)
+    y, frob = run_nvfp4(c, rows)
+    # whole output: written (finite, checked in run_nvfp4), of the expected
+    # magnitude and nonzero almost everywhere (the sampled rows carry the exact check)
+    yb = oracle.bf16_bits_to_f64(bf16_bits(y))
+    assert np.abs(yb).max() < 1e4 and (yb != 0).mean() > 0.99
+
+
+def test_nvfp4_mlp_down_from_gelu_of_up():
+    # the down projection's input is GELU of the up projection's GPU output,
+    # re-quantized at run time with a re-calibrated input scale
+    up = Nvfp4Case(4096, 3072, 12288, seed=0)
+    d = up.device_args()
+    y_up = q.nvfp4_linear(d["x"], d["w"], d["w_scale"], d["weight_scale_2"], d["input_scale"])
+    h = torch.nn.functional.gelu(y_up.float()).to(torch.bfloat16).cpu()
+    down = Nvfp4Case(4096, 12288, 3072, seed=1, x=h)
+    run_nvfp4(down, sample_rows(4096, 20, seed=2))
+
+
+def test_nvfp4_linear_split_calls_match_fused():
+    c = Nvfp4Case(512, 3072, 3072, seed=5, bias=True)
+    d = c.device_args()
+    ws = torch.empty(q.nvfp4_linear_workspace_size(512, 3072, 3072), dtype=torch.uint8,
+                     device="cuda")
+    y1 = q.nvfp4_linear(d["x"], d["w"], d["w_scale"], d["weight_scale_2"], d["input_scale"],
+                        bias=d["bias"], workspace=ws)
+    q.nvfp4_linear_prologue(d["x"], d["w_scale"], d["input_scale"], ws)
+    y2 = q.nvfp4_linear_gemm(512, d["w"], d["weight_scale_2"], d["input_scale"], ws,
+                             bias=d["bias"])
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)  # same kernels, same order: bit-identical
+
+
+def test_nvfp4_linear_repeatable():
+    c = Nvfp4Case(1024, 3072, 3072, seed=6)
+    d = c.device_args()
+    ys = [q.nvfp4_linear(d["x"], d["w"], d["w_scale"], d["weight_scale_2"], d["input_scale"])
+          for _ in range(3)]
+    torch.cuda.synchronize()
+    assert torch.equal(ys[0], ys[1]) and torch.equal(ys[1], ys[2])
+
+
+def run_fp8r(c: Fp8rCase, rows=None):
+    d = c.device_args()
+    y = q.fp8r_linear(d["x"], d["w"], d["w_scale"], bias=d["bias"], y=nan_output(c.M, c.N))
+    torch.cuda.synchronize()
+    assert bool(torch.isfinite(y).all()), "unwritten or non-finite outputs"
+    y_ref, y64, T = c.reference(rows)
+    yc = y if rows is None else y[torch.from_numpy(rows).cuda()]
+    return y, check_linear(yc, y64, T, f"fp8r {c.M}x{c.K}x{c.N}")
+
+
+@pytest.mark.parametrize("M,K,N,bias", [
+    (128, 256, 256, False),
+    (1, 16, 8, True),
+    (77, 208, 136, True),
+    (200, 400, 392, False),
+    (130, 1024, 1536, True),
+    (300, 768, 4096, False),
+    (64, 512, 200, False),
+])
+def test_fp8r_linear_small_full(M, K, N, bias):
+    run_fp8r(Fp8rCase(M, K, N, seed=M + K, bias=bias))
+
+
+def test_fp8r_linear_4096x3072x3072_sampled():
+    c = Fp8rCase(4096, 3072, 3072, seed=0)
+    y, _ = run_fp8r(c, sample_rows(4096, 24, seed=3))
+    yb = oracle.bf16_bits_to_f64(bf16_bits(y))
+    assert (yb != 0).mean() > 0.99
+
+
+def test_fp8r_gemm_from_prequantized_matches_linear():
+    c = Fp8rCase(256, 3072, 3072, seed=4, bias=True)
+    d = c.device_args()
+    y1 = q.fp8r_linear(d["x"], d["w"], d["w_scale"], bias=d["bias"])
+    xq, xs = q.fp8r_quantize_rows(d["x"])
+    y2 = q.fp8r_linear_gemm(xq, xs, d["w"], d["w_scale"], bias=d["bias"])
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
