@@ -484,6 +484,31 @@ def run_ours(args):
     return 0
 
 
+def run_profile(args):
+    """Short fixed sequence for profilers: `--profile <piece>` runs `--steps` calls
+    of one piece of the headline workload (no flushes, no timing): `step`,
+    `prologue`, `gemm`, `fp8r_step`, `fp8r_quant` or `fp8r_gemm`."""
+    import torch
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    M, K, N = WORKLOAD["M"], WORKLOAD["K"], WORKLOAD["N"]
+    if args.profile.startswith("fp8r"):
+        L = Fp8rLayer(4096, 3072, 3072, False, device)
+        fn = {"fp8r_step": L.step, "fp8r_gemm": L.gemm,
+              "fp8r_quant": lambda: L.q.fp8r_quantize_rows(L.x, L.xq, L.xs)}[args.profile]
+    else:
+        L = Nvfp4Layer(M, K, N, False, device)
+        L.prologue()
+        fn = {"step": L.step, "prologue": L.prologue, "gemm": L.gemm}[args.profile]
+    for _ in range(args.steps):
+        fn()
+    torch.cuda.synchronize()
+    import fp8_rowwise_quantized_b200 as q
+    assert q.read_device_status() == 0
+    print(json.dumps({"profile": args.profile, "steps": args.steps, "ok": True}))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -493,8 +518,13 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-variants", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=["step", "prologue", "gemm", "fp8r_step", "fp8r_quant",
+                                          "fp8r_gemm"], default=None,
+                    help="run a short fixed sequence for a profiler instead of the benchmark")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    if args.profile:
+        return run_profile(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -38,6 +38,7 @@ constexpr int kBM = 128;
 constexpr int kThreads = 192;
 constexpr int kSmemLimit = 232448;  // 227 KB opt-in per block
 constexpr int kTmemCols = 512;
+constexpr int kEpiBufBytes = 32 * 128;  // 32 rows x 64 bf16 (128-byte swizzled), one TMA box
 
 struct GemmArgs {
   int M, N, K;
@@ -53,6 +54,7 @@ struct GemmArgs {
   uint64_t timeout_ns;
   int inject_fault;
   int wait_prior_grid;
+  int use_tma_store;        // Y written through shared memory + TMA (needs N % 8 == 0)
 };
 
 template <bool FP4, int BN>
@@ -63,13 +65,15 @@ struct Cfg {
   static constexpr int SFA_BYTES = FP4 ? 4 * kSfAtomBytes : 0;      // 4 K-groups x 1 atom
   static constexpr int SFB_BYTES = FP4 ? 4 * NA * kSfAtomBytes : 0; // 4 K-groups x NA atoms
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  static constexpr int RESERVED = 1024 /*alignment*/ + 1024 /*barriers*/;
+  static constexpr int EPI_BYTES = 4 * 2 * kEpiBufBytes;            // 4 warps x 2 staging buffers
+  static constexpr int RESERVED = 1024 /*alignment*/ + 1024 /*barriers*/ + EPI_BYTES;
   static constexpr int STAGES_FIT = (kSmemLimit - RESERVED) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
   static constexpr int NACC = (2 * BN + 16 + 4 * NA * 4 <= kTmemCols) ? 2 : 1;
   static constexpr int SFA_COL = NACC * BN;
   static constexpr int SFB_COL = SFA_COL + 16;
   static constexpr int SMEM = RESERVED + STAGES * STAGE_BYTES;
+  static_assert(BN % 64 == 0, "epilogue works in 64-column slabs");
   // instruction descriptor: M = 128, N = BN, K-major A and B, fp32 accumulate;
   // FP4: E2M1 x E2M1 with UE4M3 scales; FP8: E4M3 x E4M3.
   static constexpr uint32_t IDESC =
@@ -77,7 +81,7 @@ struct Cfg {
           : ((1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(kBM >> 4) << 24));
   static_assert(STAGES >= 2, "shared memory too small for two stages");
   static_assert(SFB_COL + 4 * NA * 4 <= kTmemCols, "TMEM budget");
-  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "tile width");
+  static_assert(BN >= 64 && BN <= 256, "tile width");
 };
 
 __device__ __forceinline__ void record_timeout(int* status) {
@@ -92,7 +96,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 template <bool FP4, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-             const GemmArgs args) {
+             const __grid_constant__ CUtensorMap tmap_y, const GemmArgs args) {
   using C = Cfg<FP4, BN>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -101,7 +105,8 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
   uint8_t* smem_b = smem_a + C::STAGES * C::A_BYTES;
   uint8_t* smem_sfa = smem_b + C::STAGES * C::B_BYTES;
   uint8_t* smem_sfb = smem_sfa + C::STAGES * C::SFA_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_sfb + C::STAGES * C::SFB_BYTES);
+  uint8_t* smem_epi = smem_sfb + C::STAGES * C::SFB_BYTES;  // 1024-aligned
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_epi + C::EPI_BYTES);
   uint64_t* full_bar = bars;
   uint64_t* empty_bar = bars + C::STAGES;
   uint64_t* tfull_bar = bars + 2 * C::STAGES;
@@ -118,6 +123,7 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
   if (threadIdx.x == 0) {
     prefetch_tmap(&tmap_a);
     prefetch_tmap(&tmap_b);
+    if (args.use_tma_store) prefetch_tmap(&tmap_y);
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
@@ -288,11 +294,12 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     // ------------------------------------------------------------ epilogue
     const int q = warp % 4;  // TMEM lane quadrant this warp may access
     const int row_in_tile = q * 32 + lane;
+    uint8_t* stage = smem_epi + (warp - 2) * 2 * kEpiBufBytes;
+    int buf = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     float alpha = 1.0f;
     if constexpr (FP4) alpha = __fmul_rn(__ldg(args.scale_a), __ldg(args.scale_b));
-    const bool vec_ok = (args.N % 8) == 0;
     for (int tile = blockIdx.x; tile < args.total_tiles; tile += gridDim.x) {
       const int m_blk = tile % args.tiles_m;
       const int n_blk = tile / args.tiles_m;
@@ -304,62 +311,68 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
       const int m = m_blk * kBM + row_in_tile;
       float row_scale = 1.0f;
       if constexpr (!FP4) row_scale = (m < args.M) ? __ldg(args.scale_a + m) : 0.0f;
-      uint16_t* yrow = args.y + static_cast<int64_t>(m) * args.N;
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(acc * BN);
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
+      for (int sl = 0; sl < BN / 64; ++sl) {
+        uint32_t r[64];
         __syncwarp();  // tcgen05.ld is warp-collective
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                               static_cast<uint32_t>(acc * BN + c * 32),
-                           r);
+        tmem_ld_32x32b_x32(tbase + sl * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld_32x32b_x32(tbase + sl * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
         tmem_ld_wait();
-        if (c == BN / 32 - 1) {  // all columns read: hand the buffer back early
+        if (sl == BN / 64 - 1) {  // all columns read: hand the buffer back early
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&tempty_bar[acc]);
         }
-        const int n0 = n_blk * BN + c * 32;
-        if (m >= args.M || n0 >= args.N) continue;
-        if (vec_ok && n0 + 32 <= args.N) {
-          float sc[32], bi[32];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            float4 b4 = args.bias ? __ldg(reinterpret_cast<const float4*>(args.bias + n0) + i)
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-            bi[4 * i] = b4.x;
-            bi[4 * i + 1] = b4.y;
-            bi[4 * i + 2] = b4.z;
-            bi[4 * i + 3] = b4.w;
-            if constexpr (FP4) {
-              sc[4 * i] = sc[4 * i + 1] = sc[4 * i + 2] = sc[4 * i + 3] = alpha;
-            } else {
-              const float4 w4 = __ldg(reinterpret_cast<const float4*>(args.scale_b + n0) + i);
-              sc[4 * i] = __fmul_rn(row_scale, w4.x);
-              sc[4 * i + 1] = __fmul_rn(row_scale, w4.y);
-              sc[4 * i + 2] = __fmul_rn(row_scale, w4.z);
-              sc[4 * i + 3] = __fmul_rn(row_scale, w4.w);
-            }
-          }
-          uint32_t packed[16];
+        const int n0 = n_blk * BN + sl * 64;
+        if (n0 >= args.N) continue;  // warp-uniform
+        if (args.use_tma_store) {
+          // columns n0 .. n0+63 of rows m_blk*128 + 32q .. +31: scale, bias, bf16,
+          // into a 128-byte-swizzled staging tile, then one TMA store per warp.
+          uint32_t packed[32];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float v0 = __fmaf_rn(__uint_as_float(r[2 * i]), sc[2 * i], bi[2 * i]);
-            const float v1 = __fmaf_rn(__uint_as_float(r[2 * i + 1]), sc[2 * i + 1], bi[2 * i + 1]);
-            packed[i] = pack_bf16(v0, v1);
+            const int n = n0 + 4 * i;
+            const bool in = n < args.N;  // N % 8 == 0: a float4 is all in or all out
+            const float4 b4 = (args.bias && in) ? __ldg(reinterpret_cast<const float4*>(args.bias + n))
+                                                : make_float4(0.f, 0.f, 0.f, 0.f);
+            float4 s4 = make_float4(alpha, alpha, alpha, alpha);
+            if constexpr (!FP4) {
+              const float4 w4 = in ? __ldg(reinterpret_cast<const float4*>(args.scale_b + n))
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+              s4 = make_float4(__fmul_rn(row_scale, w4.x), __fmul_rn(row_scale, w4.y),
+                               __fmul_rn(row_scale, w4.z), __fmul_rn(row_scale, w4.w));
+            }
+            packed[2 * i] = pack_bf16(__fmaf_rn(__uint_as_float(r[4 * i]), s4.x, b4.x),
+                                      __fmaf_rn(__uint_as_float(r[4 * i + 1]), s4.y, b4.y));
+            packed[2 * i + 1] = pack_bf16(__fmaf_rn(__uint_as_float(r[4 * i + 2]), s4.z, b4.z),
+                                          __fmaf_rn(__uint_as_float(r[4 * i + 3]), s4.w, b4.w));
           }
-          uint4* dst = reinterpret_cast<uint4*>(yrow + n0);
+          uint8_t* sbuf = stage + buf * kEpiBufBytes;
+          if (lane == 0) bulk_wait_group_read<1>();  // the store that used this buffer has read it
+          __syncwarp();
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(sbuf + lane * 128 + ((j ^ (lane & 7)) * 16)) =
+                make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+          fence_proxy_async_shared();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmap_y, sbuf, n0, m_blk * kBM + q * 32);
+            bulk_commit_group();
+          }
+          buf ^= 1;
         } else {
+          if (m >= args.M) continue;
+          uint16_t* yrow = args.y + static_cast<int64_t>(m) * args.N;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
+          for (int i = 0; i < 64; ++i) {
             const int n = n0 + i;
             if (n < args.N) {
-              const float s = FP4 ? alpha : __fmul_rn(row_scale, __ldg(args.scale_b + n));
+              const float sc = FP4 ? alpha : __fmul_rn(row_scale, __ldg(args.scale_b + n));
               const float b = args.bias ? __ldg(args.bias + n) : 0.0f;
-              const float v = __fmaf_rn(__uint_as_float(r[i]), s, b);
-              const __nv_bfloat16 h = __float2bfloat16_rn(v);
+              const __nv_bfloat16 h = __float2bfloat16_rn(__fmaf_rn(__uint_as_float(r[i]), sc, b));
               yrow[n] = *reinterpret_cast<const uint16_t*>(&h);
             }
           }
@@ -372,6 +385,7 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
         acc_phase ^= 1u;
       }
     }
+    if (lane == 0) bulk_wait_group_all();  // outstanding stores complete before exit
   }
 
   // ------------------------------------------------------------ teardown
@@ -419,6 +433,20 @@ bool make_tmap(CUtensorMap* map, const void* base, int64_t rows, int64_t cols_by
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 row-major [rows, cols] in boxes of [32 rows, 64 columns] with the 128-byte
+// swizzle of the epilogue's staging tiles.
+bool make_tmap_y(CUtensorMap* map, void* base, int64_t rows, int64_t cols) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols * 2)};
+  const cuuint32_t box[2] = {64u, 32u};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <bool FP4, int BN>
 cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
   using Cf = Cfg<FP4, BN>;
@@ -440,9 +468,12 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
 
   const int64_t k_bytes = FP4 ? p.K / 2 : p.K;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, ty;
   if (!make_tmap(&ta, p.a, p.M, k_bytes, kBM) || !make_tmap(&tb, p.b, p.N, k_bytes, BN))
     return cudaErrorInvalidValue;
+  const bool tma_store = (p.N % 8) == 0 && (reinterpret_cast<uintptr_t>(p.y) & 15) == 0;
+  std::memset(&ty, 0, sizeof(ty));
+  if (tma_store && !make_tmap_y(&ty, p.y, p.M, p.N)) return cudaErrorInvalidValue;
 
   GemmArgs a{};
   a.M = static_cast<int>(p.M);
@@ -463,6 +494,7 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
   a.timeout_ns = p.timeout_ns;
   a.inject_fault = p.inject_fault;
   a.wait_prior_grid = p.pdl ? 1 : 0;
+  a.use_tma_store = tma_store ? 1 : 0;
 
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(a.total_tiles < sms ? a.total_tiles : sms));
@@ -474,7 +506,7 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = p.pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kern, ta, tb, a);
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, ty, a);
 }
 
 }  // namespace

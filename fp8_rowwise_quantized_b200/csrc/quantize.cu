@@ -61,63 +61,80 @@ __device__ __forceinline__ void nvfp4_block(const uint32_t (&w)[8], float c, flo
   *hi = cvt_e2m1x8(b);
 }
 
-// One thread per (row r, 64-element group kg): up to 4 blocks of 16.
+// One warp per (row r, 1024-element segment of K): four 256-element slices, each
+// loaded as one fully coalesced 512-byte warp access (lane l holds elements
+// 8l..8l+7 of the slice). A 16-element block is held by a lane pair; its amax is
+// combined with one shuffle. Each lane writes its 8 codes as one 32-bit word
+// (128 contiguous bytes per warp and slice); lanes 0, 8, 16, 24 gather the four
+// block scales of one 64-element group and write them as one 32-bit word.
 //   x  bf16 [M, K]; xq uint8 [M, K/2]
-//   SF_MMA == false: xs uint8 [M, K/16] row-major
-//   SF_MMA == true:  xs in the atom layout for rows padded to 128 and K groups
-//                    padded to whole K tiles (padding written as zero)
+//   SF_MMA == false: xs uint8 [M, K/16] row-major (only blocks inside K)
+//   SF_MMA == true:  xs in the atom layout over rows padded to 128 and KG groups
+//                    of 64 (padding written as zero scales)
 template <bool SF_MMA>
-__device__ __forceinline__ void nvfp4_quantize_group(int64_t idx, const uint16_t* __restrict__ x,
-                                                     int64_t M, int64_t K,
-                                                     const float* __restrict__ g_ptr,
-                                                     uint8_t* __restrict__ xq,
-                                                     uint8_t* __restrict__ xs, int64_t rows_total,
-                                                     int64_t kg_total) {
-  if (idx >= rows_total * kg_total) return;
-  const int64_t r = idx / kg_total;
-  const int64_t kg = idx % kg_total;
+__device__ __forceinline__ void nvfp4_quantize_segment(int64_t warp_id, int lane,
+                                                       const uint16_t* __restrict__ x, int64_t M,
+                                                       int64_t K, float g, float c,
+                                                       uint8_t* __restrict__ xq,
+                                                       uint8_t* __restrict__ xs, int64_t rows_total,
+                                                       int64_t segs, int64_t KG) {
+  if (warp_id >= rows_total * segs) return;  // warp-uniform
+  const int64_t r = warp_id / segs;
+  const int64_t seg = warp_id % segs;
   const int64_t nblk = K / 16;
-  const float g = __ldg(g_ptr);
-  const float c = __frcp_rn(__fmul_rn(6.0f, g));
-
-  int nb = 0;  // valid 16-blocks in this group
-  if (r < M && 4 * kg < nblk) nb = (nblk - 4 * kg >= 4) ? 4 : static_cast<int>(nblk - 4 * kg);
-
-  uint32_t scales[4] = {0u, 0u, 0u, 0u};
-  if (nb > 0) {
-    const uint16_t* xr = x + r * K + kg * 64;
-    uint8_t* qr = xq + r * (K / 2) + kg * 32;
-    uint4 raw[8];
+  uint4 raw[4];
+  bool valid[4];
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      if (b < nb) {
-        raw[2 * b] = ldg16(xr + b * 16);
-        raw[2 * b + 1] = ldg16(xr + b * 16 + 8);
-      }
-    }
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      if (b < nb) {
-        const uint32_t w[8] = {raw[2 * b].x, raw[2 * b].y, raw[2 * b].z, raw[2 * b].w,
-                               raw[2 * b + 1].x, raw[2 * b + 1].y, raw[2 * b + 1].z,
-                               raw[2 * b + 1].w};
-        uint32_t lo, hi;
-        nvfp4_block(w, c, g, &scales[b], &lo, &hi);
-        *reinterpret_cast<uint2*>(qr + b * 8) = make_uint2(lo, hi);
-      }
-    }
+  for (int i = 0; i < 4; ++i) {
+    const int64_t e = seg * 1024 + i * 256 + lane * 8;
+    valid[i] = (r < M) && (e < K);  // K % 16 == 0: a lane pair is valid together
+    raw[i] = valid[i] ? ldg16(x + r * K + e) : make_uint4(0u, 0u, 0u, 0u);
   }
-  const uint32_t word = scales[0] | (scales[1] << 8) | (scales[2] << 16) | (scales[3] << 24);
-  if (SF_MMA) {
-    *reinterpret_cast<uint32_t*>(xs + sf_act_word_offset(r, kg, kg_total)) = word;
-  } else if (nb > 0) {
-    uint8_t* sr = xs + r * nblk + kg * 4;
-    if (nb == 4 && (reinterpret_cast<uintptr_t>(sr) & 3) == 0) {
-      *reinterpret_cast<uint32_t*>(sr) = word;
-    } else {
 #pragma unroll
-      for (int b = 0; b < 4; ++b)
-        if (b < nb) sr[b] = static_cast<uint8_t>(scales[b]);
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[2 * j] = bf16_lo(w[j]);
+      v[2 * j + 1] = bf16_hi(w[j]);
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[j]));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    const float sf = __fmul_rn(amax, c);
+    const uint32_t s = cvt_e4m3x4(sf, 0.0f, 0.0f, 0.0f) & 0xFFu;
+    const float d = __fmul_rn(e4m3_positive_value(s), g);
+    uint32_t codes = 0u;
+    if (d != 0.0f) {
+      const float inv = __frcp_rn(d);
+      float a[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a[j] = __fmul_rn(v[j], inv);
+      codes = cvt_e2m1x8(a);
+    }
+    const int64_t e = seg * 1024 + i * 256 + lane * 8;
+    if (valid[i]) *reinterpret_cast<uint32_t*>(xq + r * (K / 2) + e / 2) = codes;
+    // scales of blocks (lane/2) .. : gather 4 consecutive blocks into lane % 8 == 0
+    const uint32_t s1 = __shfl_down_sync(0xffffffffu, s, 2);
+    const uint32_t s2 = __shfl_down_sync(0xffffffffu, s, 4);
+    const uint32_t s3 = __shfl_down_sync(0xffffffffu, s, 6);
+    if ((lane & 7) == 0) {
+      const uint32_t word = s | (s1 << 8) | (s2 << 16) | (s3 << 24);
+      const int64_t kg = (seg * 1024 + i * 256) / 64 + lane / 8;
+      if (SF_MMA) {
+        if (kg < KG) *reinterpret_cast<uint32_t*>(xs + sf_act_word_offset(r, kg, KG)) = word;
+      } else if (r < M && 4 * kg < nblk) {
+        uint8_t* sr = xs + r * nblk + kg * 4;
+        if (4 * kg + 4 <= nblk && (reinterpret_cast<uintptr_t>(sr) & 3) == 0) {
+          *reinterpret_cast<uint32_t*>(sr) = word;
+        } else {
+#pragma unroll
+          for (int b = 0; b < 4; ++b)
+            if (4 * kg + b < nblk) sr[b] = static_cast<uint8_t>(word >> (8 * b));
+        }
+      }
     }
   }
 }
@@ -126,32 +143,62 @@ template <bool SF_MMA>
 __global__ void __launch_bounds__(kQuantThreads)
 nvfp4_quantize_kernel(const uint16_t* __restrict__ x, int64_t M, int64_t K,
                       const float* __restrict__ g_ptr, uint8_t* __restrict__ xq,
-                      uint8_t* __restrict__ xs, int64_t rows_total, int64_t kg_total) {
-  nvfp4_quantize_group<SF_MMA>(static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x, x, M,
-                               K, g_ptr, xq, xs, rows_total, kg_total);
+                      uint8_t* __restrict__ xs, int64_t rows_total, int64_t segs, int64_t KG) {
+  const float g = __ldg(g_ptr);
+  const float c = __frcp_rn(__fmul_rn(6.0f, g));
+  const int64_t warp_id = static_cast<int64_t>(blockIdx.x) * (kQuantThreads / 32) + threadIdx.x / 32;
+  nvfp4_quantize_segment<SF_MMA>(warp_id, threadIdx.x % 32, x, M, K, g, c, xq, xs, rows_total,
+                                 segs, KG);
 }
 
-// Row-major weight scales [N, K/16] -> atom layout for tiles of `bn` rows.
-// One thread per (tile, row slot nn < na*128, group kg).
-__device__ __forceinline__ void nvfp4_weight_scale_word(int64_t idx, const uint8_t* __restrict__ ws,
-                                                        int64_t N, int64_t K, int bn, int na,
-                                                        int64_t n_tiles, int64_t KG,
-                                                        uint8_t* __restrict__ out) {
-  const int64_t slots = static_cast<int64_t>(na) * 128;
-  if (idx >= n_tiles * slots * KG) return;
-  const int64_t kg = idx % KG;
-  const int64_t nn = (idx / KG) % slots;
-  const int64_t t = idx / (KG * slots);
-  const int64_t n = t * bn + nn;
+// Row-major weight scales [N, K/16] -> atom layout for tiles of `bn` rows, through
+// shared memory so that both the reads (64 contiguous bytes per row) and the
+// writes (whole 512-byte atoms) are coalesced. One block per (tile, 128-row atom
+// a, 16 consecutive 64-element groups).
+constexpr int kWsGroups = 16;
+__device__ __forceinline__ void nvfp4_weight_scale_atoms(int64_t job, int tid,
+                                                         const uint8_t* __restrict__ ws, int64_t N,
+                                                         int64_t K, int bn, int na, int64_t n_tiles,
+                                                         int64_t KG, uint8_t* __restrict__ out,
+                                                         uint32_t (*tile)[kWsGroups + 1]) {
+  const int64_t kg_chunks = ceil_div64(KG, kWsGroups);
+  const int64_t kc = job % kg_chunks;
+  const int a = static_cast<int>((job / kg_chunks) % na);
+  const int64_t t = job / (kg_chunks * na);
   const int64_t nblk = K / 16;
-  uint32_t word = 0;
-  if (nn < bn && n < N) {
-    const uint8_t* src = ws + n * nblk + kg * 4;
+  // load: 128 rows x 16 groups; thread -> (row = tid / 2, groups 8 * (tid % 2) .. +8)
+  {
+    const int rr = tid / 2;
+    const int g0 = (tid % 2) * 8;
+    const int64_t nn = static_cast<int64_t>(a) * 128 + rr;
+    const int64_t n = t * bn + nn;
+    const bool row_ok = nn < bn && n < N;
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
-      if (4 * kg + j < nblk) word |= static_cast<uint32_t>(__ldg(src + j)) << (8 * j);
+    for (int j = 0; j < 8; ++j) {
+      const int64_t kg = kc * kWsGroups + g0 + j;
+      uint32_t word = 0;
+      if (row_ok && 4 * kg < nblk) {
+        const uint8_t* src = ws + n * nblk + kg * 4;
+        if (4 * kg + 4 <= nblk && (reinterpret_cast<uintptr_t>(src) & 3) == 0) {
+          word = __ldg(reinterpret_cast<const uint32_t*>(src));
+        } else {
+          for (int b = 0; b < 4; ++b)
+            if (4 * kg + b < nblk) word |= static_cast<uint32_t>(__ldg(src + b)) << (8 * b);
+        }
+      }
+      tile[rr][g0 + j] = word;
+    }
   }
-  *reinterpret_cast<uint32_t*>(out + sf_wgt_word_offset(t, nn, kg, KG, na)) = word;
+  __syncthreads();
+  // store: per group, one 512-byte atom = 128 words; thread tid writes word tid % 128
+  for (int j = tid / 128; j < kWsGroups; j += 2) {
+    const int64_t kg = kc * kWsGroups + j;
+    if (kg >= KG) continue;
+    const int w = tid % 128;
+    const int rr = (w % 4) * 32 + w / 4;  // word w holds row rr of the atom
+    uint8_t* atom = out + static_cast<size_t>(((t * KG) + kg) * na + a) * kSfAtomBytes;
+    reinterpret_cast<uint32_t*>(atom)[w] = tile[rr][j];
+  }
 }
 
 // The prologue of nvfp4_linear in one launch: blocks [0, act_blocks) quantize the
@@ -162,23 +209,49 @@ __device__ __forceinline__ void nvfp4_weight_scale_word(int64_t idx, const uint8
 __global__ void __launch_bounds__(kQuantThreads)
 nvfp4_prologue_kernel(const uint16_t* __restrict__ x, int64_t M, int64_t K,
                       const float* __restrict__ g_ptr, uint8_t* __restrict__ xq,
-                      uint8_t* __restrict__ xs, int64_t rows_total, int64_t KG,
+                      uint8_t* __restrict__ xs, int64_t rows_total, int64_t segs, int64_t KG,
                       int64_t act_blocks, const uint8_t* __restrict__ ws, int64_t N, int bn,
                       int na, int64_t n_tiles, uint8_t* __restrict__ wout) {
+  __shared__ uint32_t tile[128][kWsGroups + 1];
   grid_dependents_launch();
   if (blockIdx.x < act_blocks) {
-    nvfp4_quantize_group<true>(static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x, x, M,
-                               K, g_ptr, xq, xs, rows_total, KG);
+    const float g = __ldg(g_ptr);
+    const float c = __frcp_rn(__fmul_rn(6.0f, g));
+    const int64_t warp_id =
+        static_cast<int64_t>(blockIdx.x) * (kQuantThreads / 32) + threadIdx.x / 32;
+    nvfp4_quantize_segment<true>(warp_id, threadIdx.x % 32, x, M, K, g, c, xq, xs, rows_total,
+                                 segs, KG);
   } else {
-    nvfp4_weight_scale_word((static_cast<int64_t>(blockIdx.x) - act_blocks) * blockDim.x +
-                                threadIdx.x,
-                            ws, N, K, bn, na, n_tiles, KG, wout);
+    nvfp4_weight_scale_atoms(static_cast<int64_t>(blockIdx.x) - act_blocks, threadIdx.x, ws, N, K,
+                             bn, na, n_tiles, KG, wout, tile);
   }
 }
 
-// FP8 row-wise: one warp per row; pass 1 takes the row amax, pass 2 encodes.
+// FP8 row-wise: one warp per row.
 //   scale = amax / 448 (fp32 division); scale == 0 -> zero codes;
 //   else codes = E4M3(x * (1/scale)).  Requires K % 8 == 0.
+// CACHED: the row is held in registers (K <= 32 * 8 * kFp8Chunks) and read once;
+// otherwise a second pass re-reads it (from L1/L2) to encode.
+constexpr int kFp8Chunks = 16;
+
+__device__ __forceinline__ uint2 fp8r_encode8(const uint4 u, float inv) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  const uint32_t lo = cvt_e4m3x4(__fmul_rn(bf16_lo(w[0]), inv), __fmul_rn(bf16_hi(w[0]), inv),
+                                 __fmul_rn(bf16_lo(w[1]), inv), __fmul_rn(bf16_hi(w[1]), inv));
+  const uint32_t hi = cvt_e4m3x4(__fmul_rn(bf16_lo(w[2]), inv), __fmul_rn(bf16_hi(w[2]), inv),
+                                 __fmul_rn(bf16_lo(w[3]), inv), __fmul_rn(bf16_hi(w[3]), inv));
+  return make_uint2(lo, hi);
+}
+
+__device__ __forceinline__ float amax8(const uint4 u) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
+  return m;
+}
+
+template <bool CACHED>
 __global__ void __launch_bounds__(kQuantThreads)
 fp8r_quantize_rows_kernel(const uint16_t* __restrict__ x, int64_t M, int64_t K,
                           uint8_t* __restrict__ xq, float* __restrict__ x_scale) {
@@ -187,33 +260,38 @@ fp8r_quantize_rows_kernel(const uint16_t* __restrict__ x, int64_t M, int64_t K,
   const int lane = threadIdx.x % 32;
   if (row >= M) return;
   const uint16_t* xr = x + row * K;
+  uint8_t* qr = xq + row * K;
   const int64_t chunks = K / 8;
   float amax = 0.0f;
-  for (int64_t ch = lane; ch < chunks; ch += 32) {
-    const uint4 u = ldg16(xr + ch * 8);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  uint4 cache[CACHED ? kFp8Chunks : 1];
+  if constexpr (CACHED) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
+    for (int i = 0; i < kFp8Chunks; ++i) {
+      const int64_t ch = lane + 32 * i;
+      cache[i] = ch < chunks ? ldg16(xr + ch * 8) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int i = 0; i < kFp8Chunks; ++i) amax = fmaxf(amax, amax8(cache[i]));
+  } else {
+    for (int64_t ch = lane; ch < chunks; ch += 32) amax = fmaxf(amax, amax8(ldg16(xr + ch * 8)));
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
   const float scale = __fdiv_rn(amax, 448.0f);
   if (lane == 0) x_scale[row] = scale;
-  uint8_t* qr = xq + row * K;
-  if (scale == 0.0f) {
+  const float inv = scale == 0.0f ? 0.0f : __frcp_rn(scale);
+  if constexpr (CACHED) {
+#pragma unroll
+    for (int i = 0; i < kFp8Chunks; ++i) {
+      const int64_t ch = lane + 32 * i;
+      if (ch < chunks)
+        *reinterpret_cast<uint2*>(qr + ch * 8) =
+            scale == 0.0f ? make_uint2(0u, 0u) : fp8r_encode8(cache[i], inv);
+    }
+  } else {
     for (int64_t ch = lane; ch < chunks; ch += 32)
-      *reinterpret_cast<uint2*>(qr + ch * 8) = make_uint2(0u, 0u);
-    return;
-  }
-  const float inv = __frcp_rn(scale);
-  for (int64_t ch = lane; ch < chunks; ch += 32) {
-    const uint4 u = ldg16(xr + ch * 8);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-    const uint32_t lo = cvt_e4m3x4(__fmul_rn(bf16_lo(w[0]), inv), __fmul_rn(bf16_hi(w[0]), inv),
-                                   __fmul_rn(bf16_lo(w[1]), inv), __fmul_rn(bf16_hi(w[1]), inv));
-    const uint32_t hi = cvt_e4m3x4(__fmul_rn(bf16_lo(w[2]), inv), __fmul_rn(bf16_hi(w[2]), inv),
-                                   __fmul_rn(bf16_lo(w[3]), inv), __fmul_rn(bf16_hi(w[3]), inv));
-    *reinterpret_cast<uint2*>(qr + ch * 8) = make_uint2(lo, hi);
+      *reinterpret_cast<uint2*>(qr + ch * 8) =
+          scale == 0.0f ? make_uint2(0u, 0u) : fp8r_encode8(ldg16(xr + ch * 8), inv);
   }
 }
 
@@ -258,9 +336,10 @@ inline unsigned grid_for(int64_t work, int threads) {
 
 cudaError_t launch_nvfp4_quantize_rowmajor(const void* x, int64_t M, int64_t K, const float* g,
                                            uint8_t* xq, uint8_t* xs, cudaStream_t s) {
-  const int64_t kg_total = ceil_div64(K, 64);
-  nvfp4_quantize_kernel<false><<<grid_for(M * kg_total, kQuantThreads), kQuantThreads, 0, s>>>(
-      static_cast<const uint16_t*>(x), M, K, g, xq, xs, M, kg_total);
+  const int64_t segs = ceil_div64(K, 1024);
+  const int warps_per_block = kQuantThreads / 32;
+  nvfp4_quantize_kernel<false><<<grid_for(M * segs, warps_per_block), kQuantThreads, 0, s>>>(
+      static_cast<const uint16_t*>(x), M, K, g, xq, xs, M, segs, ceil_div64(K, 64));
   return cudaGetLastError();
 }
 
@@ -270,13 +349,14 @@ cudaError_t launch_nvfp4_prologue(const void* x, int64_t M, int64_t K, const uin
   const Nvfp4Workspace L = nvfp4_workspace(M, K, N, bn);
   const int64_t KG = sf_kgroups(K);
   const int64_t rows = ceil_div64(M, 128) * 128;
+  const int64_t segs = ceil_div64(KG * 64, 1024);
   const int na = (bn + 127) / 128;
   const int64_t n_tiles = ceil_div64(N, bn);
-  const int64_t act_blocks = grid_for(rows * KG, kQuantThreads);
-  const int64_t w_blocks = grid_for(n_tiles * na * 128 * KG, kQuantThreads);
+  const int64_t act_blocks = grid_for(rows * segs, kQuantThreads / 32);
+  const int64_t w_blocks = n_tiles * na * ceil_div64(KG, kWsGroups);
   nvfp4_prologue_kernel<<<static_cast<unsigned>(act_blocks + w_blocks), kQuantThreads, 0, s>>>(
       static_cast<const uint16_t*>(x), M, K, input_scale, workspace + L.codes_off,
-      workspace + L.act_sf_off, rows, KG, act_blocks, w_scale, N, bn, na, n_tiles,
+      workspace + L.act_sf_off, rows, segs, KG, act_blocks, w_scale, N, bn, na, n_tiles,
       workspace + L.wgt_sf_off);
   return cudaGetLastError();
 }
@@ -284,8 +364,13 @@ cudaError_t launch_nvfp4_prologue(const void* x, int64_t M, int64_t K, const uin
 cudaError_t launch_fp8r_quantize_rows(const void* x, int64_t M, int64_t K, uint8_t* xq,
                                       float* x_scale, cudaStream_t s) {
   const int rows_per_block = kQuantThreads / 32;
-  fp8r_quantize_rows_kernel<<<grid_for(M, rows_per_block), kQuantThreads, 0, s>>>(
-      static_cast<const uint16_t*>(x), M, K, xq, x_scale);
+  if (K <= 32 * 8 * kFp8Chunks) {
+    fp8r_quantize_rows_kernel<true><<<grid_for(M, rows_per_block), kQuantThreads, 0, s>>>(
+        static_cast<const uint16_t*>(x), M, K, xq, x_scale);
+  } else {
+    fp8r_quantize_rows_kernel<false><<<grid_for(M, rows_per_block), kQuantThreads, 0, s>>>(
+        static_cast<const uint16_t*>(x), M, K, xq, x_scale);
+  }
   return cudaGetLastError();
 }
 
