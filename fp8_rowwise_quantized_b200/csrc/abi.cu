@@ -140,13 +140,13 @@ int nvfp4_quantize_act(const void* x, int64_t M, int64_t K, const float* input_s
 
 size_t nvfp4_linear_workspace_size(int64_t M, int64_t K, int64_t N) {
   if (!nvfp4_shape_ok(M, K, N)) return 0;
-  return ql::nvfp4_workspace(M, K, N, ql::choose_bn(true, M, N)).total;
+  return ql::nvfp4_workspace(M, K, N, ql::choose_config(true, M, N).bn).total;
 }
 
 int nvfp4_linear_workspace_layout(int64_t M, int64_t K, int64_t N, size_t* codes_offset,
                                   size_t* act_scales_offset, size_t* weight_scales_offset) {
   if (!nvfp4_shape_ok(M, K, N)) return QL_ERR_SHAPE;
-  const ql::Nvfp4Workspace L = ql::nvfp4_workspace(M, K, N, ql::choose_bn(true, M, N));
+  const ql::Nvfp4Workspace L = ql::nvfp4_workspace(M, K, N, ql::choose_config(true, M, N).bn);
   if (codes_offset) *codes_offset = L.codes_off;
   if (act_scales_offset) *act_scales_offset = L.act_sf_off;
   if (weight_scales_offset) *weight_scales_offset = L.wgt_sf_off;
@@ -159,7 +159,7 @@ int nvfp4_linear_prologue(const void* x, int64_t M, int64_t K, const uint8_t* w_
   if (!x || !w_scale || !input_scale || M <= 0 || N <= 0 || K <= 0) return QL_ERR_INVALID_ARG;
   if (!nvfp4_shape_ok(M, K, N)) return fail_shape("nvfp4: needs K >= 32 and K % 32 == 0");
   if (!aligned16(x)) return QL_ERR_ALIGN;
-  const int bn = ql::choose_bn(true, M, N);
+  const int bn = ql::choose_config(true, M, N).bn;
   const ql::Nvfp4Workspace L = ql::nvfp4_workspace(M, K, N, bn);
   if (!workspace || workspace_bytes < L.total) return QL_ERR_WORKSPACE;
   if (!aligned16(workspace)) return QL_ERR_ALIGN;
@@ -179,7 +179,8 @@ static int nvfp4_gemm_impl(int64_t M, int64_t K, const uint8_t* w, int64_t N,
     return QL_ERR_INVALID_ARG;
   if (!nvfp4_shape_ok(M, K, N)) return fail_shape("nvfp4: needs K >= 32 and K % 32 == 0");
   if (!aligned16(w) || !aligned16(y) || (bias && !aligned16(bias))) return QL_ERR_ALIGN;
-  const int bn = ql::choose_bn(true, M, N);
+  const ql::GemmConfig cfg = ql::choose_config(true, M, N);
+  const int bn = cfg.bn;
   const ql::Nvfp4Workspace L = ql::nvfp4_workspace(M, K, N, bn);
   if (!workspace || workspace_bytes < L.total) return QL_ERR_WORKSPACE;
   if (!aligned16(workspace)) return QL_ERR_ALIGN;
@@ -190,6 +191,7 @@ static int nvfp4_gemm_impl(int64_t M, int64_t K, const uint8_t* w, int64_t N,
   ql::GemmProblem p{};
   p.fp4 = true;
   p.bn = bn;
+  p.cg = cfg.cg;
   p.M = M;
   p.N = N;
   p.K = K;
@@ -225,7 +227,7 @@ int nvfp4_linear(const void* x, int64_t M, int64_t K, const uint8_t* w, const ui
   if (!nvfp4_shape_ok(M, K, N)) return fail_shape("nvfp4: needs K >= 32 and K % 32 == 0");
   if (!aligned16(x) || !aligned16(w) || !aligned16(y) || (bias && !aligned16(bias)))
     return QL_ERR_ALIGN;
-  const ql::Nvfp4Workspace L = ql::nvfp4_workspace(M, K, N, ql::choose_bn(true, M, N));
+  const ql::Nvfp4Workspace L = ql::nvfp4_workspace(M, K, N, ql::choose_config(true, M, N).bn);
   if (!workspace || workspace_bytes < L.total) return QL_ERR_WORKSPACE;
   int rc = nvfp4_linear_prologue(x, M, K, w_scale, N, input_scale, workspace, workspace_bytes,
                                  stream);
@@ -276,7 +278,9 @@ static int fp8r_gemm_impl(const uint8_t* xq, const float* x_scale, int64_t M, in
   if (rc != QL_OK) return rc;
   ql::GemmProblem p{};
   p.fp4 = false;
-  p.bn = ql::choose_bn(false, M, N);
+  const ql::GemmConfig cfg = ql::choose_config(false, M, N);
+  p.bn = cfg.bn;
+  p.cg = cfg.cg;
   p.M = M;
   p.N = N;
   p.K = K;

@@ -7,15 +7,20 @@
 // with row-wise scales" step of the Diffusers page "BFL (fp8r / nvfp4)", section
 // "Kernels", table.
 //
-// Structure: one persistent CTA per SM walks output tiles of 128 x BN.
-//   warp 0     TMA producer: A and B tiles (128-byte swizzle), scale atoms (bulk
-//              copies), into a STAGES-deep shared-memory ring;
-//   warp 1     allocates TMEM and issues the MMAs from one thread: per stage it
-//              copies the scale atoms into TMEM (tcgen05.cp) and issues 4 MMAs of
-//              K = 64 (FP4) or K = 32 (FP8) into a TMEM accumulator;
-//   warps 2-5  epilogue: TMEM -> registers (tcgen05.ld), scale, bias, bf16, store.
-// Accumulators are double-buffered in TMEM when they fit (BN <= 192), so the
-// epilogue of one tile overlaps the main loop of the next.
+// Structure: persistent CTAs, CG = 1 (one SM per 128 x BN tile) or CG = 2 (a CTA
+// pair per 256 x BN tile: one tcgen05 MMA spans both SMs; each CTA holds 128 rows
+// of A, half of B and the scales its MMA rows need, so each SM streams about half
+// the B bytes per flop). Per CTA:
+//   warp 0     TMA producer: A, B tiles (128-byte swizzle) and scale atoms into a
+//              STAGES-deep shared-memory ring; in a pair every load's bytes are
+//              counted on the leader CTA's barrier;
+//   warp 1     TMEM allocation; in the leader CTA, one thread per stage copies the
+//              scale atoms into TMEM (tcgen05.cp) and issues 4 MMAs of K = 64 (FP4)
+//              or K = 32 (FP8) into a TMEM accumulator;
+//   warps 2-5  epilogue: TMEM -> registers (tcgen05.ld), scale, bias, bf16,
+//              128-byte-swizzled staging tile, TMA store.
+// Accumulators are double-buffered in TMEM when they fit, so the epilogue of one
+// tile overlaps the main loop of the next.
 // Every wait is bounded by a deadline; on expiry the kernel records
 // QL_ERR_TIMEOUT in the device status word, drains its own copies and MMAs,
 // frees TMEM and returns.
@@ -34,7 +39,7 @@ namespace ql {
 
 namespace {
 
-constexpr int kBM = 128;
+constexpr int kRowsPerCta = 128;
 constexpr int kThreads = 192;
 constexpr int kSmemLimit = 232448;  // 227 KB opt-in per block
 constexpr int kTmemCols = 512;
@@ -44,8 +49,6 @@ struct GemmArgs {
   int M, N, K;
   int tiles_m, tiles_n, num_k_tiles, total_tiles;
   int64_t kg;               // FP4: 64-element scale groups per row (padded)
-  const uint8_t* sfa;       // FP4: activation scale atoms
-  const uint8_t* sfb;       // FP4: weight scale atoms
   const float* scale_a;     // FP4: input_scale (scalar)   FP8: x_scale [M]
   const float* scale_b;     // FP4: weight_scale_2 (scalar) FP8: w_scale [N]
   const float* bias;        // [N] or null
@@ -57,31 +60,35 @@ struct GemmArgs {
   int use_tma_store;        // Y written through shared memory + TMA (needs N % 8 == 0)
 };
 
-template <bool FP4, int BN>
+template <bool FP4, int BN, int CG>
 struct Cfg {
-  static constexpr int NA = (BN + 127) / 128;                       // 128-row scale atoms of B
-  static constexpr int A_BYTES = kBM * 128;
-  static constexpr int B_BYTES = BN * 128;
-  static constexpr int SFA_BYTES = FP4 ? 4 * kSfAtomBytes : 0;      // 4 K-groups x 1 atom
-  static constexpr int SFB_BYTES = FP4 ? 4 * NA * kSfAtomBytes : 0; // 4 K-groups x NA atoms
+  static constexpr int NA = (BN + 127) / 128;                        // 128-row scale atoms of B
+  static constexpr int B_ROWS = BN / CG;                             // B rows held by one CTA
+  static constexpr int A_BYTES = kRowsPerCta * 128;
+  static constexpr int B_BYTES = B_ROWS * 128;
+  static constexpr int SFA_BYTES = FP4 ? 4 * kSfAtomBytes : 0;       // 4 K-groups x 1 atom
+  static constexpr int SFB_BYTES = FP4 ? 4 * NA * kSfAtomBytes : 0;  // 4 K-groups x NA atoms
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  static constexpr int EPI_BYTES = 4 * 2 * kEpiBufBytes;            // 4 warps x 2 staging buffers
+  static constexpr int EPI_BYTES = 4 * 2 * kEpiBufBytes;             // 4 warps x 2 buffers
   static constexpr int RESERVED = 1024 /*alignment*/ + 1024 /*barriers*/ + EPI_BYTES;
   static constexpr int STAGES_FIT = (kSmemLimit - RESERVED) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
-  static constexpr int NACC = (2 * BN + 16 + 4 * NA * 4 <= kTmemCols) ? 2 : 1;
+  static constexpr int SF_COLS = FP4 ? 16 + 4 * NA * 4 : 0;
+  static constexpr int NACC = (2 * BN + SF_COLS <= kTmemCols) ? 2 : 1;
   static constexpr int SFA_COL = NACC * BN;
   static constexpr int SFB_COL = SFA_COL + 16;
   static constexpr int SMEM = RESERVED + STAGES * STAGE_BYTES;
-  static_assert(BN % 64 == 0, "epilogue works in 64-column slabs");
-  // instruction descriptor: M = 128, N = BN, K-major A and B, fp32 accumulate;
+  static constexpr int TILE_M = kRowsPerCta * CG;
+  // instruction descriptor: M = 128 * CG, N = BN, K-major A and B, fp32 accumulate;
   // FP4: E2M1 x E2M1 with UE4M3 scales; FP8: E4M3 x E4M3.
   static constexpr uint32_t IDESC =
-      FP4 ? ((1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(kBM >> 4) << 24))
-          : ((1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(kBM >> 4) << 24));
+      FP4 ? ((1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(TILE_M >> 4) << 24))
+          : ((1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(TILE_M >> 4) << 24));
   static_assert(STAGES >= 2, "shared memory too small for two stages");
-  static_assert(SFB_COL + 4 * NA * 4 <= kTmemCols, "TMEM budget");
-  static_assert(BN >= 64 && BN <= 256, "tile width");
+  static_assert(NACC * BN + SF_COLS <= kTmemCols, "TMEM budget");
+  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "tile width");
+  static_assert(CG == 1 || CG == 2, "one SM or a CTA pair");
+  static_assert(B_ROWS % 8 == 0, "B half must be whole 8-row core groups");
 };
 
 __device__ __forceinline__ void record_timeout(int* status) {
@@ -93,11 +100,13 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&p);
 }
 
-template <bool FP4, int BN>
+template <bool FP4, int BN, int CG>
 __global__ void __launch_bounds__(kThreads, 1)
 qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+             const __grid_constant__ CUtensorMap tmap_sfa,
+             const __grid_constant__ CUtensorMap tmap_sfb,
              const __grid_constant__ CUtensorMap tmap_y, const GemmArgs args) {
-  using C = Cfg<FP4, BN>;
+  using C = Cfg<FP4, BN, CG>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -114,15 +123,22 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
   uint64_t* drain_bar = tempty_bar + 2;
   uint64_t* never_bar = drain_bar + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(never_bar + 1);
-  int* abort_flag = reinterpret_cast<int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
+  const uint32_t rank = (CG == 2) ? cluster_ctarank() : 0u;  // 0 = leader of the pair
+  const bool leader = rank == 0;
+  const int group = (CG == 2) ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
+  const int ngroups = (CG == 2) ? static_cast<int>(nclusters_x()) : static_cast<int>(gridDim.x);
   const uint64_t deadline = globaltimer_ns() + args.timeout_ns;
 
   if (threadIdx.x == 0) {
     prefetch_tmap(&tmap_a);
     prefetch_tmap(&tmap_b);
+    if constexpr (FP4) {
+      prefetch_tmap(&tmap_sfa);
+      prefetch_tmap(&tmap_sfb);
+    }
     if (args.use_tma_store) prefetch_tmap(&tmap_y);
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
@@ -130,21 +146,30 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull_bar[b], 1);
-      mbar_init(&tempty_bar[b], 4);
+      mbar_init(&tempty_bar[b], 4 * CG);
     }
     mbar_init(drain_bar, 1);
     mbar_init(never_bar, 1);
-    *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, kTmemCols);
-    tmem_relinquish();
+    if constexpr (CG == 2) {
+      tmem_alloc_pair(tmem_holder, kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_holder, kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (CG == 2) cluster_sync_all();  // peer barriers are initialised
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // The leader's barriers, addressed from either CTA of the pair.
+  const uint32_t full_bar0 = (CG == 2) ? map_to_cta(smem_u32(full_bar), 0) : smem_u32(full_bar);
+  const uint32_t tempty_bar0 =
+      (CG == 2) ? map_to_cta(smem_u32(tempty_bar), 0) : smem_u32(tempty_bar);
 
   // Everything above overlaps the tail of the previous kernel on the stream;
   // global inputs are read only after it has completed.
@@ -164,27 +189,43 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     uint32_t phase = 0;
     bool ok = true;
     int issued = 0;
-    for (int tile = blockIdx.x; ok && tile < args.total_tiles; tile += gridDim.x) {
+    for (int tile = group; ok && tile < args.total_tiles; tile += ngroups) {
       const int m_blk = tile % args.tiles_m;
       const int n_blk = tile / args.tiles_m;
+      const int a_row = m_blk * C::TILE_M + static_cast<int>(rank) * kRowsPerCta;
+      const int b_row = n_blk * BN + static_cast<int>(rank) * C::B_ROWS;
       for (int kt = 0; kt < args.num_k_tiles; ++kt) {
         if (!warp_wait_bounded(&empty_bar[stage], phase ^ 1u, deadline)) {
           ok = false;
           break;
         }
         if (elect_one()) {
-          mbar_arrive_expect_tx(&full_bar[stage], C::STAGE_BYTES);
-          tma_load_2d(smem_a + stage * C::A_BYTES, &tmap_a, &full_bar[stage], kt * 128,
-                      m_blk * kBM);
-          tma_load_2d(smem_b + stage * C::B_BYTES, &tmap_b, &full_bar[stage], kt * 128,
-                      n_blk * BN);
-          if constexpr (FP4) {
-            const uint8_t* sfa = args.sfa + (static_cast<int64_t>(m_blk) * args.kg + kt * 4) *
-                                                kSfAtomBytes;
-            const uint8_t* sfb = args.sfb + ((static_cast<int64_t>(n_blk) * args.kg + kt * 4) *
-                                             C::NA) * kSfAtomBytes;
-            bulk_load(smem_sfa + stage * C::SFA_BYTES, sfa, C::SFA_BYTES, &full_bar[stage]);
-            bulk_load(smem_sfb + stage * C::SFB_BYTES, sfb, C::SFB_BYTES, &full_bar[stage]);
+          const uint32_t fb = full_bar0 + stage * 8u;
+          uint8_t* sa = smem_a + stage * C::A_BYTES;
+          uint8_t* sb = smem_b + stage * C::B_BYTES;
+          uint8_t* ssa = smem_sfa + stage * C::SFA_BYTES;
+          uint8_t* ssb = smem_sfb + stage * C::SFB_BYTES;
+          // scale atoms: rows of the 2-D atom maps are 512-byte atoms
+          const int sfa_atom = static_cast<int>((static_cast<int64_t>(m_blk) * CG + rank) * args.kg +
+                                                kt * 4);
+          const int sfb_atom = static_cast<int>((static_cast<int64_t>(n_blk) * args.kg + kt * 4) *
+                                                C::NA);
+          if constexpr (CG == 2) {
+            if (leader) mbar_arrive_expect_tx(&full_bar[stage], CG * C::STAGE_BYTES);
+            tma_load_2d_pair(sa, &tmap_a, fb, kt * 128, a_row);
+            tma_load_2d_pair(sb, &tmap_b, fb, kt * 128, b_row);
+            if constexpr (FP4) {
+              tma_load_2d_pair(ssa, &tmap_sfa, fb, 0, sfa_atom);
+              tma_load_2d_pair(ssb, &tmap_sfb, fb, 0, sfb_atom);
+            }
+          } else {
+            mbar_arrive_expect_tx(&full_bar[stage], C::STAGE_BYTES);
+            tma_load_2d(sa, &tmap_a, &full_bar[stage], kt * 128, a_row);
+            tma_load_2d(sb, &tmap_b, &full_bar[stage], kt * 128, b_row);
+            if constexpr (FP4) {
+              tma_load_2d(ssa, &tmap_sfa, &full_bar[stage], 0, sfa_atom);
+              tma_load_2d(ssb, &tmap_sfb, &full_bar[stage], 0, sfb_atom);
+            }
           }
         }
         __syncwarp();
@@ -197,21 +238,23 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     }
     if (!ok) {
       record_timeout(args.status);
-      *abort_flag = 1;
-      // wait (bounded) for the copies this warp still has in flight
-      const uint64_t drain_deadline = globaltimer_ns() + 100000000ull;
-      const int n = issued < C::STAGES ? issued : C::STAGES;
-      int s = stage;
-      uint32_t p = phase;
-      for (int i = 0; i < n; ++i) {
-        if (--s < 0) {
-          s = C::STAGES - 1;
-          p ^= 1u;
+      // wait (bounded) for the copies still in flight: in a pair their bytes are
+      // counted on the leader's full barriers, which the leader drains
+      if (leader) {
+        const uint64_t drain_deadline = globaltimer_ns() + 100000000ull;
+        const int n = issued < C::STAGES ? issued : C::STAGES;
+        int s = stage;
+        uint32_t p = phase;
+        for (int i = 0; i < n; ++i) {
+          if (--s < 0) {
+            s = C::STAGES - 1;
+            p ^= 1u;
+          }
+          mbar_wait_bounded(&full_bar[s], p, drain_deadline);
         }
-        mbar_wait_bounded(&full_bar[s], p, drain_deadline);
       }
     }
-  } else if (run && warp == 1) {
+  } else if (run && warp == 1 && leader) {
     // ------------------------------------------------------------ MMA issuer
     int stage = 0;
     uint32_t phase = 0;
@@ -219,7 +262,7 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     uint32_t acc_phase = 0;
     bool ok = true;
     bool issued_any = false;
-    for (int tile = blockIdx.x; ok && tile < args.total_tiles; tile += gridDim.x) {
+    for (int tile = group; ok && tile < args.total_tiles; tile += ngroups) {
       if (!warp_wait_bounded(&tempty_bar[acc], acc_phase ^ 1u, deadline)) {
         ok = false;
         break;
@@ -240,29 +283,50 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
             const uint32_t sfb_addr = smem_u32(smem_sfb + stage * C::SFB_BYTES);
 #pragma unroll
             for (int kb = 0; kb < 4; ++kb) {
-              tmem_cp_32x128b_x4(tmem_base + C::SFA_COL + kb * 4,
-                                 smem_desc(sfa_addr + kb * kSfAtomBytes, 0, 128, 0));
+              const uint64_t da = smem_desc(sfa_addr + kb * kSfAtomBytes, 0, 128, 0);
+              if constexpr (CG == 2)
+                tmem_cp_32x128b_x4_pair(tmem_base + C::SFA_COL + kb * 4, da);
+              else
+                tmem_cp_32x128b_x4(tmem_base + C::SFA_COL + kb * 4, da);
 #pragma unroll
-              for (int a = 0; a < C::NA; ++a)
-                tmem_cp_32x128b_x4(tmem_base + C::SFB_COL + (kb * C::NA + a) * 4,
-                                   smem_desc(sfb_addr + (kb * C::NA + a) * kSfAtomBytes, 0, 128, 0));
+              for (int a = 0; a < C::NA; ++a) {
+                const uint64_t db = smem_desc(sfb_addr + (kb * C::NA + a) * kSfAtomBytes, 0, 128, 0);
+                const uint32_t col = tmem_base + C::SFB_COL + (kb * C::NA + a) * 4;
+                if constexpr (CG == 2)
+                  tmem_cp_32x128b_x4_pair(col, db);
+                else
+                  tmem_cp_32x128b_x4(col, db);
+              }
             }
 #pragma unroll
             for (int kb = 0; kb < 4; ++kb) {
-              mma_nvf4(d_tmem, smem_desc(a_addr + kb * 32, 16, 1024, 2),
-                       smem_desc(b_addr + kb * 32, 16, 1024, 2), C::IDESC,
-                       tmem_base + C::SFA_COL + kb * 4, tmem_base + C::SFB_COL + kb * C::NA * 4,
-                       (kt | kb) != 0 ? 1u : 0u);
+              const uint64_t ad = smem_desc(a_addr + kb * 32, 16, 1024, 2);
+              const uint64_t bd = smem_desc(b_addr + kb * 32, 16, 1024, 2);
+              const uint32_t sfa = tmem_base + C::SFA_COL + kb * 4;
+              const uint32_t sfb = tmem_base + C::SFB_COL + kb * C::NA * 4;
+              const uint32_t accum = (kt | kb) != 0 ? 1u : 0u;
+              if constexpr (CG == 2)
+                mma_nvf4_pair(d_tmem, ad, bd, C::IDESC, sfa, sfb, accum);
+              else
+                mma_nvf4(d_tmem, ad, bd, C::IDESC, sfa, sfb, accum);
             }
           } else {
 #pragma unroll
             for (int kb = 0; kb < 4; ++kb) {
-              mma_f8f6f4(d_tmem, smem_desc(a_addr + kb * 32, 16, 1024, 2),
-                         smem_desc(b_addr + kb * 32, 16, 1024, 2), C::IDESC,
-                         (kt | kb) != 0 ? 1u : 0u);
+              const uint64_t ad = smem_desc(a_addr + kb * 32, 16, 1024, 2);
+              const uint64_t bd = smem_desc(b_addr + kb * 32, 16, 1024, 2);
+              const uint32_t accum = (kt | kb) != 0 ? 1u : 0u;
+              if constexpr (CG == 2)
+                mma_f8f6f4_pair(d_tmem, ad, bd, C::IDESC, accum);
+              else
+                mma_f8f6f4(d_tmem, ad, bd, C::IDESC, accum);
             }
           }
-          tc_commit(&empty_bar[stage]);  // frees the stage once these MMAs have read it
+          // frees the stage (in both CTAs of a pair) once these MMAs have read it
+          if constexpr (CG == 2)
+            tc_commit_pair(&empty_bar[stage], 0x3);
+          else
+            tc_commit(&empty_bar[stage]);
         }
         __syncwarp();
         issued_any = true;
@@ -272,7 +336,12 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
         }
       }
       if (!ok) break;
-      if (elect_one()) tc_commit(&tfull_bar[acc]);  // accumulator ready for the epilogue
+      if (elect_one()) {  // accumulator ready for the epilogue (of both CTAs)
+        if constexpr (CG == 2)
+          tc_commit_pair(&tfull_bar[acc], 0x3);
+        else
+          tc_commit(&tfull_bar[acc]);
+      }
       __syncwarp();
       if (C::NACC == 2) {
         acc ^= 1;
@@ -283,24 +352,28 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     }
     if (!ok) {
       record_timeout(args.status);
-      *abort_flag = 1;
       if (issued_any) {  // wait (bounded) for this thread's MMAs and copies to finish
-        if (elect_one()) tc_commit(drain_bar);
+        if (elect_one()) {
+          if constexpr (CG == 2)
+            tc_commit_pair(drain_bar, 0x1);
+          else
+            tc_commit(drain_bar);
+        }
         __syncwarp();
         mbar_wait_bounded(drain_bar, 0, globaltimer_ns() + 100000000ull);
       }
     }
-  } else if (run) {
+  } else if (run && warp >= 2) {
     // ------------------------------------------------------------ epilogue
     const int q = warp % 4;  // TMEM lane quadrant this warp may access
-    const int row_in_tile = q * 32 + lane;
+    const int row_in_tile = static_cast<int>(rank) * kRowsPerCta + q * 32 + lane;
     uint8_t* stage = smem_epi + (warp - 2) * 2 * kEpiBufBytes;
     int buf = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     float alpha = 1.0f;
     if constexpr (FP4) alpha = __fmul_rn(__ldg(args.scale_a), __ldg(args.scale_b));
-    for (int tile = blockIdx.x; tile < args.total_tiles; tile += gridDim.x) {
+    for (int tile = group; tile < args.total_tiles; tile += ngroups) {
       const int m_blk = tile % args.tiles_m;
       const int n_blk = tile / args.tiles_m;
       if (!warp_wait_bounded(&tfull_bar[acc], acc_phase, deadline)) {
@@ -308,7 +381,8 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
         break;
       }
       tc_fence_after();
-      const int m = m_blk * kBM + row_in_tile;
+      const int m = m_blk * C::TILE_M + row_in_tile;
+      const int row0 = m_blk * C::TILE_M + static_cast<int>(rank) * kRowsPerCta + q * 32;
       float row_scale = 1.0f;
       if constexpr (!FP4) row_scale = (m < args.M) ? __ldg(args.scale_a + m) : 0.0f;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
@@ -323,13 +397,13 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
         if (sl == BN / 64 - 1) {  // all columns read: hand the buffer back early
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty_bar[acc]);
+          if (lane == 0) mbar_arrive_cluster(tempty_bar0 + acc * 8u);
         }
         const int n0 = n_blk * BN + sl * 64;
         if (n0 >= args.N) continue;  // warp-uniform
         if (args.use_tma_store) {
-          // columns n0 .. n0+63 of rows m_blk*128 + 32q .. +31: scale, bias, bf16,
-          // into a 128-byte-swizzled staging tile, then one TMA store per warp.
+          // columns n0 .. n0+63 of this warp's 32 rows: scale, bias, bf16, into a
+          // 128-byte-swizzled staging tile, then one TMA store per warp.
           uint32_t packed[32];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -359,7 +433,7 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
           fence_proxy_async_shared();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&tmap_y, sbuf, n0, m_blk * kBM + q * 32);
+            tma_store_2d(&tmap_y, sbuf, n0, row0);
             bulk_commit_group();
           }
           buf ^= 1;
@@ -391,9 +465,13 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
   // ------------------------------------------------------------ teardown
   tc_fence_before();
   __syncthreads();
+  if constexpr (CG == 2) cluster_sync_all();  // no peer accesses this CTA's memory any more
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if constexpr (CG == 2)
+      tmem_dealloc_pair(tmem_base, kTmemCols);
+    else
+      tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 
@@ -418,39 +496,24 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// Row-major uint8 matrix [rows, cols_bytes] viewed in boxes of [box_rows, 128 bytes]
-// with the 128-byte swizzle that the K-major MMA descriptors expect.
-bool make_tmap(CUtensorMap* map, const void* base, int64_t rows, int64_t cols_bytes, int box_rows) {
+bool encode_2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, uint64_t inner,
+               uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows,
+               CUtensorMapSwizzle swz, CUtensorMapL2promotion promo) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols_bytes), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols_bytes)};
-  const cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
   const cuuint32_t estr[2] = {1u, 1u};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  return enc(map, type, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, promo,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// bf16 row-major [rows, cols] in boxes of [32 rows, 64 columns] with the 128-byte
-// swizzle of the epilogue's staging tiles.
-bool make_tmap_y(CUtensorMap* map, void* base, int64_t rows, int64_t cols) {
-  EncodeTiledFn enc = get_encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols * 2)};
-  const cuuint32_t box[2] = {64u, 32u};
-  const cuuint32_t estr[2] = {1u, 1u};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-template <bool FP4, int BN>
+template <bool FP4, int BN, int CG>
 cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
-  using Cf = Cfg<FP4, BN>;
-  auto kern = qgemm_kernel<FP4, BN>;
+  using Cf = Cfg<FP4, BN, CG>;
+  auto kern = qgemm_kernel<FP4, BN, CG>;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -468,24 +531,41 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
 
   const int64_t k_bytes = FP4 ? p.K / 2 : p.K;
-  CUtensorMap ta, tb, ty;
-  if (!make_tmap(&ta, p.a, p.M, k_bytes, kBM) || !make_tmap(&tb, p.b, p.N, k_bytes, BN))
-    return cudaErrorInvalidValue;
-  const bool tma_store = (p.N % 8) == 0 && (reinterpret_cast<uintptr_t>(p.y) & 15) == 0;
+  CUtensorMap ta, tb, tsa, tsb, ty;
+  std::memset(&tsa, 0, sizeof(tsa));
+  std::memset(&tsb, 0, sizeof(tsb));
   std::memset(&ty, 0, sizeof(ty));
-  if (tma_store && !make_tmap_y(&ty, p.y, p.M, p.N)) return cudaErrorInvalidValue;
+  // A / B: uint8 rows of K* bytes, boxes of [rows, 128 bytes], 128-byte swizzle
+  if (!encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.a, k_bytes, p.M, k_bytes, 128, kRowsPerCta,
+                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
+      !encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.b, k_bytes, p.N, k_bytes, 128, Cf::B_ROWS,
+                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
+    return cudaErrorInvalidValue;
+  const int64_t kg = sf_kgroups(p.K);
+  if (FP4) {
+    // scale atoms as rows of 128 32-bit words; one stage = 4 (A) or 4 * NA (B) atoms
+    const int64_t a_atoms = ceil_div64(p.M, kRowsPerCta) * kg;
+    const int64_t b_atoms = ceil_div64(p.N, BN) * kg * Cf::NA;
+    if (!encode_2d(&tsa, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.sfa, 128, a_atoms, kSfAtomBytes, 128, 4,
+                   CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
+        !encode_2d(&tsb, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.sfb, 128, b_atoms, kSfAtomBytes, 128,
+                   4 * Cf::NA, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
+      return cudaErrorInvalidValue;
+  }
+  const bool tma_store = (p.N % 8) == 0 && (reinterpret_cast<uintptr_t>(p.y) & 15) == 0;
+  if (tma_store && !encode_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.y, p.N, p.M, p.N * 2, 64,
+                              32, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE))
+    return cudaErrorInvalidValue;
 
   GemmArgs a{};
   a.M = static_cast<int>(p.M);
   a.N = static_cast<int>(p.N);
   a.K = static_cast<int>(p.K);
-  a.tiles_m = static_cast<int>(ceil_div64(p.M, kBM));
+  a.tiles_m = static_cast<int>(ceil_div64(p.M, Cf::TILE_M));
   a.tiles_n = static_cast<int>(ceil_div64(p.N, BN));
   a.num_k_tiles = static_cast<int>(ceil_div64(p.K, FP4 ? kKTileFp4 : kKTileFp8));
   a.total_tiles = a.tiles_m * a.tiles_n;
-  a.kg = sf_kgroups(p.K);
-  a.sfa = p.sfa;
-  a.sfb = p.sfb;
+  a.kg = kg;
   a.scale_a = p.scale_a;
   a.scale_b = p.scale_b;
   a.bias = p.bias;
@@ -497,42 +577,76 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
   a.use_tma_store = tma_store ? 1 : 0;
 
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned>(a.total_tiles < sms ? a.total_tiles : sms));
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = Cf::SMEM;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int nattr = 0;
+  if (CG == 2) {
+    attr[nattr].id = cudaLaunchAttributeClusterDimension;
+    attr[nattr].val.clusterDim.x = 2;
+    attr[nattr].val.clusterDim.y = 1;
+    attr[nattr].val.clusterDim.z = 1;
+    ++nattr;
+  }
+  // Persistent grid: as many CTA groups as can be resident at once (pairs need two
+  // free SMs of one GPC, so fewer than SMs / 2 pairs may fit).
+  static int resident_groups[64] = {};
+  int max_groups = sms / CG;
+  if (dev < 64 && resident_groups[dev] == 0) {
+    int n = max_groups;
+    if (CG == 2) {
+      cfg.gridDim = dim3(static_cast<unsigned>(max_groups * CG));
+      cfg.attrs = attr;
+      cfg.numAttrs = nattr;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = max_groups;
+      }
+    }
+    resident_groups[dev] = n < max_groups ? n : max_groups;
+  }
+  if (dev < 64) max_groups = resident_groups[dev];
+  const int groups = a.total_tiles < max_groups ? a.total_tiles : max_groups;
+  cfg.gridDim = dim3(static_cast<unsigned>(groups * CG));
+  if (p.pdl) {
+    attr[nattr].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[nattr].val.programmaticStreamSerializationAllowed = 1;
+    ++nattr;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = p.pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kern, ta, tb, ty, a);
+  cfg.numAttrs = nattr;
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, ty, a);
 }
 
 }  // namespace
 
-int choose_bn(bool fp4, int64_t M, int64_t N) {
+GemmConfig choose_config(bool fp4, int64_t M, int64_t N) {
   (void)fp4;
-  (void)M;
-  if (N % 192 == 0 && N >= 1536) return 192;
-  if (N % 256 == 0 && N >= 4096) return 256;
-  return 128;
+  GemmConfig c{};
+  c.cg = M >= 512 ? 2 : 1;
+  c.bn = 128;
+  if (N % 192 == 0 && N >= 1536) c.bn = 192;
+  else if (N % 256 == 0 && N >= 4096) c.bn = 256;
+  return c;
 }
 
 cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream) {
-  if (p.fp4) {
-    switch (p.bn) {
-      case 128: return launch_typed<true, 128>(p, stream);
-      case 192: return launch_typed<true, 192>(p, stream);
-      case 256: return launch_typed<true, 256>(p, stream);
-    }
-  } else {
-    switch (p.bn) {
-      case 128: return launch_typed<false, 128>(p, stream);
-      case 192: return launch_typed<false, 192>(p, stream);
-      case 256: return launch_typed<false, 256>(p, stream);
-    }
-  }
+#define QL_CASE(FP4_, BN_, CG_) \
+  if (p.fp4 == FP4_ && p.bn == BN_ && p.cg == CG_) return launch_typed<FP4_, BN_, CG_>(p, stream);
+  QL_CASE(true, 128, 1)
+  QL_CASE(true, 192, 1)
+  QL_CASE(true, 256, 1)
+  QL_CASE(true, 128, 2)
+  QL_CASE(true, 192, 2)
+  QL_CASE(true, 256, 2)
+  QL_CASE(false, 128, 1)
+  QL_CASE(false, 192, 1)
+  QL_CASE(false, 256, 1)
+  QL_CASE(false, 128, 2)
+  QL_CASE(false, 192, 2)
+  QL_CASE(false, 256, 2)
+#undef QL_CASE
   return cudaErrorInvalidValue;
 }
 

@@ -10,9 +10,16 @@ constexpr int QL_ERR_TIMEOUT_CODE = 7;  // same value as QL_ERR_TIMEOUT in qline
 
 // One GEMM launch (both schemes). a, b: row-major codes [M, K*] and [N, K*]
 // (K* = K/2 bytes for FP4, K bytes for FP8).
+// Tile choice: output tiles of (128 * cg) x bn; cg = 2 runs one MMA over a CTA pair.
+struct GemmConfig {
+  int bn;
+  int cg;
+};
+
 struct GemmProblem {
   bool fp4;
   int bn;
+  int cg;
   int64_t M, N, K;
   const void* a;
   const void* b;
@@ -28,7 +35,7 @@ struct GemmProblem {
   bool pdl;              // launched right after its producer kernel (programmatic dependency)
 };
 
-int choose_bn(bool fp4, int64_t M, int64_t N);
+GemmConfig choose_config(bool fp4, int64_t M, int64_t N);
 cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream);
 
 cudaError_t launch_nvfp4_quantize_rowmajor(const void* x, int64_t M, int64_t K, const float* g,

@@ -40,6 +40,11 @@ def run_nvfp4(c: Nvfp4Case, rows=None, workspace=None):
     (130, 1024, 1536),   # tile width 192
     (300, 768, 4096),    # tile width 256 (single TMEM accumulator)
     (64, 3072, 200),     # N not a multiple of 8 -> scalar tail stores
+    (512, 256, 384),     # CTA-pair tiles (M >= 512), exact fit
+    (600, 512, 520),     # CTA pair: last pair tile half empty (follower rows all out)
+    (777, 1056, 1000),   # CTA pair, ragged M, N and K
+    (1024, 768, 1536),   # CTA pair, tile width 192
+    (520, 512, 4096),    # CTA pair, tile width 256 (single TMEM accumulator)
 ])
 def test_nvfp4_linear_small_full(M, K, N):
     run_nvfp4(Nvfp4Case(M, K, N, seed=M + N))
@@ -117,6 +122,9 @@ def run_fp8r(c: Fp8rCase, rows=None):
     (130, 1024, 1536, True),
     (300, 768, 4096, False),
     (64, 512, 200, False),
+    (600, 400, 520, True),     # CTA pair, ragged
+    (1000, 1024, 1536, False),  # CTA pair, tile width 192
+    (520, 256, 4096, True),    # CTA pair, tile width 256
 ])
 def test_fp8r_linear_small_full(M, K, N, bias):
     run_fp8r(Fp8rCase(M, K, N, seed=M + K, bias=bias))
