@@ -451,6 +451,18 @@ def run_ours(args):
                               "gemm_frac_of_peak": fl / (gms / 1e3) / 1e12 / pk}
             del L
         torch.cuda.empty_cache()
+        # GEMM tile sweep on the headline layer: (128 * cg) x bn output tiles
+        sweep = {}
+        for bn, cg in [(192, 2), (256, 2), (128, 2), (192, 1), (256, 1)]:
+            q.set_tile_override(bn, cg)
+            try:
+                layer.prologue()
+                gms, _ = time_events(layer.gemm, v_steps, 3, flush, stream)
+            finally:
+                q.set_tile_override(0, 0)
+            sweep[f"bn{bn}_cg{cg}"] = {"gemm_us": gms * 1e3,
+                                      "gemm_tflops": flops / (gms / 1e3) / 1e12}
+        variants["mlp_up_gemm_tile_sweep"] = sweep
 
     # --------------------------------------------------- CPU oracle baseline (rank 0, N=1)
     cpu = None

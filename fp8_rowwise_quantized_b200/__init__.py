@@ -23,6 +23,7 @@ __all__ = [
     "nvfp4_linear_workspace_size", "nvfp4_linear_workspace_layout", "nvfp4_global_scale",
     "fp8r_quantize_rows", "fp8r_linear", "fp8r_linear_gemm", "fp8r_linear_workspace_size",
     "ql_encode_e4m3", "ql_encode_e2m1", "read_device_status", "set_fault_injection",
+    "set_tile_override",
     "prepare_nvfp4_weight", "prepare_fp8r_weight", "QLinearError", "library_path",
 ]
 
@@ -251,3 +252,9 @@ def read_device_status() -> int:
 
 def set_fault_injection(enable: bool, timeout_ms: int = 0) -> None:
     _lib.load().ql_set_fault_injection(1 if enable else 0, int(timeout_ms))
+
+
+def set_tile_override(bn: int = 0, cg: int = 0) -> None:
+    """Force the GEMM tile ((128 * cg) x bn) for later calls; bn = 0 restores the
+    automatic choice."""
+    _lib.check("ql_set_tile_override", _lib.load().ql_set_tile_override(int(bn), int(cg)))

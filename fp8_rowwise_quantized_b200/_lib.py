@@ -42,6 +42,7 @@ SIGNATURES = {
     "ql_encode_e2m1": (C.c_int, [_f32p, _u8p, _i64, _vp]),
     "ql_read_device_status": (C.c_int, [C.POINTER(C.c_int)]),
     "ql_set_fault_injection": (None, [C.c_int, C.c_int]),
+    "ql_set_tile_override": (C.c_int, [C.c_int, C.c_int]),
     "ql_status_string": (C.c_char_p, [C.c_int]),
     "ql_last_error_message": (C.c_char_p, []),
 }

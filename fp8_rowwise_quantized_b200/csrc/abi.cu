@@ -140,7 +140,17 @@ int nvfp4_quantize_act(const void* x, int64_t M, int64_t K, const float* input_s
 
 size_t nvfp4_linear_workspace_size(int64_t M, int64_t K, int64_t N) {
   if (!nvfp4_shape_ok(M, K, N)) return 0;
-  return ql::nvfp4_workspace(M, K, N, ql::choose_config(true, M, N).bn).total;
+  // large enough for the weight-scale layout of every tile width
+  size_t need = 0;
+  for (int bn : {128, 192, 256}) {
+    const size_t t = ql::nvfp4_workspace(M, K, N, bn).total;
+    need = t > need ? t : need;
+  }
+  return need;
+}
+
+int ql_set_tile_override(int bn, int cg) {
+  return ql::set_tile_override(bn, cg) ? QL_OK : QL_ERR_INVALID_ARG;
 }
 
 int nvfp4_linear_workspace_layout(int64_t M, int64_t K, int64_t N, size_t* codes_offset,
@@ -161,7 +171,7 @@ int nvfp4_linear_prologue(const void* x, int64_t M, int64_t K, const uint8_t* w_
   if (!aligned16(x)) return QL_ERR_ALIGN;
   const int bn = ql::choose_config(true, M, N).bn;
   const ql::Nvfp4Workspace L = ql::nvfp4_workspace(M, K, N, bn);
-  if (!workspace || workspace_bytes < L.total) return QL_ERR_WORKSPACE;
+  if (!workspace || workspace_bytes < nvfp4_linear_workspace_size(M, K, N)) return QL_ERR_WORKSPACE;
   if (!aligned16(workspace)) return QL_ERR_ALIGN;
   int rc = check_device(nullptr);
   if (rc != QL_OK) return rc;
@@ -182,7 +192,7 @@ static int nvfp4_gemm_impl(int64_t M, int64_t K, const uint8_t* w, int64_t N,
   const ql::GemmConfig cfg = ql::choose_config(true, M, N);
   const int bn = cfg.bn;
   const ql::Nvfp4Workspace L = ql::nvfp4_workspace(M, K, N, bn);
-  if (!workspace || workspace_bytes < L.total) return QL_ERR_WORKSPACE;
+  if (!workspace || workspace_bytes < nvfp4_linear_workspace_size(M, K, N)) return QL_ERR_WORKSPACE;
   if (!aligned16(workspace)) return QL_ERR_ALIGN;
   int dev = 0;
   int rc = check_device(&dev);
@@ -228,7 +238,7 @@ int nvfp4_linear(const void* x, int64_t M, int64_t K, const uint8_t* w, const ui
   if (!aligned16(x) || !aligned16(w) || !aligned16(y) || (bias && !aligned16(bias)))
     return QL_ERR_ALIGN;
   const ql::Nvfp4Workspace L = ql::nvfp4_workspace(M, K, N, ql::choose_config(true, M, N).bn);
-  if (!workspace || workspace_bytes < L.total) return QL_ERR_WORKSPACE;
+  if (!workspace || workspace_bytes < nvfp4_linear_workspace_size(M, K, N)) return QL_ERR_WORKSPACE;
   int rc = nvfp4_linear_prologue(x, M, K, w_scale, N, input_scale, workspace, workspace_bytes,
                                  stream);
   if (rc != QL_OK) return rc;

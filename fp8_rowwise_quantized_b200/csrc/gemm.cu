@@ -19,8 +19,9 @@
 //              or K = 32 (FP8) into a TMEM accumulator;
 //   warps 2-5  epilogue: TMEM -> registers (tcgen05.ld), scale, bias, bf16,
 //              128-byte-swizzled staging tile, TMA store.
-// Accumulators are double-buffered in TMEM when they fit, so the epilogue of one
-// tile overlaps the main loop of the next.
+// Accumulators are double-buffered in TMEM (for 256-column FP4 tiles the two
+// buffers share one 64-column slab), so the epilogue of one tile overlaps the main
+// loop of the next.
 // Every wait is bounded by a deadline; on expiry the kernel records
 // QL_ERR_TIMEOUT in the device status word, drains its own copies and MMAs,
 // frees TMEM and returns.
@@ -29,6 +30,7 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "internal.h"
@@ -74,8 +76,13 @@ struct Cfg {
   static constexpr int STAGES_FIT = (kSmemLimit - RESERVED) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
   static constexpr int SF_COLS = FP4 ? 16 + 4 * NA * 4 : 0;
-  static constexpr int NACC = (2 * BN + SF_COLS <= kTmemCols) ? 2 : 1;
-  static constexpr int SFA_COL = NACC * BN;
+  // Two accumulator buffers. When two full BN-column buffers and the scale columns
+  // do not fit in TMEM (BN = 256 with scales), the second buffer starts 64 columns
+  // early and the two share one 64-column slab: the epilogue drains that slab
+  // first and hands the buffer back right after it.
+  static constexpr bool OVERLAP = (2 * BN + SF_COLS > kTmemCols);
+  static constexpr int ACC_STRIDE = OVERLAP ? BN - 64 : BN;  // column of buffer 1
+  static constexpr int SFA_COL = ACC_STRIDE + BN;
   static constexpr int SFB_COL = SFA_COL + 16;
   static constexpr int SMEM = RESERVED + STAGES * STAGE_BYTES;
   static constexpr int TILE_M = kRowsPerCta * CG;
@@ -85,7 +92,8 @@ struct Cfg {
       FP4 ? ((1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(TILE_M >> 4) << 24))
           : ((1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(TILE_M >> 4) << 24));
   static_assert(STAGES >= 2, "shared memory too small for two stages");
-  static_assert(NACC * BN + SF_COLS <= kTmemCols, "TMEM budget");
+  static_assert(SFA_COL + SF_COLS <= kTmemCols, "TMEM budget");
+  static_assert(!OVERLAP || BN == 256, "only the 256-column tile shares a slab");
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "tile width");
   static_assert(CG == 1 || CG == 2, "one SM or a CTA pair");
   static_assert(B_ROWS % 8 == 0, "B half must be whole 8-row core groups");
@@ -263,12 +271,15 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     bool ok = true;
     bool issued_any = false;
     for (int tile = group; ok && tile < args.total_tiles; tile += ngroups) {
-      if (!warp_wait_bounded(&tempty_bar[acc], acc_phase ^ 1u, deadline)) {
+      // with shared slabs one barrier pair orders consecutive tiles (the next
+      // tile's MMAs wait for this tile's shared slab); otherwise one per buffer
+      const int bi = C::OVERLAP ? 0 : acc;
+      if (!warp_wait_bounded(&tempty_bar[bi], acc_phase ^ 1u, deadline)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::ACC_STRIDE);
       for (int kt = 0; kt < args.num_k_tiles; ++kt) {
         if (!warp_wait_bounded(&full_bar[stage], phase, deadline)) {
           ok = false;
@@ -338,17 +349,13 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
       if (!ok) break;
       if (elect_one()) {  // accumulator ready for the epilogue (of both CTAs)
         if constexpr (CG == 2)
-          tc_commit_pair(&tfull_bar[acc], 0x3);
+          tc_commit_pair(&tfull_bar[bi], 0x3);
         else
-          tc_commit(&tfull_bar[acc]);
+          tc_commit(&tfull_bar[bi]);
       }
       __syncwarp();
-      if (C::NACC == 2) {
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
-      } else {
-        acc_phase ^= 1u;
-      }
+      acc ^= 1;
+      if (C::OVERLAP || acc == 0) acc_phase ^= 1u;
     }
     if (!ok) {
       record_timeout(args.status);
@@ -376,7 +383,8 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     for (int tile = group; tile < args.total_tiles; tile += ngroups) {
       const int m_blk = tile % args.tiles_m;
       const int n_blk = tile / args.tiles_m;
-      if (!warp_wait_bounded(&tfull_bar[acc], acc_phase, deadline)) {
+      const int bi = C::OVERLAP ? 0 : acc;
+      if (!warp_wait_bounded(&tfull_bar[bi], acc_phase, deadline)) {
         record_timeout(args.status);
         break;
       }
@@ -386,18 +394,23 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
       float row_scale = 1.0f;
       if constexpr (!FP4) row_scale = (m < args.M) ? __ldg(args.scale_a + m) : 0.0f;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                             static_cast<uint32_t>(acc * BN);
+                             static_cast<uint32_t>(acc * C::ACC_STRIDE);
 #pragma unroll 1
-      for (int sl = 0; sl < BN / 64; ++sl) {
+      for (int it = 0; it < BN / 64; ++it) {
+        // slab order: with shared slabs, buffer 0 drains its last slab (the shared
+        // one) first; otherwise slabs go in order
+        const int sl = (C::OVERLAP && acc == 0) ? (it + BN / 64 - 1) % (BN / 64) : it;
         uint32_t r[64];
         __syncwarp();  // tcgen05.ld is warp-collective
         tmem_ld_32x32b_x32(tbase + sl * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
         tmem_ld_32x32b_x32(tbase + sl * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
         tmem_ld_wait();
-        if (sl == BN / 64 - 1) {  // all columns read: hand the buffer back early
+        // hand the buffer back once the MMA can no longer overwrite unread columns:
+        // after the shared slab, or after the last slab
+        if (it == (C::OVERLAP ? 0 : BN / 64 - 1)) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(tempty_bar0 + acc * 8u);
+          if (lane == 0) mbar_arrive_cluster(tempty_bar0 + bi * 8u);
         }
         const int n0 = n_blk * BN + sl * 64;
         if (n0 >= args.N) continue;  // warp-uniform
@@ -452,12 +465,8 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
           }
         }
       }
-      if (C::NACC == 2) {
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
-      } else {
-        acc_phase ^= 1u;
-      }
+      acc ^= 1;
+      if (C::OVERLAP || acc == 0) acc_phase ^= 1u;
     }
     if (lane == 0) bulk_wait_group_all();  // outstanding stores complete before exit
   }
@@ -621,9 +630,31 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
 
 }  // namespace
 
+namespace {
+std::atomic<int> g_force_bn{0};
+std::atomic<int> g_force_cg{0};
+}  // namespace
+
+bool set_tile_override(int bn, int cg) {
+  if (bn == 0) {
+    g_force_bn.store(0);
+    g_force_cg.store(0);
+    return true;
+  }
+  if ((bn != 128 && bn != 192 && bn != 256) || (cg != 1 && cg != 2)) return false;
+  g_force_cg.store(cg);
+  g_force_bn.store(bn);
+  return true;
+}
+
 GemmConfig choose_config(bool fp4, int64_t M, int64_t N) {
   (void)fp4;
   GemmConfig c{};
+  if (g_force_bn.load() != 0) {
+    c.bn = g_force_bn.load();
+    c.cg = g_force_cg.load();
+    return c;
+  }
   c.cg = M >= 512 ? 2 : 1;
   c.bn = 128;
   if (N % 192 == 0 && N >= 1536) c.bn = 192;

@@ -36,6 +36,7 @@ struct GemmProblem {
 };
 
 GemmConfig choose_config(bool fp4, int64_t M, int64_t N);
+bool set_tile_override(int bn, int cg);  // bn == 0 restores the automatic choice
 cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream);
 
 cudaError_t launch_nvfp4_quantize_rowmajor(const void* x, int64_t M, int64_t K, const float* g,

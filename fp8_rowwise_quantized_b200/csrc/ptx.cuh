@@ -365,6 +365,30 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&v)[8]) {
   return r;
 }
 
+// Exact value of an E4M3 code (low byte of `code`), through the hardware
+// E4M3 -> f16 conversion (every E4M3 value is exact in f16) and f16 -> f32.
+__device__ __forceinline__ float e4m3_to_float(uint32_t code) {
+  float f;
+  asm("{\n\t.reg .b16 c;\n\t.reg .b32 h2;\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.u16.u32 c, %1;\n\t"
+      "cvt.rn.f16x2.e4m3x2 h2, c;\n\t"
+      "mov.b32 {lo, hi}, h2;\n\t"
+      "cvt.f32.f16 %0, lo;\n\t}"
+      : "=f"(f)
+      : "r"(code & 0xFFu));
+  return f;
+}
+
+// Largest magnitude of the 8 bf16 values in four packed words, as an fp32 value:
+// sign bits cleared, then unsigned 16-bit maxima (non-negative floats order like
+// their bit patterns).
+__device__ __forceinline__ float bf16x8_amax(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
+  const uint32_t m = __vmaxu2(__vmaxu2(w0 & 0x7FFF7FFFu, w1 & 0x7FFF7FFFu),
+                              __vmaxu2(w2 & 0x7FFF7FFFu, w3 & 0x7FFF7FFFu));
+  const uint32_t hi = m >> 16, lo = m & 0xFFFFu;
+  return __uint_as_float((hi > lo ? hi : lo) << 16);
+}
+
 // Exact value of an E4M3 code with a clear sign bit (used for block scales).
 __device__ __forceinline__ float e4m3_positive_value(uint32_t code) {
   uint32_t e = (code >> 3) & 0xF, m = code & 0x7;

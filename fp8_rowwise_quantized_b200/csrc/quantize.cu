@@ -26,107 +26,76 @@ __device__ __forceinline__ uint4 ldg16(const void* p) {
   return __ldg(reinterpret_cast<const uint4*>(p));
 }
 
-// Quantize one 16-element block held as 8 packed bf16 pairs. Returns the E4M3
-// scale code in *scale_code and the 8 packed code bytes in (lo, hi).
-// Arithmetic (each step one fp32 rounding): sf = amax * c; s = E4M3(sf);
-// d = value(s) * g; d == 0 -> zero codes; else codes = E2M1(x * (1/d)).
-__device__ __forceinline__ void nvfp4_block(const uint32_t (&w)[8], float c, float g,
-                                            uint32_t* scale_code, uint32_t* lo, uint32_t* hi) {
-  float v[16];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    v[2 * i] = bf16_lo(w[i]);
-    v[2 * i + 1] = bf16_hi(w[i]);
-  }
-  float amax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-  const float sf = __fmul_rn(amax, c);
-  const uint32_t s = cvt_e4m3x4(sf, 0.0f, 0.0f, 0.0f) & 0xFFu;
-  const float d = __fmul_rn(e4m3_positive_value(s), g);
-  *scale_code = s;
-  if (d == 0.0f) {
-    *lo = 0u;
-    *hi = 0u;
-    return;
-  }
-  const float inv = __frcp_rn(d);
-  float a[8], b[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    a[i] = __fmul_rn(v[i], inv);
-    b[i] = __fmul_rn(v[8 + i], inv);
-  }
-  *lo = cvt_e2m1x8(a);
-  *hi = cvt_e2m1x8(b);
-}
-
-// One warp per (row r, 1024-element segment of K): four 256-element slices, each
-// loaded as one fully coalesced 512-byte warp access (lane l holds elements
-// 8l..8l+7 of the slice). A 16-element block is held by a lane pair; its amax is
-// combined with one shuffle. Each lane writes its 8 codes as one 32-bit word
-// (128 contiguous bytes per warp and slice); lanes 0, 8, 16, 24 gather the four
-// block scales of one 64-element group and write them as one 32-bit word.
+// One warp per (row r, 1024-element segment of K), in two 512-element slices: in
+// each slice lane l owns the 16-element block l (two 16-byte loads; the warp's
+// loads cover 1 KB contiguously), so each block's scale arithmetic runs once.
+// Each lane writes its 16 codes as one 8-byte word (256 contiguous bytes per warp
+// and slice); lanes 0, 4, ..., 28 gather the scales of four consecutive blocks
+// (one 64-element group) and write them as one 32-bit word.
 //   x  bf16 [M, K]; xq uint8 [M, K/2]
 //   SF_MMA == false: xs uint8 [M, K/16] row-major (only blocks inside K)
 //   SF_MMA == true:  xs in the atom layout over rows padded to 128 and KG groups
 //                    of 64 (padding written as zero scales)
 template <bool SF_MMA>
-__device__ __forceinline__ void nvfp4_quantize_segment(int64_t warp_id, int lane,
-                                                       const uint16_t* __restrict__ x, int64_t M,
-                                                       int64_t K, float g, float c,
+__device__ __forceinline__ void nvfp4_quantize_segment(uint32_t warp_id, int lane,
+                                                       const uint16_t* __restrict__ x, int M,
+                                                       int K, float g, float c,
                                                        uint8_t* __restrict__ xq,
-                                                       uint8_t* __restrict__ xs, int64_t rows_total,
-                                                       int64_t segs, int64_t KG) {
+                                                       uint8_t* __restrict__ xs, uint32_t rows_total,
+                                                       uint32_t segs, int KG) {
   if (warp_id >= rows_total * segs) return;  // warp-uniform
-  const int64_t r = warp_id / segs;
-  const int64_t seg = warp_id % segs;
-  const int64_t nblk = K / 16;
+  const int r = static_cast<int>(warp_id / segs);
+  const int seg = static_cast<int>(warp_id - static_cast<uint32_t>(r) * segs);
+  const int nblk = K >> 4;
+  const uint16_t* xr = x + static_cast<int64_t>(r) * K;
+  uint8_t* qr = xq + static_cast<int64_t>(r) * (K >> 1);
   uint4 raw[4];
-  bool valid[4];
+  bool valid[2];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int64_t e = seg * 1024 + i * 256 + lane * 8;
-    valid[i] = (r < M) && (e < K);  // K % 16 == 0: a lane pair is valid together
-    raw[i] = valid[i] ? ldg16(x + r * K + e) : make_uint4(0u, 0u, 0u, 0u);
+  for (int i = 0; i < 2; ++i) {
+    const int e = seg * 1024 + i * 512 + lane * 16;
+    valid[i] = (r < M) && (e < K);  // K % 16 == 0: a block is inside or outside as a whole
+    raw[2 * i] = valid[i] ? ldg16(xr + e) : make_uint4(0u, 0u, 0u, 0u);
+    raw[2 * i + 1] = valid[i] ? ldg16(xr + e + 8) : make_uint4(0u, 0u, 0u, 0u);
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
-    float v[8];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      v[2 * j] = bf16_lo(w[j]);
-      v[2 * j + 1] = bf16_hi(w[j]);
-    }
-    float amax = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[j]));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+  for (int i = 0; i < 2; ++i) {
+    const uint4 u = raw[2 * i], v = raw[2 * i + 1];
+    const float amax = fmaxf(bf16x8_amax(u.x, u.y, u.z, u.w), bf16x8_amax(v.x, v.y, v.z, v.w));
     const float sf = __fmul_rn(amax, c);
     const uint32_t s = cvt_e4m3x4(sf, 0.0f, 0.0f, 0.0f) & 0xFFu;
-    const float d = __fmul_rn(e4m3_positive_value(s), g);
-    uint32_t codes = 0u;
+    const float d = __fmul_rn(e4m3_to_float(s), g);
+    uint2 codes = make_uint2(0u, 0u);
     if (d != 0.0f) {
       const float inv = __frcp_rn(d);
-      float a[8];
+      const uint32_t w[8] = {u.x, u.y, u.z, u.w, v.x, v.y, v.z, v.w};
+      float a[8], b[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) a[j] = __fmul_rn(v[j], inv);
-      codes = cvt_e2m1x8(a);
+      for (int j = 0; j < 4; ++j) {
+        a[2 * j] = __fmul_rn(bf16_lo(w[j]), inv);
+        a[2 * j + 1] = __fmul_rn(bf16_hi(w[j]), inv);
+        b[2 * j] = __fmul_rn(bf16_lo(w[4 + j]), inv);
+        b[2 * j + 1] = __fmul_rn(bf16_hi(w[4 + j]), inv);
+      }
+      codes = make_uint2(cvt_e2m1x8(a), cvt_e2m1x8(b));
     }
-    const int64_t e = seg * 1024 + i * 256 + lane * 8;
-    if (valid[i]) *reinterpret_cast<uint32_t*>(xq + r * (K / 2) + e / 2) = codes;
-    // scales of blocks (lane/2) .. : gather 4 consecutive blocks into lane % 8 == 0
-    const uint32_t s1 = __shfl_down_sync(0xffffffffu, s, 2);
-    const uint32_t s2 = __shfl_down_sync(0xffffffffu, s, 4);
-    const uint32_t s3 = __shfl_down_sync(0xffffffffu, s, 6);
-    if ((lane & 7) == 0) {
+    const int e = seg * 1024 + i * 512 + lane * 16;
+    if (valid[i]) *reinterpret_cast<uint2*>(qr + (e >> 1)) = codes;
+    // gather the scales of blocks lane .. lane+3 into lanes 0, 4, ..., 28
+    const uint32_t s1 = __shfl_down_sync(0xffffffffu, s, 1);
+    const uint32_t s2 = __shfl_down_sync(0xffffffffu, s, 2);
+    const uint32_t s3 = __shfl_down_sync(0xffffffffu, s, 3);
+    if ((lane & 3) == 0) {
       const uint32_t word = s | (s1 << 8) | (s2 << 16) | (s3 << 24);
-      const int64_t kg = (seg * 1024 + i * 256) / 64 + lane / 8;
+      const int kg = seg * 16 + i * 8 + (lane >> 2);
       if (SF_MMA) {
-        if (kg < KG) *reinterpret_cast<uint32_t*>(xs + sf_act_word_offset(r, kg, KG)) = word;
+        if (kg < KG) {
+          const int rr = r & 127;
+          const int off = ((r >> 7) * KG + kg) * kSfAtomBytes + (rr & 31) * 16 + (rr >> 5) * 4;
+          *reinterpret_cast<uint32_t*>(xs + off) = word;
+        }
       } else if (r < M && 4 * kg < nblk) {
-        uint8_t* sr = xs + r * nblk + kg * 4;
+        uint8_t* sr = xs + static_cast<int64_t>(r) * nblk + kg * 4;
         if (4 * kg + 4 <= nblk && (reinterpret_cast<uintptr_t>(sr) & 3) == 0) {
           *reinterpret_cast<uint32_t*>(sr) = word;
         } else {
@@ -141,12 +110,12 @@ __device__ __forceinline__ void nvfp4_quantize_segment(int64_t warp_id, int lane
 
 template <bool SF_MMA>
 __global__ void __launch_bounds__(kQuantThreads)
-nvfp4_quantize_kernel(const uint16_t* __restrict__ x, int64_t M, int64_t K,
+nvfp4_quantize_kernel(const uint16_t* __restrict__ x, int M, int K,
                       const float* __restrict__ g_ptr, uint8_t* __restrict__ xq,
-                      uint8_t* __restrict__ xs, int64_t rows_total, int64_t segs, int64_t KG) {
+                      uint8_t* __restrict__ xs, uint32_t rows_total, uint32_t segs, int KG) {
   const float g = __ldg(g_ptr);
   const float c = __frcp_rn(__fmul_rn(6.0f, g));
-  const int64_t warp_id = static_cast<int64_t>(blockIdx.x) * (kQuantThreads / 32) + threadIdx.x / 32;
+  const uint32_t warp_id = blockIdx.x * (kQuantThreads / 32) + threadIdx.x / 32;
   nvfp4_quantize_segment<SF_MMA>(warp_id, threadIdx.x % 32, x, M, K, g, c, xq, xs, rows_total,
                                  segs, KG);
 }
@@ -203,28 +172,29 @@ __device__ __forceinline__ void nvfp4_weight_scale_atoms(int64_t job, int tid,
 
 // The prologue of nvfp4_linear in one launch: blocks [0, act_blocks) quantize the
 // activations into the workspace (codes row-major, scales in atom layout), the
-// remaining blocks lay out the weight scales for the GEMM's tile width. It lets
-// the dependent GEMM launch start its set-up right away; the GEMM reads the
-// workspace only after this grid has completed.
+// remaining blocks lay out the weight scales for the GEMM's tile width. Each block
+// allows the dependent GEMM launch once its own work is issued, so the GEMM's
+// set-up overlaps the prologue's tail (the GEMM reads the workspace only after this
+// grid has completed); triggering earlier would let resident GEMM CTAs take the
+// shared memory the remaining prologue blocks need.
 __global__ void __launch_bounds__(kQuantThreads)
-nvfp4_prologue_kernel(const uint16_t* __restrict__ x, int64_t M, int64_t K,
+nvfp4_prologue_kernel(const uint16_t* __restrict__ x, int M, int K,
                       const float* __restrict__ g_ptr, uint8_t* __restrict__ xq,
-                      uint8_t* __restrict__ xs, int64_t rows_total, int64_t segs, int64_t KG,
-                      int64_t act_blocks, const uint8_t* __restrict__ ws, int64_t N, int bn,
+                      uint8_t* __restrict__ xs, uint32_t rows_total, uint32_t segs, int KG,
+                      uint32_t act_blocks, const uint8_t* __restrict__ ws, int64_t N, int bn,
                       int na, int64_t n_tiles, uint8_t* __restrict__ wout) {
   __shared__ uint32_t tile[128][kWsGroups + 1];
-  grid_dependents_launch();
   if (blockIdx.x < act_blocks) {
     const float g = __ldg(g_ptr);
     const float c = __frcp_rn(__fmul_rn(6.0f, g));
-    const int64_t warp_id =
-        static_cast<int64_t>(blockIdx.x) * (kQuantThreads / 32) + threadIdx.x / 32;
+    const uint32_t warp_id = blockIdx.x * (kQuantThreads / 32) + threadIdx.x / 32;
     nvfp4_quantize_segment<true>(warp_id, threadIdx.x % 32, x, M, K, g, c, xq, xs, rows_total,
                                  segs, KG);
   } else {
-    nvfp4_weight_scale_atoms(static_cast<int64_t>(blockIdx.x) - act_blocks, threadIdx.x, ws, N, K,
+    nvfp4_weight_scale_atoms(static_cast<int64_t>(blockIdx.x - act_blocks), threadIdx.x, ws, N, K,
                              bn, na, n_tiles, KG, wout, tile);
   }
+  grid_dependents_launch();
 }
 
 // FP8 row-wise: one warp per row.
@@ -255,7 +225,6 @@ template <bool CACHED>
 __global__ void __launch_bounds__(kQuantThreads)
 fp8r_quantize_rows_kernel(const uint16_t* __restrict__ x, int64_t M, int64_t K,
                           uint8_t* __restrict__ xq, float* __restrict__ x_scale) {
-  grid_dependents_launch();
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (kQuantThreads / 32) + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   if (row >= M) return;
@@ -293,6 +262,7 @@ fp8r_quantize_rows_kernel(const uint16_t* __restrict__ x, int64_t M, int64_t K,
       *reinterpret_cast<uint2*>(qr + ch * 8) =
           scale == 0.0f ? make_uint2(0u, 0u) : fp8r_encode8(ldg16(xr + ch * 8), inv);
   }
+  grid_dependents_launch();  // the dependent GEMM may start its set-up
 }
 
 // amax(|x|) over n bf16 values into *slot (as the bit pattern of a non-negative
@@ -339,7 +309,8 @@ cudaError_t launch_nvfp4_quantize_rowmajor(const void* x, int64_t M, int64_t K, 
   const int64_t segs = ceil_div64(K, 1024);
   const int warps_per_block = kQuantThreads / 32;
   nvfp4_quantize_kernel<false><<<grid_for(M * segs, warps_per_block), kQuantThreads, 0, s>>>(
-      static_cast<const uint16_t*>(x), M, K, g, xq, xs, M, segs, ceil_div64(K, 64));
+      static_cast<const uint16_t*>(x), static_cast<int>(M), static_cast<int>(K), g, xq, xs,
+      static_cast<uint32_t>(M), static_cast<uint32_t>(segs), static_cast<int>(ceil_div64(K, 64)));
   return cudaGetLastError();
 }
 
@@ -355,9 +326,10 @@ cudaError_t launch_nvfp4_prologue(const void* x, int64_t M, int64_t K, const uin
   const int64_t act_blocks = grid_for(rows * segs, kQuantThreads / 32);
   const int64_t w_blocks = n_tiles * na * ceil_div64(KG, kWsGroups);
   nvfp4_prologue_kernel<<<static_cast<unsigned>(act_blocks + w_blocks), kQuantThreads, 0, s>>>(
-      static_cast<const uint16_t*>(x), M, K, input_scale, workspace + L.codes_off,
-      workspace + L.act_sf_off, rows, segs, KG, act_blocks, w_scale, N, bn, na, n_tiles,
-      workspace + L.wgt_sf_off);
+      static_cast<const uint16_t*>(x), static_cast<int>(M), static_cast<int>(K), input_scale,
+      workspace + L.codes_off, workspace + L.act_sf_off, static_cast<uint32_t>(rows),
+      static_cast<uint32_t>(segs), static_cast<int>(KG), static_cast<uint32_t>(act_blocks),
+      w_scale, N, bn, na, n_tiles, workspace + L.wgt_sf_off);
   return cudaGetLastError();
 }
 

@@ -184,6 +184,12 @@ int ql_read_device_status(int* status);
  * GEMM kernels (default 2000 ms; 0 restores the default). Host-side settings. */
 void ql_set_fault_injection(int enable, int timeout_ms);
 
+/* Tuning override of the GEMM tile shape for later calls (both schemes): output
+ * tiles of (128 * cg) rows x bn columns, cg = 2 running each MMA across a pair of
+ * SMs. bn in {128, 192, 256}, cg in {1, 2}; bn = 0 restores the automatic choice.
+ * Returns QL_OK or QL_ERR_INVALID_ARG. Workspace sizes already cover every tile. */
+int ql_set_tile_override(int bn, int cg);
+
 /* Text of a status code, and of the last CUDA error recorded by this thread. */
 const char* ql_status_string(int status);
 const char* ql_last_error_message(void);

@@ -145,3 +145,34 @@ def test_fp8r_gemm_from_prequantized_matches_linear():
     y2 = q.fp8r_linear_gemm(xq, xs, d["w"], d["w_scale"], bias=d["bias"])
     torch.cuda.synchronize()
     assert torch.equal(y1, y2)
+
+
+TILES = [(128, 1), (192, 1), (256, 1), (128, 2), (192, 2), (256, 2)]
+
+
+@pytest.mark.parametrize("bn,cg", TILES)
+def test_nvfp4_linear_every_tile_config(bn, cg):
+    # ragged in M, N and K for every tile width and for one SM or a CTA pair,
+    # including the 256-column tile whose two TMEM buffers share a slab
+    try:
+        q.set_tile_override(bn, cg)
+        run_nvfp4(Nvfp4Case(700, 1280, 1000, seed=bn + cg, bias=True))
+        run_nvfp4(Nvfp4Case(1536, 3072, 3072, seed=3), sample_rows(1536, 8, seed=bn))
+    finally:
+        q.set_tile_override(0, 0)
+
+
+@pytest.mark.parametrize("bn,cg", TILES)
+def test_fp8r_linear_every_tile_config(bn, cg):
+    try:
+        q.set_tile_override(bn, cg)
+        run_fp8r(Fp8rCase(700, 1024, 1000, seed=bn * cg, bias=True))
+    finally:
+        q.set_tile_override(0, 0)
+
+
+def test_tile_override_rejects_bad_values():
+    with pytest.raises(q.QLinearError):
+        q.set_tile_override(96, 1)
+    with pytest.raises(q.QLinearError):
+        q.set_tile_override(128, 3)
