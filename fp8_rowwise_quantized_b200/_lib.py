@@ -34,6 +34,8 @@ SIGNATURES = {
     "nvfp4_linear_workspace_layout": (C.c_int, [_i64, _i64, _i64, C.POINTER(C.c_size_t),
                                                 C.POINTER(C.c_size_t), C.POINTER(C.c_size_t)]),
     "nvfp4_global_scale": (C.c_int, [_vp, _i64, _f32p, _vp]),
+    "nvfp4_linear_noalloc": (C.c_int, [_vp, _i64, _i64, _u8p, _u8p, _i64, _f32p, _f32p, _f32p,
+                                       _vp, _vp]),
     "fp8r_quantize_rows": (C.c_int, [_vp, _i64, _i64, _u8p, _f32p, _vp]),
     "fp8r_linear_workspace_size": (C.c_size_t, [_i64, _i64, _i64]),
     "fp8r_linear": (C.c_int, [_vp, _i64, _i64, _u8p, _f32p, _i64, _f32p, _vp, _vp, _sz, _vp]),
@@ -86,6 +88,6 @@ def load():
 def check(fn_name, status):
     if status != QL_OK:
         detail = ""
-        if status in (QL_ERR_LAUNCH, QL_ERR_DEVICE, QL_ERR_SHAPE):
+        if status in (QL_ERR_LAUNCH, QL_ERR_DEVICE, QL_ERR_SHAPE, QL_ERR_WORKSPACE):
             detail = load().ql_last_error_message().decode()
         raise QLinearError(fn_name, status, detail)

@@ -86,6 +86,10 @@ bool fp8r_shape_ok(int64_t M, int64_t K, int64_t N) {
 
 }  // namespace
 
+void ql::set_error_text(const char* text) {
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s", text);
+}
+
 extern "C" {
 
 const char* ql_status_string(int status) {

@@ -49,4 +49,7 @@ cudaError_t launch_fp8r_quantize_rows(const void* x, int64_t M, int64_t K, uint8
 cudaError_t launch_global_scale(const void* x, int64_t n, float* out, cudaStream_t s);
 cudaError_t launch_encode(const float* in, uint8_t* out, int64_t n, bool fp4, cudaStream_t s);
 
+// Sets the text ql_last_error_message() returns on this thread.
+void set_error_text(const char* text);
+
 }  // namespace ql

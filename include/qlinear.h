@@ -127,6 +127,26 @@ int nvfp4_linear_workspace_layout(int64_t M, int64_t K, int64_t N, size_t* codes
  *   x bf16 [n]; out fp32 scalar (device, overwritten). Requires n >= 1. */
 int nvfp4_global_scale(const void* x, int64_t n, float* out, ql_stream_t stream);
 
+/* nvfp4_linear without a caller workspace. No counterpart in the BFL page; it is
+ * for callers that cannot allocate device memory themselves: a plugin whose host
+ * application owns all device memory and forbids allocations on its hot path, a
+ * serving loop that must never enter the allocator (an allocation can synchronise
+ * the device or fail under memory pressure), or a C caller with no memory manager.
+ * Same arguments and results as nvfp4_linear, minus the workspace: the scratch
+ * lives in one fixed 32 MiB array in device memory inside this library, held by
+ * every GPU that loads it until the process exits. Problems that need more
+ * scratch than that (nvfp4_linear_workspace_size(M, K, N) > 32 MiB) are rejected
+ * with QL_ERR_WORKSPACE and a message in ql_last_error_message(). The call
+ * allocates and frees nothing. The first call on each device looks up the
+ * array's device address (cudaGetSymbolAddress) and keeps it; make that first
+ * call before any stream capture. All calls on a device share the array and each
+ * rewrites what it reads, so nothing needs clearing between calls, but calls whose
+ * kernels overlap on the GPU (unordered streams) race on it. */
+int nvfp4_linear_noalloc(const void* x, int64_t M, int64_t K,
+                         const uint8_t* w, const uint8_t* w_scale, int64_t N,
+                         const float* weight_scale_2, const float* input_scale,
+                         const float* bias, void* y, ql_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* fp8r (FP8 row-wise)                                                       */
 /* ------------------------------------------------------------------------ */
