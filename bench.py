@@ -395,6 +395,11 @@ def run_ours(args):
     layer.prologue()
     gemm_ms, _ = time_events(layer.gemm, roof_steps, 3, flush, stream)
     prol_ms, _ = time_events(layer.prologue, roof_steps, 3, flush, stream)
+    xq_buf = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
+    xs_buf = torch.empty((M, K // 16), dtype=torch.uint8, device=device)
+    quant_ms, _ = time_events(lambda: q.nvfp4_quantize_act(layer.x, layer.gx, xq_buf, xs_buf),
+                              roof_steps, 3, flush, stream)
+    quant_bytes = 2 * M * K + M * K // 2 + M * K // 16
     gemm_tflops = flops / (gemm_ms / 1e3) / 1e12
     prologue_bytes = 2 * M * K + M * K // 2 + M * K // 16 + 2 * (N * K // 16)
     roofline = {
@@ -408,6 +413,8 @@ def run_ours(args):
         "prologue_us": prol_ms * 1e3,
         "prologue_gbs": prologue_bytes / (prol_ms / 1e3) / 1e9,
         "prologue_hbm_frac": prologue_bytes / (prol_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+        "quantize_act_us": quant_ms * 1e3,
+        "quantize_act_gbs": quant_bytes / (quant_ms / 1e3) / 1e9,
         "frac_of_nominal_9pf": gemm_tflops / 9000.0,
         "step_frac_of_fp4_peak": value / world / fp4_peak,
     }
@@ -499,7 +506,8 @@ def run_ours(args):
 def run_profile(args):
     """Short fixed sequence for profilers: `--profile <piece>` runs `--steps` calls
     of one piece of the headline workload (no flushes, no timing): `step`,
-    `prologue`, `gemm`, `fp8r_step`, `fp8r_quant` or `fp8r_gemm`."""
+    `prologue`, `gemm`, `quant` (activation quantization alone), `fp8r_step`,
+    `fp8r_quant` or `fp8r_gemm`."""
     import torch
     torch.cuda.set_device(0)
     device = torch.device("cuda", 0)
@@ -511,7 +519,10 @@ def run_profile(args):
     else:
         L = Nvfp4Layer(M, K, N, False, device)
         L.prologue()
-        fn = {"step": L.step, "prologue": L.prologue, "gemm": L.gemm}[args.profile]
+        xq = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
+        xs = torch.empty((M, K // 16), dtype=torch.uint8, device=device)
+        fn = {"step": L.step, "prologue": L.prologue, "gemm": L.gemm,
+              "quant": lambda: L.q.nvfp4_quantize_act(L.x, L.gx, xq, xs)}[args.profile]
     for _ in range(args.steps):
         fn()
     torch.cuda.synchronize()
@@ -530,8 +541,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-variants", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["step", "prologue", "gemm", "fp8r_step", "fp8r_quant",
-                                          "fp8r_gemm"], default=None,
+    ap.add_argument("--profile", choices=["step", "prologue", "gemm", "quant", "fp8r_step",
+                                          "fp8r_quant", "fp8r_gemm"], default=None,
                     help="run a short fixed sequence for a profiler instead of the benchmark")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps

@@ -46,6 +46,10 @@ constexpr int kThreads = 192;
 constexpr int kSmemLimit = 232448;  // 227 KB opt-in per block
 constexpr int kTmemCols = 512;
 constexpr int kEpiBufBytes = 32 * 128;  // 32 rows x 64 bf16 (128-byte swizzled), one TMA box
+// One staging buffer per epilogue warp: the shared memory goes to one more
+// pipeline stage instead (the TMA store reads a 4 KB buffer long before the warp
+// has its next slab ready).
+constexpr int kEpiBufsPerWarp = 1;
 
 struct GemmArgs {
   int M, N, K;
@@ -71,7 +75,8 @@ struct Cfg {
   static constexpr int SFA_BYTES = FP4 ? 4 * kSfAtomBytes : 0;       // 4 K-groups x 1 atom
   static constexpr int SFB_BYTES = FP4 ? 4 * NA * kSfAtomBytes : 0;  // 4 K-groups x NA atoms
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  static constexpr int EPI_BYTES = 4 * 2 * kEpiBufBytes;             // 4 warps x 2 buffers
+  static constexpr int EPI_BUFS = kEpiBufsPerWarp;
+  static constexpr int EPI_BYTES = 4 * EPI_BUFS * kEpiBufBytes;      // 4 epilogue warps
   static constexpr int RESERVED = 1024 /*alignment*/ + 1024 /*barriers*/ + EPI_BYTES;
   static constexpr int STAGES_FIT = (kSmemLimit - RESERVED) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
@@ -374,7 +379,7 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     // ------------------------------------------------------------ epilogue
     const int q = warp % 4;  // TMEM lane quadrant this warp may access
     const int row_in_tile = static_cast<int>(rank) * kRowsPerCta + q * 32 + lane;
-    uint8_t* stage = smem_epi + (warp - 2) * 2 * kEpiBufBytes;
+    uint8_t* stage = smem_epi + (warp - 2) * C::EPI_BUFS * kEpiBufBytes;
     int buf = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -437,7 +442,12 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                                           __fmaf_rn(__uint_as_float(r[4 * i + 3]), s4.w, b4.w));
           }
           uint8_t* sbuf = stage + buf * kEpiBufBytes;
-          if (lane == 0) bulk_wait_group_read<1>();  // the store that used this buffer has read it
+          if (lane == 0) {  // the store that last used this buffer has read it
+            if constexpr (C::EPI_BUFS == 1)
+              bulk_wait_group_read<0>();
+            else
+              bulk_wait_group_read<1>();
+          }
           __syncwarp();
 #pragma unroll
           for (int j = 0; j < 8; ++j)
@@ -449,7 +459,7 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
             tma_store_2d(&tmap_y, sbuf, n0, row0);
             bulk_commit_group();
           }
-          buf ^= 1;
+          buf = (buf + 1) % C::EPI_BUFS;
         } else {
           if (m >= args.M) continue;
           uint16_t* yrow = args.y + static_cast<int64_t>(m) * args.N;

@@ -26,41 +26,50 @@ __device__ __forceinline__ uint4 ldg16(const void* p) {
   return __ldg(reinterpret_cast<const uint4*>(p));
 }
 
-// One warp per (row r, 1024-element segment of K), in two 512-element slices: in
-// each slice lane l owns the 16-element block l (two 16-byte loads; the warp's
-// loads cover 1 KB contiguously), so each block's scale arithmetic runs once.
-// Each lane writes its 16 codes as one 8-byte word (256 contiguous bytes per warp
-// and slice); lanes 0, 4, ..., 28 gather the scales of four consecutive blocks
-// (one 64-element group) and write them as one 32-bit word.
+// NVFP4 quantization of (row r, 1024-element segment of K) work items. A warp
+// handles one item in two 512-element slices: in each slice lane l owns the
+// 16-element block l (two 16-byte loads; the warp's loads cover 1 KB
+// contiguously), so each block's scale arithmetic runs once. Each lane writes its
+// 16 codes as one 8-byte word (256 contiguous bytes per warp and slice); lanes 0,
+// 4, ..., 28 gather the scales of four consecutive blocks (one 64-element group)
+// and write them as one 32-bit word.
 //   x  bf16 [M, K]; xq uint8 [M, K/2]
 //   SF_MMA == false: xs uint8 [M, K/16] row-major (only blocks inside K)
 //   SF_MMA == true:  xs in the atom layout over rows padded to 128 and KG groups
 //                    of 64 (padding written as zero scales)
-template <bool SF_MMA>
-__device__ __forceinline__ void nvfp4_quantize_segment(uint32_t warp_id, int lane,
-                                                       const uint16_t* __restrict__ x, int M,
-                                                       int K, float g, float c,
-                                                       uint8_t* __restrict__ xq,
-                                                       uint8_t* __restrict__ xs, uint32_t rows_total,
-                                                       uint32_t segs, int KG) {
-  if (warp_id >= rows_total * segs) return;  // warp-uniform
-  const int r = static_cast<int>(warp_id / segs);
-  const int seg = static_cast<int>(warp_id - static_cast<uint32_t>(r) * segs);
-  const int nblk = K >> 4;
-  const uint16_t* xr = x + static_cast<int64_t>(r) * K;
-  uint8_t* qr = xq + static_cast<int64_t>(r) * (K >> 1);
+struct QuantItem {
   uint4 raw[4];
-  bool valid[2];
+};
+
+__device__ __forceinline__ void nvfp4_load_item(uint32_t item, int lane,
+                                                const uint16_t* __restrict__ x, int M, int K,
+                                                uint32_t segs, QuantItem& q) {
+  const int r = static_cast<int>(item / segs);
+  const int seg = static_cast<int>(item - static_cast<uint32_t>(r) * segs);
+  const uint16_t* xr = x + static_cast<int64_t>(r) * K;
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
     const int e = seg * 1024 + i * 512 + lane * 16;
-    valid[i] = (r < M) && (e < K);  // K % 16 == 0: a block is inside or outside as a whole
-    raw[2 * i] = valid[i] ? ldg16(xr + e) : make_uint4(0u, 0u, 0u, 0u);
-    raw[2 * i + 1] = valid[i] ? ldg16(xr + e + 8) : make_uint4(0u, 0u, 0u, 0u);
+    const bool valid = (r < M) && (e < K);  // K % 16 == 0: a block is inside or out as a whole
+    q.raw[2 * i] = valid ? ldg16(xr + e) : make_uint4(0u, 0u, 0u, 0u);
+    q.raw[2 * i + 1] = valid ? ldg16(xr + e + 8) : make_uint4(0u, 0u, 0u, 0u);
   }
+}
+
+template <bool SF_MMA>
+__device__ __forceinline__ void nvfp4_encode_item(uint32_t item, int lane, const QuantItem& q,
+                                                  int M, int K, float g, float c,
+                                                  uint8_t* __restrict__ xq,
+                                                  uint8_t* __restrict__ xs, uint32_t segs, int KG) {
+  const int r = static_cast<int>(item / segs);
+  const int seg = static_cast<int>(item - static_cast<uint32_t>(r) * segs);
+  const int nblk = K >> 4;
+  uint8_t* qr = xq + static_cast<int64_t>(r) * (K >> 1);
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
-    const uint4 u = raw[2 * i], v = raw[2 * i + 1];
+    const uint4 u = q.raw[2 * i], v = q.raw[2 * i + 1];
+    const int e = seg * 1024 + i * 512 + lane * 16;
+    const bool valid = (r < M) && (e < K);
     const float amax = fmaxf(bf16x8_amax(u.x, u.y, u.z, u.w), bf16x8_amax(v.x, v.y, v.z, v.w));
     const float sf = __fmul_rn(amax, c);
     const uint32_t s = cvt_e4m3x4(sf, 0.0f, 0.0f, 0.0f) & 0xFFu;
@@ -69,18 +78,17 @@ __device__ __forceinline__ void nvfp4_quantize_segment(uint32_t warp_id, int lan
     if (d != 0.0f) {
       const float inv = __frcp_rn(d);
       const uint32_t w[8] = {u.x, u.y, u.z, u.w, v.x, v.y, v.z, v.w};
-      float a[8], b[8];
+      float fa[8], fb[8];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        a[2 * j] = __fmul_rn(bf16_lo(w[j]), inv);
-        a[2 * j + 1] = __fmul_rn(bf16_hi(w[j]), inv);
-        b[2 * j] = __fmul_rn(bf16_lo(w[4 + j]), inv);
-        b[2 * j + 1] = __fmul_rn(bf16_hi(w[4 + j]), inv);
+        fa[2 * j] = __fmul_rn(bf16_lo(w[j]), inv);
+        fa[2 * j + 1] = __fmul_rn(bf16_hi(w[j]), inv);
+        fb[2 * j] = __fmul_rn(bf16_lo(w[4 + j]), inv);
+        fb[2 * j + 1] = __fmul_rn(bf16_hi(w[4 + j]), inv);
       }
-      codes = make_uint2(cvt_e2m1x8(a), cvt_e2m1x8(b));
+      codes = make_uint2(cvt_e2m1x8(fa), cvt_e2m1x8(fb));
     }
-    const int e = seg * 1024 + i * 512 + lane * 16;
-    if (valid[i]) *reinterpret_cast<uint2*>(qr + (e >> 1)) = codes;
+    if (valid) *reinterpret_cast<uint2*>(qr + (e >> 1)) = codes;
     // gather the scales of blocks lane .. lane+3 into lanes 0, 4, ..., 28
     const uint32_t s1 = __shfl_down_sync(0xffffffffu, s, 1);
     const uint32_t s2 = __shfl_down_sync(0xffffffffu, s, 2);
@@ -108,6 +116,27 @@ __device__ __forceinline__ void nvfp4_quantize_segment(uint32_t warp_id, int lan
   }
 }
 
+// Grid-stride loop of warps over the work items, with the next item's loads in
+// flight while the current one is encoded (the grid is one wave of resident
+// blocks, so there is no tail wave).
+template <bool SF_MMA>
+__device__ __forceinline__ void nvfp4_quantize_items(uint32_t warp_id, uint32_t nwarps, int lane,
+                                                     const uint16_t* __restrict__ x, int M, int K,
+                                                     float g, float c, uint8_t* __restrict__ xq,
+                                                     uint8_t* __restrict__ xs, uint32_t total,
+                                                     uint32_t segs, int KG) {
+  if (warp_id >= total) return;  // warp-uniform
+  QuantItem cur;
+  nvfp4_load_item(warp_id, lane, x, M, K, segs, cur);
+  for (uint32_t item = warp_id; item < total; item += nwarps) {
+    QuantItem nxt;
+    const uint32_t next = item + nwarps;
+    if (next < total) nvfp4_load_item(next, lane, x, M, K, segs, nxt);
+    nvfp4_encode_item<SF_MMA>(item, lane, cur, M, K, g, c, xq, xs, segs, KG);
+    cur = nxt;
+  }
+}
+
 template <bool SF_MMA>
 __global__ void __launch_bounds__(kQuantThreads)
 nvfp4_quantize_kernel(const uint16_t* __restrict__ x, int M, int K,
@@ -115,9 +144,10 @@ nvfp4_quantize_kernel(const uint16_t* __restrict__ x, int M, int K,
                       uint8_t* __restrict__ xs, uint32_t rows_total, uint32_t segs, int KG) {
   const float g = __ldg(g_ptr);
   const float c = __frcp_rn(__fmul_rn(6.0f, g));
-  const uint32_t warp_id = blockIdx.x * (kQuantThreads / 32) + threadIdx.x / 32;
-  nvfp4_quantize_segment<SF_MMA>(warp_id, threadIdx.x % 32, x, M, K, g, c, xq, xs, rows_total,
-                                 segs, KG);
+  constexpr uint32_t kWarps = kQuantThreads / 32;
+  nvfp4_quantize_items<SF_MMA>(blockIdx.x * kWarps + threadIdx.x / 32, gridDim.x * kWarps,
+                               threadIdx.x % 32, x, M, K, g, c, xq, xs, rows_total * segs, segs,
+                               KG);
 }
 
 // Row-major weight scales [N, K/16] -> atom layout for tiles of `bn` rows, through
@@ -170,29 +200,28 @@ __device__ __forceinline__ void nvfp4_weight_scale_atoms(int64_t job, int tid,
   }
 }
 
-// The prologue of nvfp4_linear in one launch: blocks [0, act_blocks) quantize the
-// activations into the workspace (codes row-major, scales in atom layout), the
-// remaining blocks lay out the weight scales for the GEMM's tile width. Each block
-// allows the dependent GEMM launch once its own work is issued, so the GEMM's
-// set-up overlaps the prologue's tail (the GEMM reads the workspace only after this
-// grid has completed); triggering earlier would let resident GEMM CTAs take the
-// shared memory the remaining prologue blocks need.
+// The prologue of nvfp4_linear in one launch, one wave of resident blocks: each
+// block's warps first quantize activation items (codes row-major, scales in atom
+// layout) in a grid-stride loop, then the block takes weight-scale layout jobs.
+// Each block allows the dependent GEMM launch once its own work is issued, so the
+// GEMM's set-up overlaps the prologue's tail (the GEMM reads the workspace only
+// after this grid has completed); triggering earlier would let resident GEMM CTAs
+// take the shared memory the prologue blocks need.
 __global__ void __launch_bounds__(kQuantThreads)
 nvfp4_prologue_kernel(const uint16_t* __restrict__ x, int M, int K,
                       const float* __restrict__ g_ptr, uint8_t* __restrict__ xq,
                       uint8_t* __restrict__ xs, uint32_t rows_total, uint32_t segs, int KG,
-                      uint32_t act_blocks, const uint8_t* __restrict__ ws, int64_t N, int bn,
-                      int na, int64_t n_tiles, uint8_t* __restrict__ wout) {
+                      const uint8_t* __restrict__ ws, int64_t N, int bn, int na, int64_t n_tiles,
+                      int64_t w_jobs, uint8_t* __restrict__ wout) {
   __shared__ uint32_t tile[128][kWsGroups + 1];
-  if (blockIdx.x < act_blocks) {
-    const float g = __ldg(g_ptr);
-    const float c = __frcp_rn(__fmul_rn(6.0f, g));
-    const uint32_t warp_id = blockIdx.x * (kQuantThreads / 32) + threadIdx.x / 32;
-    nvfp4_quantize_segment<true>(warp_id, threadIdx.x % 32, x, M, K, g, c, xq, xs, rows_total,
-                                 segs, KG);
-  } else {
-    nvfp4_weight_scale_atoms(static_cast<int64_t>(blockIdx.x - act_blocks), threadIdx.x, ws, N, K,
-                             bn, na, n_tiles, KG, wout, tile);
+  const float g = __ldg(g_ptr);
+  const float c = __frcp_rn(__fmul_rn(6.0f, g));
+  constexpr uint32_t kWarps = kQuantThreads / 32;
+  nvfp4_quantize_items<true>(blockIdx.x * kWarps + threadIdx.x / 32, gridDim.x * kWarps,
+                             threadIdx.x % 32, x, M, K, g, c, xq, xs, rows_total * segs, segs, KG);
+  for (int64_t job = blockIdx.x; job < w_jobs; job += gridDim.x) {
+    nvfp4_weight_scale_atoms(job, threadIdx.x, ws, N, K, bn, na, n_tiles, KG, wout, tile);
+    __syncthreads();  // the tile buffer is reused by the next job
   }
   grid_dependents_launch();
 }
@@ -304,11 +333,30 @@ inline unsigned grid_for(int64_t work, int threads) {
 
 }  // namespace
 
+// Blocks of `kernel` that fit on the current device at once (one full wave).
+template <typename Kernel>
+int64_t resident_blocks(Kernel kernel) {
+  int dev = 0, sms = 148, per_sm = 1;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kQuantThreads, 0) !=
+          cudaSuccess ||
+      per_sm < 1) {
+    cudaGetLastError();
+    per_sm = 1;
+  }
+  return static_cast<int64_t>(sms) * per_sm;
+}
+
 cudaError_t launch_nvfp4_quantize_rowmajor(const void* x, int64_t M, int64_t K, const float* g,
                                            uint8_t* xq, uint8_t* xs, cudaStream_t s) {
   const int64_t segs = ceil_div64(K, 1024);
-  const int warps_per_block = kQuantThreads / 32;
-  nvfp4_quantize_kernel<false><<<grid_for(M * segs, warps_per_block), kQuantThreads, 0, s>>>(
+  const int64_t items = M * segs;
+  static int64_t wave = 0;
+  if (wave == 0) wave = resident_blocks(nvfp4_quantize_kernel<false>);
+  const int64_t need = ceil_div64(items, kQuantThreads / 32);
+  const int64_t blocks = need < wave ? need : wave;
+  nvfp4_quantize_kernel<false><<<static_cast<unsigned>(blocks), kQuantThreads, 0, s>>>(
       static_cast<const uint16_t*>(x), static_cast<int>(M), static_cast<int>(K), g, xq, xs,
       static_cast<uint32_t>(M), static_cast<uint32_t>(segs), static_cast<int>(ceil_div64(K, 64)));
   return cudaGetLastError();
@@ -323,13 +371,17 @@ cudaError_t launch_nvfp4_prologue(const void* x, int64_t M, int64_t K, const uin
   const int64_t segs = ceil_div64(KG * 64, 1024);
   const int na = (bn + 127) / 128;
   const int64_t n_tiles = ceil_div64(N, bn);
-  const int64_t act_blocks = grid_for(rows * segs, kQuantThreads / 32);
-  const int64_t w_blocks = n_tiles * na * ceil_div64(KG, kWsGroups);
-  nvfp4_prologue_kernel<<<static_cast<unsigned>(act_blocks + w_blocks), kQuantThreads, 0, s>>>(
+  const int64_t w_jobs = n_tiles * na * ceil_div64(KG, kWsGroups);
+  static int64_t wave = 0;
+  if (wave == 0) wave = resident_blocks(nvfp4_prologue_kernel);
+  int64_t need = ceil_div64(rows * segs, kQuantThreads / 32);
+  if (need < w_jobs) need = w_jobs;
+  const int64_t blocks = need < wave ? need : wave;
+  nvfp4_prologue_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, 0, s>>>(
       static_cast<const uint16_t*>(x), static_cast<int>(M), static_cast<int>(K), input_scale,
       workspace + L.codes_off, workspace + L.act_sf_off, static_cast<uint32_t>(rows),
-      static_cast<uint32_t>(segs), static_cast<int>(KG), static_cast<uint32_t>(act_blocks),
-      w_scale, N, bn, na, n_tiles, workspace + L.wgt_sf_off);
+      static_cast<uint32_t>(segs), static_cast<int>(KG), w_scale, N, bn, na, n_tiles, w_jobs,
+      workspace + L.wgt_sf_off);
   return cudaGetLastError();
 }
 
