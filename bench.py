@@ -460,7 +460,7 @@ def run_ours(args):
         torch.cuda.empty_cache()
         # GEMM tile sweep on the headline layer: (128 * cg) x bn output tiles
         sweep = {}
-        for bn, cg in [(192, 2), (256, 2), (128, 2), (192, 1), (256, 1)]:
+        for bn, cg in [(192, 2), (224, 2), (256, 2), (128, 2), (192, 1)]:
             q.set_tile_override(bn, cg)
             try:
                 layer.prologue()

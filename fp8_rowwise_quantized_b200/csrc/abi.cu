@@ -146,7 +146,7 @@ size_t nvfp4_linear_workspace_size(int64_t M, int64_t K, int64_t N) {
   if (!nvfp4_shape_ok(M, K, N)) return 0;
   // large enough for the weight-scale layout of every tile width
   size_t need = 0;
-  for (int bn : {128, 192, 256}) {
+  for (int bn : {128, 192, 224, 256}) {
     const size_t t = ql::nvfp4_workspace(M, K, N, bn).total;
     need = t > need ? t : need;
   }
@@ -160,7 +160,7 @@ int ql_set_tile_override(int bn, int cg) {
 int nvfp4_linear_workspace_layout(int64_t M, int64_t K, int64_t N, size_t* codes_offset,
                                   size_t* act_scales_offset, size_t* weight_scales_offset) {
   if (!nvfp4_shape_ok(M, K, N)) return QL_ERR_SHAPE;
-  const ql::Nvfp4Workspace L = ql::nvfp4_workspace(M, K, N, ql::choose_config(true, M, N).bn);
+  const ql::Nvfp4Workspace L = ql::nvfp4_workspace(M, K, N, ql::choose_config(true, M, N, K).bn);
   if (codes_offset) *codes_offset = L.codes_off;
   if (act_scales_offset) *act_scales_offset = L.act_sf_off;
   if (weight_scales_offset) *weight_scales_offset = L.wgt_sf_off;
@@ -173,7 +173,7 @@ int nvfp4_linear_prologue(const void* x, int64_t M, int64_t K, const uint8_t* w_
   if (!x || !w_scale || !input_scale || M <= 0 || N <= 0 || K <= 0) return QL_ERR_INVALID_ARG;
   if (!nvfp4_shape_ok(M, K, N)) return fail_shape("nvfp4: needs K >= 32 and K % 32 == 0");
   if (!aligned16(x)) return QL_ERR_ALIGN;
-  const int bn = ql::choose_config(true, M, N).bn;
+  const int bn = ql::choose_config(true, M, N, K).bn;
   const ql::Nvfp4Workspace L = ql::nvfp4_workspace(M, K, N, bn);
   if (!workspace || workspace_bytes < nvfp4_linear_workspace_size(M, K, N)) return QL_ERR_WORKSPACE;
   if (!aligned16(workspace)) return QL_ERR_ALIGN;
@@ -193,7 +193,7 @@ static int nvfp4_gemm_impl(int64_t M, int64_t K, const uint8_t* w, int64_t N,
     return QL_ERR_INVALID_ARG;
   if (!nvfp4_shape_ok(M, K, N)) return fail_shape("nvfp4: needs K >= 32 and K % 32 == 0");
   if (!aligned16(w) || !aligned16(y) || (bias && !aligned16(bias))) return QL_ERR_ALIGN;
-  const ql::GemmConfig cfg = ql::choose_config(true, M, N);
+  const ql::GemmConfig cfg = ql::choose_config(true, M, N, K);
   const int bn = cfg.bn;
   const ql::Nvfp4Workspace L = ql::nvfp4_workspace(M, K, N, bn);
   if (!workspace || workspace_bytes < nvfp4_linear_workspace_size(M, K, N)) return QL_ERR_WORKSPACE;
@@ -241,7 +241,6 @@ int nvfp4_linear(const void* x, int64_t M, int64_t K, const uint8_t* w, const ui
   if (!nvfp4_shape_ok(M, K, N)) return fail_shape("nvfp4: needs K >= 32 and K % 32 == 0");
   if (!aligned16(x) || !aligned16(w) || !aligned16(y) || (bias && !aligned16(bias)))
     return QL_ERR_ALIGN;
-  const ql::Nvfp4Workspace L = ql::nvfp4_workspace(M, K, N, ql::choose_config(true, M, N).bn);
   if (!workspace || workspace_bytes < nvfp4_linear_workspace_size(M, K, N)) return QL_ERR_WORKSPACE;
   int rc = nvfp4_linear_prologue(x, M, K, w_scale, N, input_scale, workspace, workspace_bytes,
                                  stream);
@@ -292,7 +291,7 @@ static int fp8r_gemm_impl(const uint8_t* xq, const float* x_scale, int64_t M, in
   if (rc != QL_OK) return rc;
   ql::GemmProblem p{};
   p.fp4 = false;
-  const ql::GemmConfig cfg = ql::choose_config(false, M, N);
+  const ql::GemmConfig cfg = ql::choose_config(false, M, N, K);
   p.bn = cfg.bn;
   p.cg = cfg.cg;
   p.M = M;

@@ -77,7 +77,8 @@ struct Cfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int EPI_BUFS = kEpiBufsPerWarp;
   static constexpr int EPI_BYTES = 4 * EPI_BUFS * kEpiBufBytes;      // 4 epilogue warps
-  static constexpr int RESERVED = 1024 /*alignment*/ + 1024 /*barriers*/ + EPI_BYTES;
+  static constexpr int COLVEC_BYTES = 2 * 2 * 256 * 4;  // bias + column scales, 2 tiles deep
+  static constexpr int RESERVED = 1024 /*alignment*/ + 1024 /*barriers*/ + EPI_BYTES + COLVEC_BYTES;
   static constexpr int STAGES_FIT = (kSmemLimit - RESERVED) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
   static constexpr int SF_COLS = FP4 ? 16 + 4 * NA * 4 : 0;
@@ -99,7 +100,11 @@ struct Cfg {
   static_assert(STAGES >= 2, "shared memory too small for two stages");
   static_assert(SFA_COL + SF_COLS <= kTmemCols, "TMEM budget");
   static_assert(!OVERLAP || BN == 256, "only the 256-column tile shares a slab");
-  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "tile width");
+  static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "tile width");
+  // epilogue slab: 64 columns (128-byte rows, 128-byte swizzle) when BN allows,
+  // else 32 columns (64-byte rows, 64-byte swizzle)
+  static constexpr int SLAB = (BN % 64 == 0) ? 64 : 32;
+  static constexpr int NSLAB = BN / SLAB;
   static_assert(CG == 1 || CG == 2, "one SM or a CTA pair");
   static_assert(B_ROWS % 8 == 0, "B half must be whole 8-row core groups");
 };
@@ -128,7 +133,9 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
   uint8_t* smem_sfa = smem_b + C::STAGES * C::B_BYTES;
   uint8_t* smem_sfb = smem_sfa + C::STAGES * C::SFA_BYTES;
   uint8_t* smem_epi = smem_sfb + C::STAGES * C::SFB_BYTES;  // 1024-aligned
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_epi + C::EPI_BYTES);
+  // per-tile column vectors for the epilogue: [2 tiles][bias | column scale][256]
+  float* colvec = reinterpret_cast<float*>(smem_epi + C::EPI_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_epi + C::EPI_BYTES + C::COLVEC_BYTES);
   uint64_t* full_bar = bars;
   uint64_t* empty_bar = bars + C::STAGES;
   uint64_t* tfull_bar = bars + 2 * C::STAGES;
@@ -385,11 +392,27 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     uint32_t acc_phase = 0;
     float alpha = 1.0f;
     if constexpr (FP4) alpha = __fmul_rn(__ldg(args.scale_a), __ldg(args.scale_b));
-    for (int tile = group; tile < args.total_tiles; tile += ngroups) {
+    int titer = 0;
+    for (int tile = group; tile < args.total_tiles; tile += ngroups, ++titer) {
       const int m_blk = tile % args.tiles_m;
       const int n_blk = tile / args.tiles_m;
       const int bi = C::OVERLAP ? 0 : acc;
-      if (!warp_wait_bounded(&tfull_bar[bi], acc_phase, deadline)) {
+      // the tile's bias and column scales into shared memory (double-buffered by
+      // tile), loaded by the 128 epilogue threads while the accumulator is
+      // still being computed; one barrier among the epilogue warps per tile (all
+      // of them have finished the previous tile, whose buffer the next load uses)
+      float* cv_bias = colvec + (titer & 1) * 512;
+      float* cv_scale = cv_bias + 256;
+      for (int j = threadIdx.x - 64; j < BN; j += 128) {
+        const int n = n_blk * BN + j;
+        const bool in = n < args.N;
+        cv_bias[j] = (args.bias && in) ? __ldg(args.bias + n) : 0.0f;
+        if constexpr (!FP4) cv_scale[j] = in ? __ldg(args.scale_b + n) : 0.0f;
+      }
+      const bool ready = warp_wait_bounded(&tfull_bar[bi], acc_phase, deadline);
+      // publishes the column vectors to all epilogue warps, and makes every
+      // epilogue warp leave together if any wait expired
+      if (barrier1_any<128>(!ready)) {
         record_timeout(args.status);
         break;
       }
@@ -401,38 +424,37 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * C::ACC_STRIDE);
 #pragma unroll 1
-      for (int it = 0; it < BN / 64; ++it) {
+      for (int it = 0; it < C::NSLAB; ++it) {
         // slab order: with shared slabs, buffer 0 drains its last slab (the shared
         // one) first; otherwise slabs go in order
-        const int sl = (C::OVERLAP && acc == 0) ? (it + BN / 64 - 1) % (BN / 64) : it;
-        uint32_t r[64];
+        const int sl = (C::OVERLAP && acc == 0) ? (it + C::NSLAB - 1) % C::NSLAB : it;
+        uint32_t r[C::SLAB];
         __syncwarp();  // tcgen05.ld is warp-collective
-        tmem_ld_32x32b_x32(tbase + sl * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-        tmem_ld_32x32b_x32(tbase + sl * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+#pragma unroll
+        for (int h = 0; h < C::SLAB / 32; ++h)
+          tmem_ld_32x32b_x32(tbase + sl * C::SLAB + 32 * h,
+                             *reinterpret_cast<uint32_t(*)[32]>(&r[32 * h]));
         tmem_ld_wait();
         // hand the buffer back once the MMA can no longer overwrite unread columns:
         // after the shared slab, or after the last slab
-        if (it == (C::OVERLAP ? 0 : BN / 64 - 1)) {
+        if (it == (C::OVERLAP ? 0 : C::NSLAB - 1)) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(tempty_bar0 + bi * 8u);
         }
-        const int n0 = n_blk * BN + sl * 64;
+        const int n0 = n_blk * BN + sl * C::SLAB;
         if (n0 >= args.N) continue;  // warp-uniform
         if (args.use_tma_store) {
-          // columns n0 .. n0+63 of this warp's 32 rows: scale, bias, bf16, into a
-          // 128-byte-swizzled staging tile, then one TMA store per warp.
-          uint32_t packed[32];
+          // columns n0 .. n0+SLAB-1 of this warp's 32 rows: scale, bias, bf16, into a
+          // swizzled staging tile, then one TMA store per warp.
+          uint32_t packed[C::SLAB / 2];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int n = n0 + 4 * i;
-            const bool in = n < args.N;  // N % 8 == 0: a float4 is all in or all out
-            const float4 b4 = (args.bias && in) ? __ldg(reinterpret_cast<const float4*>(args.bias + n))
-                                                : make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int i = 0; i < C::SLAB / 4; ++i) {
+            const int j = sl * C::SLAB + 4 * i;  // column within the tile
+            const float4 b4 = *reinterpret_cast<const float4*>(cv_bias + j);
             float4 s4 = make_float4(alpha, alpha, alpha, alpha);
             if constexpr (!FP4) {
-              const float4 w4 = in ? __ldg(reinterpret_cast<const float4*>(args.scale_b + n))
-                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+              const float4 w4 = *reinterpret_cast<const float4*>(cv_scale + j);
               s4 = make_float4(__fmul_rn(row_scale, w4.x), __fmul_rn(row_scale, w4.y),
                                __fmul_rn(row_scale, w4.z), __fmul_rn(row_scale, w4.w));
             }
@@ -449,10 +471,14 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
               bulk_wait_group_read<1>();
           }
           __syncwarp();
+          // 16-byte chunk j of row `lane` goes to chunk j ^ f(row), the TMA's swizzle
+          // (128-byte rows: f = row % 8; 64-byte rows: f = (row / 2) % 4)
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            *reinterpret_cast<uint4*>(sbuf + lane * 128 + ((j ^ (lane & 7)) * 16)) =
+          for (int j = 0; j < C::SLAB / 8; ++j) {
+            const int pos = (C::SLAB == 64) ? (j ^ (lane & 7)) : (j ^ ((lane >> 1) & 3));
+            *reinterpret_cast<uint4*>(sbuf + lane * (C::SLAB * 2) + pos * 16) =
                 make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+          }
           fence_proxy_async_shared();
           __syncwarp();
           if (lane == 0) {
@@ -464,7 +490,7 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
           if (m >= args.M) continue;
           uint16_t* yrow = args.y + static_cast<int64_t>(m) * args.N;
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
+          for (int i = 0; i < C::SLAB; ++i) {
             const int n = n0 + i;
             if (n < args.N) {
               const float sc = FP4 ? alpha : __fmul_rn(row_scale, __ldg(args.scale_b + n));
@@ -572,8 +598,10 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
       return cudaErrorInvalidValue;
   }
   const bool tma_store = (p.N % 8) == 0 && (reinterpret_cast<uintptr_t>(p.y) & 15) == 0;
-  if (tma_store && !encode_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.y, p.N, p.M, p.N * 2, 64,
-                              32, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE))
+  if (tma_store &&
+      !encode_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.y, p.N, p.M, p.N * 2, Cf::SLAB, 32,
+                 Cf::SLAB == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                 CU_TENSOR_MAP_L2_PROMOTION_NONE))
     return cudaErrorInvalidValue;
 
   GemmArgs a{};
@@ -651,24 +679,42 @@ bool set_tile_override(int bn, int cg) {
     g_force_cg.store(0);
     return true;
   }
-  if ((bn != 128 && bn != 192 && bn != 256) || (cg != 1 && cg != 2)) return false;
+  if ((bn != 128 && bn != 192 && bn != 224 && bn != 256) || (cg != 1 && cg != 2)) return false;
   g_force_cg.store(cg);
   g_force_bn.store(bn);
   return true;
 }
 
-GemmConfig choose_config(bool fp4, int64_t M, int64_t N) {
-  (void)fp4;
+GemmConfig choose_config(bool fp4, int64_t M, int64_t N, int64_t K) {
   GemmConfig c{};
   if (g_force_bn.load() != 0) {
     c.bn = g_force_bn.load();
     c.cg = g_force_cg.load();
     return c;
   }
+  // CTA pairs once there are two 128-row blocks to pair. Tile width from a cost
+  // model fitted to B200 measurements: waves over the resident groups x (K steps
+  // x operand KB one group loads per K step), plus a fixed per-tile cost for the
+  // 256-column FP4 tile, whose TMEM buffers share a slab (the next tile's MMAs
+  // wait for the epilogue to drain it; about 1.5 us, worth ~240 KB of loads).
   c.cg = M >= 512 ? 2 : 1;
+  const int64_t groups = c.cg == 2 ? 74 : 148;
+  const int64_t tiles_m = ceil_div64(M, 128 * c.cg);
+  const int64_t ksteps = ceil_div64(K, fp4 ? kKTileFp4 : kKTileFp8);
+  double best = 0.0;
   c.bn = 128;
-  if (N % 192 == 0 && N >= 1536) c.bn = 192;
-  else if (N % 256 == 0 && N >= 4096) c.bn = 256;
+  for (int bn : {128, 192, 224, 256}) {
+    const int64_t tiles = tiles_m * ceil_div64(N, bn);
+    const int64_t waves = ceil_div64(tiles, groups);
+    const int na = (bn + 127) / 128;
+    const double kb = c.cg * 16.0 + bn * 0.125 + (fp4 ? c.cg * (2.0 + 2.0 * na) : 0.0);
+    const double per_tile = static_cast<double>(ksteps) * kb + ((fp4 && bn == 256) ? 240.0 : 0.0);
+    const double cost = static_cast<double>(waves) * per_tile;
+    if (best == 0.0 || cost < best * 0.999) {
+      best = cost;
+      c.bn = bn;
+    }
+  }
   return c;
 }
 
@@ -678,12 +724,16 @@ cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream) {
   QL_CASE(true, 128, 1)
   QL_CASE(true, 192, 1)
   QL_CASE(true, 256, 1)
+  QL_CASE(true, 224, 1)
+  QL_CASE(true, 224, 2)
   QL_CASE(true, 128, 2)
   QL_CASE(true, 192, 2)
   QL_CASE(true, 256, 2)
   QL_CASE(false, 128, 1)
   QL_CASE(false, 192, 1)
   QL_CASE(false, 256, 1)
+  QL_CASE(false, 224, 1)
+  QL_CASE(false, 224, 2)
   QL_CASE(false, 128, 2)
   QL_CASE(false, 192, 2)
   QL_CASE(false, 256, 2)

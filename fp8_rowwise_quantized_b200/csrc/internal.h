@@ -35,7 +35,7 @@ struct GemmProblem {
   bool pdl;              // launched right after its producer kernel (programmatic dependency)
 };
 
-GemmConfig choose_config(bool fp4, int64_t M, int64_t N);
+GemmConfig choose_config(bool fp4, int64_t M, int64_t N, int64_t K);
 bool set_tile_override(int bn, int cg);  // bn == 0 restores the automatic choice
 cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream);
 

@@ -78,6 +78,22 @@ __device__ __forceinline__ bool warp_wait_bounded(uint64_t* bar, uint32_t parity
   return __all_sync(0xffffffffu, ok);
 }
 
+// Barrier 1 over `nthreads` threads that also ORs a flag across them: every
+// participant gets the same answer (used to leave a loop together).
+template <int NTHREADS>
+__device__ __forceinline__ bool barrier1_any(bool flag) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, 1, %2, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(flag ? 1u : 0u), "n"(NTHREADS)
+      : "memory");
+  return r != 0;
+}
+
 // ---------------------------------------------------------------- clusters (CTA pairs)
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;

@@ -206,7 +206,7 @@ void ql_set_fault_injection(int enable, int timeout_ms);
 
 /* Tuning override of the GEMM tile shape for later calls (both schemes): output
  * tiles of (128 * cg) rows x bn columns, cg = 2 running each MMA across a pair of
- * SMs. bn in {128, 192, 256}, cg in {1, 2}; bn = 0 restores the automatic choice.
+ * SMs. bn in {128, 192, 224, 256}, cg in {1, 2}; bn = 0 restores the automatic choice.
  * Returns QL_OK or QL_ERR_INVALID_ARG. Workspace sizes already cover every tile. */
 int ql_set_tile_override(int bn, int cg);
 

@@ -147,7 +147,7 @@ def test_fp8r_gemm_from_prequantized_matches_linear():
     assert torch.equal(y1, y2)
 
 
-TILES = [(128, 1), (192, 1), (256, 1), (128, 2), (192, 2), (256, 2)]
+TILES = [(128, 1), (192, 1), (224, 1), (256, 1), (128, 2), (192, 2), (224, 2), (256, 2)]
 
 
 @pytest.mark.parametrize("bn,cg", TILES)
