@@ -19,7 +19,8 @@ import torch
 from . import _lib
 
 __all__ = [
-    "nvfp4_quantize_act", "nvfp4_linear", "nvfp4_linear_noalloc", "nvfp4_linear_prologue",
+    "nvfp4_quantize_act", "nvfp4_linear", "nvfp4_linear_single_launch", "nvfp4_linear_noalloc",
+    "nvfp4_linear_prologue",
     "nvfp4_linear_gemm",
     "nvfp4_linear_workspace_size", "nvfp4_linear_workspace_layout", "nvfp4_global_scale",
     "fp8r_quantize_rows", "fp8r_linear", "fp8r_linear_gemm", "fp8r_linear_workspace_size",
@@ -118,6 +119,33 @@ def nvfp4_linear(x: torch.Tensor, w: torch.Tensor, w_scale: torch.Tensor,
         y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     ws = _workspace(nvfp4_linear_workspace_size(M, K, N), x.device, workspace)
     _lib.check("nvfp4_linear", _lib.load().nvfp4_linear(
+        _ptr(x), M, K, _ptr(w), _ptr(w_scale), N, _ptr(weight_scale_2), _ptr(input_scale),
+        _ptr(bias), _ptr(y), _ptr(ws), ws.numel(), _stream()))
+    return y
+
+
+def nvfp4_linear_single_launch(x: torch.Tensor, w: torch.Tensor, w_scale: torch.Tensor,
+                               weight_scale_2: torch.Tensor, input_scale: torch.Tensor,
+                               bias: Optional[torch.Tensor] = None,
+                               y: Optional[torch.Tensor] = None,
+                               workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """nvfp4_linear as one kernel launch (quantization inside the GEMM launch, then a
+    grid-wide barrier, then the GEMM); same bits as nvfp4_linear. Needs K % 256 == 0."""
+    _need(x, "x", torch.bfloat16, 2)
+    _need(w, "w", torch.uint8, 2)
+    _need(w_scale, "w_scale", torch.uint8, 2)
+    _scalar(weight_scale_2, "weight_scale_2")
+    _scalar(input_scale, "input_scale")
+    M, K = x.shape
+    N = w.shape[0]
+    if w.shape[1] * 2 != K or tuple(w_scale.shape) != (N, K // 16):
+        raise ValueError("weight shapes do not match x")
+    if bias is not None:
+        _need(bias, "bias", torch.float32, 1)
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    ws = _workspace(nvfp4_linear_workspace_size(M, K, N), x.device, workspace)
+    _lib.check("nvfp4_linear_single_launch", _lib.load().nvfp4_linear_single_launch(
         _ptr(x), M, K, _ptr(w), _ptr(w_scale), N, _ptr(weight_scale_2), _ptr(input_scale),
         _ptr(bias), _ptr(y), _ptr(ws), ws.numel(), _stream()))
     return y

@@ -4,6 +4,7 @@
 // and gemm.cu; this file only checks arguments and launches them.
 #include <cuda_runtime.h>
 #include <atomic>
+#include <chrono>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -73,6 +74,20 @@ int fail_shape(const char* what) {
 }
 
 uint64_t timeout_ns() { return static_cast<uint64_t>(g_timeout_ms.load()) * 1000000ull; }
+
+// Tag of one single-launch nvfp4_linear call: odd, and different for consecutive
+// calls (a per-process counter, mixed, from a time-dependent start), so the sync
+// words of the workspace never look finished from an earlier call.
+uint32_t next_launch_tag() {
+  static const uint32_t start = static_cast<uint32_t>(
+      std::chrono::steady_clock::now().time_since_epoch().count() * 0x9E3779B97F4A7C15ull >> 32);
+  static std::atomic<uint32_t> seq{0};
+  uint32_t t = start + seq.fetch_add(1) * 0x9E3779B9u;
+  t ^= t >> 16;
+  t *= 0x85EBCA6Bu;
+  t ^= t >> 13;
+  return t | 1u;
+}
 
 bool nvfp4_shape_ok(int64_t M, int64_t K, int64_t N) {
   return M >= 1 && N >= 1 && K >= 32 && K % 32 == 0 && M <= (1ll << 30) && N <= (1ll << 30) &&
@@ -242,11 +257,61 @@ int nvfp4_linear(const void* x, int64_t M, int64_t K, const uint8_t* w, const ui
   if (!aligned16(x) || !aligned16(w) || !aligned16(y) || (bias && !aligned16(bias)))
     return QL_ERR_ALIGN;
   if (!workspace || workspace_bytes < nvfp4_linear_workspace_size(M, K, N)) return QL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return QL_ERR_ALIGN;
   int rc = nvfp4_linear_prologue(x, M, K, w_scale, N, input_scale, workspace, workspace_bytes,
                                  stream);
   if (rc != QL_OK) return rc;
   return nvfp4_gemm_impl(M, K, w, N, weight_scale_2, input_scale, bias, y, workspace,
                          workspace_bytes, stream, true);
+}
+
+int nvfp4_linear_single_launch(const void* x, int64_t M, int64_t K, const uint8_t* w,
+                               const uint8_t* w_scale, int64_t N, const float* weight_scale_2,
+                               const float* input_scale, const float* bias, void* y,
+                               void* workspace, size_t workspace_bytes, ql_stream_t stream) {
+  if (!x || !w || !w_scale || !weight_scale_2 || !input_scale || !y || M <= 0 || N <= 0 || K <= 0)
+    return QL_ERR_INVALID_ARG;
+  if (!nvfp4_shape_ok(M, K, N) || K % 256 != 0)
+    return fail_shape("nvfp4_linear_single_launch: needs K % 256 == 0");
+  if (!aligned16(x) || !aligned16(w) || !aligned16(w_scale) || !aligned16(y) ||
+      (bias && !aligned16(bias)))
+    return QL_ERR_ALIGN;
+  if (!workspace || workspace_bytes < nvfp4_linear_workspace_size(M, K, N)) return QL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return QL_ERR_ALIGN;
+  // one launch: the GEMM kernel first quantizes the activations and lays out
+  // the weight scales into the workspace (which stays in L2), then multiplies
+  int dev = 0;
+  int rc = check_device(&dev);
+  if (rc != QL_OK) return rc;
+  const ql::GemmConfig cfg = ql::choose_config(true, M, N, K);
+  const ql::Nvfp4Workspace L = ql::nvfp4_workspace(M, K, N, cfg.bn);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  ql::GemmProblem p{};
+  p.fp4 = true;
+  p.bn = cfg.bn;
+  p.cg = cfg.cg;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.a = ws + L.codes_off;
+  p.b = w;
+  p.sfa = ws + L.act_sf_off;
+  p.sfb = ws + L.wgt_sf_off;
+  p.scale_a = input_scale;
+  p.scale_b = weight_scale_2;
+  p.bias = bias;
+  p.y = y;
+  p.status = status_ptr(dev);
+  p.timeout_ns = timeout_ns();
+  p.inject_fault = g_inject_fault.load();
+  p.pdl = false;
+  p.fused = true;
+  p.x = x;
+  p.w_scale = w_scale;
+  p.sync = reinterpret_cast<uint64_t*>(ws + L.sync_off);
+  p.tag = next_launch_tag();
+  cudaError_t e = ql::launch_gemm(p, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QL_OK : record(e, "nvfp4_linear_single_launch");
 }
 
 int nvfp4_global_scale(const void* x, int64_t n, float* out, ql_stream_t stream) {

@@ -42,7 +42,8 @@ namespace ql {
 namespace {
 
 constexpr int kRowsPerCta = 128;
-constexpr int kThreads = 192;
+constexpr int kThreads = 192;       // producer, MMA, 4 epilogue warps
+constexpr int kThreadsFused = 256;  // 8 warps share the quantization; warps 6, 7 stop there
 constexpr int kSmemLimit = 232448;  // 227 KB opt-in per block
 constexpr int kTmemCols = 512;
 constexpr int kEpiBufBytes = 32 * 128;  // 32 rows x 64 bf16 (128-byte swizzled), one TMA box
@@ -64,6 +65,16 @@ struct GemmArgs {
   int inject_fault;
   int wait_prior_grid;
   int use_tma_store;        // Y written through shared memory + TMA (needs N % 8 == 0)
+  int raster_n;             // tile order: 1 = N fastest (m_blk = tile / tiles_n), 0 = M fastest
+  // in-launch activation quantization (FP4, K % 256 == 0)
+  const uint16_t* x;        // bf16 [M, K]
+  uint8_t* xq;              // packed codes [M, K/2]: written here, read as A
+  uint8_t* xs;              // activation scale atoms: written here, read as SFA
+  const uint8_t* w_scale;   // weight scales, row-major E4M3 [N, K/16]
+  uint8_t* ws_atoms;        // weight scale atoms for tile width BN: written here, read as SFB
+  uint64_t* sync;           // sync_words tagged counters (see kSyncBarrier)
+  int sync_words;
+  uint32_t tag;             // this launch's tag, odd
 };
 
 template <bool FP4, int BN, int CG>
@@ -109,6 +120,16 @@ struct Cfg {
   static_assert(B_ROWS % 8 == 0, "B half must be whole 8-row core groups");
 };
 
+__device__ __forceinline__ void tile_coords(int tile, const GemmArgs& a, int& m_blk, int& n_blk) {
+  if (a.raster_n) {
+    m_blk = tile / a.tiles_n;
+    n_blk = tile - m_blk * a.tiles_n;
+  } else {
+    m_blk = tile % a.tiles_m;
+    n_blk = tile / a.tiles_m;
+  }
+}
+
 __device__ __forceinline__ void record_timeout(int* status) {
   if (status) atomicCAS(status, 0, static_cast<int>(QL_ERR_TIMEOUT_CODE));
 }
@@ -118,8 +139,152 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&p);
 }
 
-template <bool FP4, int BN, int CG>
-__global__ void __launch_bounds__(kThreads, 1)
+// ---------------------------------------------------------------- in-launch quantization
+// The single-launch NVFP4 linear first quantizes the activations and lays out the
+// weight scales into its workspace with every warp of every CTA, then meets at a
+// grid-wide barrier, then runs the GEMM below on that workspace (which stays in
+// L2). Words shared by the CTAs, in the workspace: the barrier count and the
+// count of CTAs that have finished. Each word holds (tag << 32) | count; a word
+// carrying another launch's tag (or leftover bytes) counts as zero. The last CTA
+// to finish writes them back to zero, so a replay of the same launch (same tag,
+// e.g. from a CUDA graph) also starts from zero. The grid is one wave of resident
+// CTAs, so the barrier does not wait for CTAs that cannot start; its wait is
+// bounded all the same.
+constexpr int kSyncBarrier = 0;
+constexpr int kSyncExit = 1;
+
+__device__ __forceinline__ uint32_t tagged_count(uint64_t w, uint32_t tag) {
+  return static_cast<uint32_t>(w >> 32) == tag ? static_cast<uint32_t>(w) : 0u;
+}
+
+// Gives a sync word this launch's tag (count 0) unless it carries it already.
+__device__ __forceinline__ void sync_word_adopt(uint64_t* w, uint32_t tag) {
+  const uint64_t fresh = static_cast<uint64_t>(tag) << 32;
+  uint64_t cur = ld_relaxed_gpu(w);
+  while (static_cast<uint32_t>(cur >> 32) != tag) {
+    const uint64_t seen = atom_cas_gpu(w, cur, fresh);
+    if (seen == cur) break;
+    cur = seen;
+  }
+}
+
+// 256-element chunks of the activation rows, quantized with the arithmetic of
+// nvfp4_quantize_act (per 16-element block: amax, E4M3 scale through the global
+// scale g, E2M1 codes): codes row-major, scales in the atom layout. Chunk c = row
+// c / (K/256), K chunk c % (K/256); each CTA takes a contiguous range of chunks.
+// Lane l holds elements 8l .. 8l+7 of a chunk, so lanes 2j and 2j+1 share block j.
+// Needs K % 256 == 0.
+// Activation staging of the quantization phase: 16 KB slots (32 chunks) of the
+// pipeline's shared memory, filled by bulk copies (warp 0) and encoded by warps
+// 1..7, each taking a contiguous part of a slot.
+constexpr int kQSlotChunks = 32;
+constexpr int kQSlotBytes = kQSlotChunks * 512;
+constexpr int kQMaxSlots = 12;
+constexpr int kQConsumers = 7;
+constexpr int kQPerWarp = (kQSlotChunks + kQConsumers - 1) / kQConsumers;
+
+// `inv_of` holds, for each block scale code s (the amax is >= 0, so s < 128),
+// 1 / (value(s) * g) rounded as nvfp4_quantize_act computes it, and 0 where
+// value(s) * g == 0 (then all codes are 0): a table read instead of a branch.
+
+// Consumer warp wq's part of a staged slot (chunks cs .. cs + n - 1): chunks
+// [wq * 32 / 7, (wq + 1) * 32 / 7) of the slot, read from shared memory and
+// encoded branch-free (chunks past the slot's end are predicated off). The
+// stages run across all the warp's chunks (every table read before any store),
+// so the chunks' dependency chains overlap.
+__device__ __forceinline__ void quantize_slot_part(const GemmArgs& a, const uint8_t* slot,
+                                                   int64_t cs, int n, int wq, const float* inv_of,
+                                                   float cinv, int lane) {
+  const int j0 = wq * kQSlotChunks / kQConsumers;
+  const int j1 = (wq + 1) * kQSlotChunks / kQConsumers;
+  constexpr int P = kQPerWarp;
+  uint4 v[P];
+  bool valid[P];
+#pragma unroll
+  for (int i = 0; i < P; ++i) {
+    const int j = j0 + i;
+    valid[i] = j < j1 && j < n;
+    v[i] = valid[i] ? *reinterpret_cast<const uint4*>(slot + j * 512 + lane * 16)
+                    : make_uint4(0u, 0u, 0u, 0u);
+  }
+  uint32_t sc[P];
+  float inv[P];
+#pragma unroll
+  for (int i = 0; i < P; ++i) {
+    const float part = bf16x8_amax(v[i].x, v[i].y, v[i].z, v[i].w);
+    const float amax = fmaxf(part, __shfl_xor_sync(0xffffffffu, part, 1));
+    sc[i] = cvt_e4m3x4(__fmul_rn(amax, cinv), 0.0f, 0.0f, 0.0f) & 0x7Fu;
+  }
+#pragma unroll
+  for (int i = 0; i < P; ++i) inv[i] = inv_of[sc[i]];
+  uint32_t codes[P], word[P];
+#pragma unroll
+  for (int i = 0; i < P; ++i) {
+    const float f[8] = {__fmul_rn(bf16_lo(v[i].x), inv[i]), __fmul_rn(bf16_hi(v[i].x), inv[i]),
+                        __fmul_rn(bf16_lo(v[i].y), inv[i]), __fmul_rn(bf16_hi(v[i].y), inv[i]),
+                        __fmul_rn(bf16_lo(v[i].z), inv[i]), __fmul_rn(bf16_hi(v[i].z), inv[i]),
+                        __fmul_rn(bf16_lo(v[i].w), inv[i]), __fmul_rn(bf16_hi(v[i].w), inv[i])};
+    codes[i] = inv[i] != 0.0f ? cvt_e2m1x8(f) : 0u;
+    // the scales of blocks 4q .. 4q+3 (one 64-element group) sit in lanes 8q,
+    // 8q+2, 8q+4, 8q+6; lane 8q writes them as one word
+    const uint32_t s1 = __shfl_down_sync(0xffffffffu, sc[i], 2);
+    const uint32_t s2 = __shfl_down_sync(0xffffffffu, sc[i], 4);
+    const uint32_t s3 = __shfl_down_sync(0xffffffffu, sc[i], 6);
+    word[i] = sc[i] | (s1 << 8) | (s2 << 16) | (s3 << 24);
+  }
+  const int kc = a.K >> 8;
+  int64_t r = (cs + j0) / kc;
+  int ck = static_cast<int>(cs + j0 - r * kc);
+#pragma unroll
+  for (int i = 0; i < P; ++i) {
+    const int64_t c = cs + j0 + i;
+    if (valid[i]) {
+      *reinterpret_cast<uint32_t*>(a.xq + c * 128 + lane * 4) = codes[i];  // row r, bytes 128 ck + 4 l
+      if ((lane & 7) == 0)
+        *reinterpret_cast<uint32_t*>(a.xs + (r >> 7) * a.kg * kSfAtomBytes + (r & 31) * 16 +
+                                     ((r >> 5) & 3) * 4 + (ck * 4 + (lane >> 3)) * kSfAtomBytes) =
+            word[i];
+    }
+    const bool wrap = ++ck == kc;
+    ck = wrap ? 0 : ck;
+    r += wrap ? 1 : 0;
+  }
+}
+
+// One weight-scale job: atom `at` (128 rows) of weight tile t for K tile kt, i.e.
+// 4 atoms (one per 64-element group) of the layout the GEMM's scale loads read.
+// Line l of atom (kg, at) holds group kg of rows 128 at + l, + 32, + 64, + 96 of
+// the tile, read from the row-major [N, K/16] scales (16 bytes per row per K
+// tile); rows beyond the tile or N are zero.
+template <int BN, int NA>
+__device__ __forceinline__ void weight_scale_job(const GemmArgs& a, int64_t job, int lane) {
+  const int64_t per_tile = static_cast<int64_t>(NA) * a.num_k_tiles;
+  const int64_t t = job / per_tile;
+  const int at = static_cast<int>((job - t * per_tile) / a.num_k_tiles);
+  const int kt = static_cast<int>(job - t * per_tile - static_cast<int64_t>(at) * a.num_k_tiles);
+  const int64_t ks = a.K >> 4;
+  uint4 v[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int nn = 128 * at + 32 * q + lane;
+    const int64_t n = t * BN + nn;
+    v[q] = (nn < BN && n < a.N)
+               ? __ldg(reinterpret_cast<const uint4*>(a.w_scale + n * ks + kt * 16))
+               : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    const uint4 line = g == 0   ? make_uint4(v[0].x, v[1].x, v[2].x, v[3].x)
+                       : g == 1 ? make_uint4(v[0].y, v[1].y, v[2].y, v[3].y)
+                       : g == 2 ? make_uint4(v[0].z, v[1].z, v[2].z, v[3].z)
+                                : make_uint4(v[0].w, v[1].w, v[2].w, v[3].w);
+    const int64_t atom = (t * a.kg + kt * 4 + g) * NA + at;
+    *reinterpret_cast<uint4*>(a.ws_atoms + atom * kSfAtomBytes + lane * 16) = line;
+  }
+}
+
+template <bool FP4, int BN, int CG, bool FUSED>
+__global__ void __launch_bounds__(FUSED ? kThreadsFused : kThreads, 1)
 qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
              const __grid_constant__ CUtensorMap tmap_sfa,
              const __grid_constant__ CUtensorMap tmap_sfb,
@@ -142,7 +307,9 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
   uint64_t* tempty_bar = tfull_bar + 2;
   uint64_t* drain_bar = tempty_bar + 2;
   uint64_t* never_bar = drain_bar + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(never_bar + 1);
+  uint64_t* qfull_bar = never_bar + 1;           // fused: staging slot filled
+  uint64_t* qfree_bar = qfull_bar + kQMaxSlots;  // fused: staging slot encoded
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(qfree_bar + kQMaxSlots);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -170,6 +337,12 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     }
     mbar_init(drain_bar, 1);
     mbar_init(never_bar, 1);
+    if constexpr (FUSED) {
+      for (int q = 0; q < kQMaxSlots; ++q) {
+        mbar_init(&qfull_bar[q], 1);
+        mbar_init(&qfree_bar[q], kQConsumers);
+      }
+    }
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -195,12 +368,107 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
   // global inputs are read only after it has completed.
   if (args.wait_prior_grid) grid_dependency_wait();
 
+
   bool run = true;
   if (args.inject_fault) {
     run = false;
     if (blockIdx.x == 0 && threadIdx.x == 0) {
       if (!mbar_wait_bounded(never_bar, 0, deadline)) record_timeout(args.status);
     }
+  }
+
+  if constexpr (FUSED) {
+    // thread 0 gives the sync words this launch's tag before any count on them
+    if (threadIdx.x == 0) {
+      sync_word_adopt(args.sync + kSyncBarrier, args.tag);
+      sync_word_adopt(args.sync + kSyncExit, args.tag);
+    }
+    // 1 / (value(s) * g) per block scale code, in the (still unused) epilogue
+    // staging memory
+    float* inv_table = reinterpret_cast<float*>(smem_epi);
+    if (threadIdx.x < 128) {
+      const float d = __fmul_rn(e4m3_to_float(threadIdx.x), __ldg(args.scale_a));
+      inv_table[threadIdx.x] = d != 0.0f ? __frcp_rn(d) : 0.0f;
+    }
+    __syncthreads();
+    if (run) {
+      // ---------------------------------------------------------- quantization
+      // this CTA's contiguous range of activation chunks, staged through the
+      // pipeline's shared memory (unused until the GEMM starts) by bulk copies
+      const int64_t chunks = static_cast<int64_t>(args.M) * (args.K >> 8);
+      const int64_t cb = chunks * blockIdx.x / gridDim.x;
+      const int64_t ce = chunks * (blockIdx.x + 1) / gridDim.x;
+      const int nslots = static_cast<int>((ce - cb + kQSlotChunks - 1) / kQSlotChunks);
+      constexpr int kRing = (C::STAGES * C::STAGE_BYTES) / kQSlotBytes < kQMaxSlots
+                                ? (C::STAGES * C::STAGE_BYTES) / kQSlotBytes
+                                : kQMaxSlots;
+      static_assert(kRing >= 2, "staging ring");
+      uint8_t* ring = smem;
+      if (warp == 0) {
+        if (lane == 0) {
+          for (int si = 0; si < nslots; ++si) {
+            const int slot = si % kRing;
+            const int round = si / kRing;
+            if (round > 0 && !mbar_wait_bounded(&qfree_bar[slot], (round - 1) & 1, deadline)) {
+              record_timeout(args.status);
+              break;
+            }
+            const int64_t cs = cb + static_cast<int64_t>(si) * kQSlotChunks;
+            const int64_t n = ce - cs < kQSlotChunks ? ce - cs : kQSlotChunks;
+            mbar_arrive_expect_tx(&qfull_bar[slot], static_cast<uint32_t>(n * 512));
+            bulk_load(ring + slot * kQSlotBytes, args.x + cs * 256, static_cast<uint32_t>(n * 512),
+                      &qfull_bar[slot]);
+          }
+        }
+        __syncwarp();
+      } else {
+        const int wq = warp - 1;
+        // weight-scale jobs first, while the first slots land
+        const int64_t nwq = static_cast<int64_t>(gridDim.x) * kQConsumers;
+        const int64_t gwq = static_cast<int64_t>(blockIdx.x) * kQConsumers + wq;
+        const int64_t jobs = static_cast<int64_t>(args.tiles_n) * C::NA * args.num_k_tiles;
+        for (int64_t j = gwq; j < jobs; j += nwq) weight_scale_job<BN, C::NA>(args, j, lane);
+        const float cinv = __frcp_rn(__fmul_rn(6.0f, __ldg(args.scale_a)));
+        for (int si = 0; si < nslots; ++si) {
+          const int slot = si % kRing;
+          if (!warp_wait_bounded(&qfull_bar[slot], (si / kRing) & 1, deadline)) {
+            record_timeout(args.status);
+            break;
+          }
+          const int64_t cs = cb + static_cast<int64_t>(si) * kQSlotChunks;
+          const int n = static_cast<int>(ce - cs < kQSlotChunks ? ce - cs : kQSlotChunks);
+          quantize_slot_part(args, ring + slot * kQSlotBytes, cs, n, wq, inv_table, cinv, lane);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&qfree_bar[slot]);
+        }
+      }
+      // the staging memory is the GEMM's next (TMA-written) pipeline memory; this
+      // CTA's workspace writes are visible GPU-wide, to TMA reads too, before it counts
+      fence_proxy_async_shared();
+      __threadfence();
+      fence_proxy_async_global();
+    }
+    __syncthreads();
+    int* s_barrier_ok = reinterpret_cast<int*>(tmem_holder + 1);
+    if (threadIdx.x == 0) {
+      int ok = 1;
+      if (run) {
+        red_add_release_gpu(args.sync + kSyncBarrier, 1ull);
+        uint32_t n = 0;
+        while (tagged_count(ld_acquire_gpu(args.sync + kSyncBarrier), args.tag) < gridDim.x) {
+          if ((++n & 15u) == 0 && globaltimer_ns() > deadline) {
+            ok = 0;
+            record_timeout(args.status);
+            break;
+          }
+          __nanosleep(100);
+        }
+      }
+      *s_barrier_ok = ok;
+    }
+    __syncthreads();
+    fence_proxy_async_global();  // the TMA loads below see every CTA's workspace writes
+    if (!*s_barrier_ok) run = false;
   }
 
   if (run && warp == 0) {
@@ -210,8 +478,8 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     bool ok = true;
     int issued = 0;
     for (int tile = group; ok && tile < args.total_tiles; tile += ngroups) {
-      const int m_blk = tile % args.tiles_m;
-      const int n_blk = tile / args.tiles_m;
+      int m_blk, n_blk;
+      tile_coords(tile, args, m_blk, n_blk);
       const int a_row = m_blk * C::TILE_M + static_cast<int>(rank) * kRowsPerCta;
       const int b_row = n_blk * BN + static_cast<int>(rank) * C::B_ROWS;
       for (int kt = 0; kt < args.num_k_tiles; ++kt) {
@@ -230,8 +498,10 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                                                 kt * 4);
           const int sfb_atom = static_cast<int>((static_cast<int64_t>(n_blk) * args.kg + kt * 4) *
                                                 C::NA);
+
+          constexpr uint32_t kTx = C::STAGE_BYTES;
           if constexpr (CG == 2) {
-            if (leader) mbar_arrive_expect_tx(&full_bar[stage], CG * C::STAGE_BYTES);
+            if (leader) mbar_arrive_expect_tx(&full_bar[stage], CG * kTx);
             tma_load_2d_pair(sa, &tmap_a, fb, kt * 128, a_row);
             tma_load_2d_pair(sb, &tmap_b, fb, kt * 128, b_row);
             if constexpr (FP4) {
@@ -239,7 +509,7 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
               tma_load_2d_pair(ssb, &tmap_sfb, fb, 0, sfb_atom);
             }
           } else {
-            mbar_arrive_expect_tx(&full_bar[stage], C::STAGE_BYTES);
+            mbar_arrive_expect_tx(&full_bar[stage], kTx);
             tma_load_2d(sa, &tmap_a, &full_bar[stage], kt * 128, a_row);
             tma_load_2d(sb, &tmap_b, &full_bar[stage], kt * 128, b_row);
             if constexpr (FP4) {
@@ -382,7 +652,7 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
         mbar_wait_bounded(drain_bar, 0, globaltimer_ns() + 100000000ull);
       }
     }
-  } else if (run && warp >= 2) {
+  } else if (run && warp >= 2 && warp <= 5) {
     // ------------------------------------------------------------ epilogue
     const int q = warp % 4;  // TMEM lane quadrant this warp may access
     const int row_in_tile = static_cast<int>(rank) * kRowsPerCta + q * 32 + lane;
@@ -394,8 +664,8 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     if constexpr (FP4) alpha = __fmul_rn(__ldg(args.scale_a), __ldg(args.scale_b));
     int titer = 0;
     for (int tile = group; tile < args.total_tiles; tile += ngroups, ++titer) {
-      const int m_blk = tile % args.tiles_m;
-      const int n_blk = tile / args.tiles_m;
+      int m_blk, n_blk;
+      tile_coords(tile, args, m_blk, n_blk);
       const int bi = C::OVERLAP ? 0 : acc;
       // the tile's bias and column scales into shared memory (double-buffered by
       // tile), loaded by the 128 epilogue threads while the accumulator is
@@ -511,6 +781,17 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
   tc_fence_before();
   __syncthreads();
   if constexpr (CG == 2) cluster_sync_all();  // no peer accesses this CTA's memory any more
+  if constexpr (FUSED) {
+    // this CTA is done with the sync words; the last CTA out resets them
+    if (threadIdx.x == 0) {
+      __threadfence();
+      const uint64_t old = atom_add_relaxed_gpu(args.sync + kSyncExit, 1ull);
+      if (tagged_count(old, args.tag) + 1u == gridDim.x) {
+        __threadfence();
+        for (int i = 0; i < args.sync_words; ++i) st_relaxed_gpu(args.sync + i, 0ull);
+      }
+    }
+  }
   if (warp == 1) {
     tc_fence_after();
     if constexpr (CG == 2)
@@ -555,10 +836,10 @@ bool encode_2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, uin
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool FP4, int BN, int CG>
+template <bool FP4, int BN, int CG, bool FUSED>
 cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
   using Cf = Cfg<FP4, BN, CG>;
-  auto kern = qgemm_kernel<FP4, BN, CG>;
+  auto kern = qgemm_kernel<FP4, BN, CG, FUSED>;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -592,10 +873,13 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
     const int64_t a_atoms = ceil_div64(p.M, kRowsPerCta) * kg;
     const int64_t b_atoms = ceil_div64(p.N, BN) * kg * Cf::NA;
     if (!encode_2d(&tsa, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.sfa, 128, a_atoms, kSfAtomBytes, 128, 4,
-                   CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
-        !encode_2d(&tsb, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.sfb, 128, b_atoms, kSfAtomBytes, 128,
-                   4 * Cf::NA, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
+                   CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
       return cudaErrorInvalidValue;
+    if (!encode_2d(&tsb, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.sfb, 128, b_atoms, kSfAtomBytes,
+                          128, 4 * Cf::NA, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B)) {
+      return cudaErrorInvalidValue;
+    }
   }
   const bool tma_store = (p.N % 8) == 0 && (reinterpret_cast<uintptr_t>(p.y) & 15) == 0;
   if (tma_store &&
@@ -622,9 +906,20 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
   a.inject_fault = p.inject_fault;
   a.wait_prior_grid = p.pdl ? 1 : 0;
   a.use_tma_store = tma_store ? 1 : 0;
+  a.raster_n = 0;
+  if (FUSED) {
+    a.x = static_cast<const uint16_t*>(p.x);
+    a.xq = static_cast<uint8_t*>(const_cast<void*>(p.a));
+    a.xs = const_cast<uint8_t*>(p.sfa);
+    a.w_scale = p.w_scale;
+    a.ws_atoms = const_cast<uint8_t*>(p.sfb);
+    a.sync = p.sync;
+    a.sync_words = 8;  // the whole 64-byte region, so that the call leaves all of it zero
+    a.tag = p.tag;
+  }
 
   cudaLaunchConfig_t cfg{};
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(FUSED ? kThreadsFused : kThreads);
   cfg.dynamicSmemBytes = Cf::SMEM;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
@@ -719,8 +1014,23 @@ GemmConfig choose_config(bool fp4, int64_t M, int64_t N, int64_t K) {
 }
 
 cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream) {
+  if (p.fused) {
+    if (!p.fp4 || !p.x || !p.w_scale || !p.sync || p.K % kKTileFp4 != 0) return cudaErrorInvalidValue;
+#define QL_FCASE(BN_, CG_) \
+  if (p.bn == BN_ && p.cg == CG_) return launch_typed<true, BN_, CG_, true>(p, stream);
+    QL_FCASE(128, 1)
+    QL_FCASE(192, 1)
+    QL_FCASE(224, 1)
+    QL_FCASE(256, 1)
+    QL_FCASE(128, 2)
+    QL_FCASE(192, 2)
+    QL_FCASE(224, 2)
+    QL_FCASE(256, 2)
+#undef QL_FCASE
+    return cudaErrorInvalidValue;
+  }
 #define QL_CASE(FP4_, BN_, CG_) \
-  if (p.fp4 == FP4_ && p.bn == BN_ && p.cg == CG_) return launch_typed<FP4_, BN_, CG_>(p, stream);
+  if (p.fp4 == FP4_ && p.bn == BN_ && p.cg == CG_) return launch_typed<FP4_, BN_, CG_, false>(p, stream);
   QL_CASE(true, 128, 1)
   QL_CASE(true, 192, 1)
   QL_CASE(true, 256, 1)

@@ -33,6 +33,14 @@ struct GemmProblem {
   uint64_t timeout_ns;
   int inject_fault;
   bool pdl;              // launched right after its producer kernel (programmatic dependency)
+  // fused (FP4, K % 256 == 0): the launch first quantizes x into a (codes) and
+  // sfa (scale atoms) and lays out the row-major weight scales into sfb (atoms for
+  // tile width bn), then runs the GEMM on them
+  bool fused;
+  const void* x;             // bf16 [M, K]
+  const uint8_t* w_scale;    // E4M3 [N, K/16] row-major
+  uint64_t* sync;            // 8 words (64 bytes) in the workspace
+  uint32_t tag;              // odd, different from the previous launch on this workspace
 };
 
 GemmConfig choose_config(bool fp4, int64_t M, int64_t N, int64_t K);

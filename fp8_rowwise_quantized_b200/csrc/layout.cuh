@@ -50,9 +50,10 @@ __host__ __device__ inline size_t sf_wgt_word_offset(int64_t n_tile, int64_t nn,
 }
 
 // nvfp4_linear workspace: [packed activation codes M x K/2][activation scale atoms]
+// [synchronisation words of the single-launch path: 64 bytes]
 // [weight scale atoms for the chosen tile width], each part 1024-byte aligned.
 struct Nvfp4Workspace {
-  size_t codes_off, act_sf_off, wgt_sf_off, total;
+  size_t codes_off, act_sf_off, sync_off, wgt_sf_off, total;
 };
 
 __host__ __device__ inline Nvfp4Workspace nvfp4_workspace(int64_t M, int64_t K, int64_t N, int bn) {
@@ -62,9 +63,11 @@ __host__ __device__ inline Nvfp4Workspace nvfp4_workspace(int64_t M, int64_t K, 
   size_t codes = static_cast<size_t>(M) * static_cast<size_t>(K / 2);
   size_t act_sf = static_cast<size_t>(ceil_div64(M, 128) * KG) * kSfAtomBytes;
   size_t wgt_sf = static_cast<size_t>(ceil_div64(N, bn) * KG * na) * kSfAtomBytes;
+  size_t sync = 64;
   w.codes_off = 0;
   w.act_sf_off = align_up(codes, 1024);
-  w.wgt_sf_off = align_up(w.act_sf_off + act_sf, 1024);
+  w.sync_off = align_up(w.act_sf_off + act_sf, 1024);
+  w.wgt_sf_off = align_up(w.sync_off + sync, 1024);
   w.total = align_up(w.wgt_sf_off + wgt_sf, 1024);
   return w;
 }

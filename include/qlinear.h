@@ -85,6 +85,8 @@ size_t nvfp4_linear_workspace_size(int64_t M, int64_t K, int64_t N);
 
 /* NVFP4 W4A4 linear forward: quantizes x at run time with input_scale and
  * contracts it on the tensor cores against the pre-quantized weight.
+ * Two launches on `stream`: nvfp4_linear_prologue, then nvfp4_linear_gemm
+ * (started early through programmatic dependent launch).
  *   x              bf16 [M, K]
  *   w              uint8 [N, K/2]  packed E2M1 weight codes
  *   w_scale        uint8 [N, K/16] E4M3 weight block scales (row-major, as stored
@@ -96,12 +98,33 @@ size_t nvfp4_linear_workspace_size(int64_t M, int64_t K, int64_t N);
  *   workspace      device buffer of >= nvfp4_linear_workspace_size(M, K, N) bytes;
  *                  holds the quantized activations and the scale layouts between
  *                  the two kernels of one call (its contents are internal)
+ *                  Calls that overlap on the GPU must not share a workspace.
  * Requires M, N >= 1, K >= 32, K % 32 == 0 (16-byte aligned packed rows). */
 int nvfp4_linear(const void* x, int64_t M, int64_t K,
                  const uint8_t* w, const uint8_t* w_scale, int64_t N,
                  const float* weight_scale_2, const float* input_scale,
                  const float* bias, void* y,
                  void* workspace, size_t workspace_bytes, ql_stream_t stream);
+
+/* The same NVFP4 linear as ONE kernel launch (the "GEMM-prologue fusion" of the
+ * activation quantization): every warp of the GEMM's persistent grid first
+ * quantizes its share of x (codes and scales into the workspace, which stays in
+ * L2) and lays out the weight scales, the CTAs meet at a grid-wide barrier, then
+ * the same GEMM as nvfp4_linear_gemm runs. Gives the same bits as nvfp4_linear.
+ * Measured slower than nvfp4_linear on B200 for the diffusion-transformer layers:
+ * the quantization gets the GEMM's one CTA of 8 warps per SM instead of a full
+ * grid of its own.
+ *   arguments as nvfp4_linear; workspace of nvfp4_linear_workspace_size bytes,
+ *   which need not be cleared: the barrier's words in it carry a per-call tag,
+ *   and every call leaves them zero. Calls that overlap on the GPU must not share
+ *   a workspace.
+ * Requires K % 256 == 0 (QL_ERR_SHAPE otherwise) and a 16-byte aligned w_scale.
+ * The barrier's wait is bounded: if some CTA of the grid cannot start (e.g. on a
+ * partitioned GPU) the call ends with QL_ERR_TIMEOUT in the device status word. */
+int nvfp4_linear_single_launch(const void* x, int64_t M, int64_t K, const uint8_t* w,
+                               const uint8_t* w_scale, int64_t N, const float* weight_scale_2,
+                               const float* input_scale, const float* bias, void* y,
+                               void* workspace, size_t workspace_bytes, ql_stream_t stream);
 
 /* The two halves of nvfp4_linear, for callers that time or schedule them apart.
  * nvfp4_linear == nvfp4_linear_prologue followed by nvfp4_linear_gemm on the same
