@@ -266,18 +266,11 @@ def source_hash(files):
 
 # ----------------------------------------------------------------------------- CPU oracle
 
-def cpu_oracle_sample(M, K, N, target_s=12.0, min_rows=4):
-    """Time the oracle (as it stands) on a bounded row sample of the workload:
-    activation quantization of the sampled rows + fp64 contraction against the
-    whole weight. Returns (TFLOP/s, threads, rows, seconds)."""
-    import numpy as np
+def oracle_rows_for(seconds, x, gx, wq, ws, gw, M):
+    """Activation rows whose oracle run (quantize + fp64 contraction against the
+    whole weight) takes about `seconds`: two timed sizes separate the per-call cost
+    (the weight's dequantization) from the per-row cost."""
     import oracle
-    from synthetic import make_linear_inputs
-    inp = make_linear_inputs(M, K, N, seed=0)
-    gw = oracle.nvfp4_global_scale(inp.w)
-    wq, ws = oracle.nvfp4_quantize(inp.w, gw)
-    gx = oracle.nvfp4_global_scale(inp.x)
-    x = inp.x
 
     def run(rows):
         t0 = time.perf_counter()
@@ -285,13 +278,36 @@ def cpu_oracle_sample(M, K, N, target_s=12.0, min_rows=4):
         oracle.nvfp4_linear(xq, xs, wq, ws, gx, gw)
         return time.perf_counter() - t0
 
-    rows = min_rows
-    t = run(rows)
-    if t < target_s / 4:
-        rows = int(min(M, max(rows, rows * (target_s / max(t, 1e-3)) * 0.9)))
-        t = run(rows)
-    tflops = nvfp4_flops(rows, K, N) / t / 1e12
-    return tflops, oracle.get_threads(), rows, t
+    # the oracle spreads rows over its threads: time whole multiples of them
+    th = max(1, oracle.get_threads())
+    a, b = min(M, 2 * th), min(M, 6 * th)
+    t_a = run(a)
+    if b == a:
+        return a
+    t_b = run(b)
+    per_row = max((t_b - t_a) / (b - a), 1e-6)
+    fixed = max(t_a - a * per_row, 0.0)
+    rows = int((seconds - fixed) / per_row) // th * th
+    return int(max(1, min(M, max(rows, th))))
+
+
+def cpu_oracle_sample(M, K, N, target_s=15.0):
+    """Time the oracle (as it stands) on a bounded row sample of the workload:
+    activation quantization of the sampled rows + fp64 contraction against the
+    whole weight, sized to about `target_s` seconds. Returns (TFLOP/s, threads,
+    rows, seconds)."""
+    import oracle
+    from synthetic import make_linear_inputs
+    inp = make_linear_inputs(M, K, N, seed=0)
+    gw = oracle.nvfp4_global_scale(inp.w)
+    wq, ws = oracle.nvfp4_quantize(inp.w, gw)
+    gx = oracle.nvfp4_global_scale(inp.x)
+    rows = oracle_rows_for(target_s, inp.x, gx, wq, ws, gw, M)
+    t0 = time.perf_counter()
+    xq, xs = oracle.nvfp4_quantize(inp.x[:rows], gx)
+    oracle.nvfp4_linear(xq, xs, wq, ws, gx, gw)
+    t = time.perf_counter() - t0
+    return nvfp4_flops(rows, K, N) / t / 1e12, oracle.get_threads(), rows, t
 
 
 # ----------------------------------------------------------------------------- arms
@@ -311,12 +327,8 @@ def run_reference(args):
     wq, ws = oracle.nvfp4_quantize(inp.w, gw)
     gx = oracle.nvfp4_global_scale(inp.x)
     # size one step so that warmup + steps take about two minutes in total
-    t0 = time.perf_counter()
-    xq, xs = oracle.nvfp4_quantize(inp.x[:4], gx)
-    oracle.nvfp4_linear(xq, xs, wq, ws, gx, gw)
-    t4 = time.perf_counter() - t0
     per_step = 120.0 / max(1, args.steps + args.warmup)
-    rows = int(max(1, min(M, 4 * per_step / max(t4, 1e-3))))
+    rows = oracle_rows_for(per_step, inp.x, gx, wq, ws, gw, M)
     times = []
     for i in range(args.warmup + args.steps):
         t0 = time.perf_counter()
@@ -391,6 +403,7 @@ def run_ours(args):
 
     # --------------------------------------------------- roofline of the GEMM kernel
     fp4_peak = peaks["bf16_tflops"] * NOMINAL_FP4_OVER_BF16
+    tile_bn, tile_cg = q.tile_config(M, N, K)
     roof_steps = max(20, min(args.steps, 200))
     layer.prologue()
     gemm_ms, _ = time_events(layer.gemm, roof_steps, 3, flush, stream)
@@ -403,7 +416,8 @@ def run_ours(args):
     gemm_tflops = flops / (gemm_ms / 1e3) / 1e12
     prologue_bytes = 2 * M * K + M * K // 2 + M * K // 16 + 2 * (N * K // 16)
     roofline = {
-        "kernel": "qgemm_kernel<FP4, BN=192> (tcgen05 block-scaled FP4 GEMM)",
+        "kernel": f"qgemm_kernel<FP4, BN={tile_bn}, {'CTA pair' if tile_cg == 2 else 'one CTA'}> "
+                  "(tcgen05 block-scaled FP4 GEMM)",
         "bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
         "frac": gemm_tflops / fp4_peak,
         "traffic": traffic_from_profiles("nvfp4_gemm_mlp_up"),

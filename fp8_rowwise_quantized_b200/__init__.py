@@ -25,7 +25,7 @@ __all__ = [
     "nvfp4_linear_workspace_size", "nvfp4_linear_workspace_layout", "nvfp4_global_scale",
     "fp8r_quantize_rows", "fp8r_linear", "fp8r_linear_gemm", "fp8r_linear_workspace_size",
     "ql_encode_e4m3", "ql_encode_e2m1", "read_device_status", "set_fault_injection",
-    "set_tile_override",
+    "set_tile_override", "tile_config",
     "prepare_nvfp4_weight", "prepare_fp8r_weight", "QLinearError", "library_path",
 ]
 
@@ -307,6 +307,14 @@ def read_device_status() -> int:
 
 def set_fault_injection(enable: bool, timeout_ms: int = 0) -> None:
     _lib.load().ql_set_fault_injection(1 if enable else 0, int(timeout_ms))
+
+
+def tile_config(M: int, N: int, K: int, fp4: bool = True) -> Tuple[int, int]:
+    """(bn, cg) of the GEMM tiles a call of this size uses: (128 * cg) x bn."""
+    bn, cg = _lib.C.c_int(), _lib.C.c_int()
+    _lib.check("ql_tile_config", _lib.load().ql_tile_config(
+        1 if fp4 else 0, M, N, K, _lib.C.byref(bn), _lib.C.byref(cg)))
+    return bn.value, cg.value
 
 
 def set_tile_override(bn: int = 0, cg: int = 0) -> None:

@@ -47,6 +47,8 @@ SIGNATURES = {
     "ql_read_device_status": (C.c_int, [C.POINTER(C.c_int)]),
     "ql_set_fault_injection": (None, [C.c_int, C.c_int]),
     "ql_set_tile_override": (C.c_int, [C.c_int, C.c_int]),
+    "ql_tile_config": (C.c_int, [C.c_int, _i64, _i64, _i64, C.POINTER(C.c_int),
+                                 C.POINTER(C.c_int)]),
     "ql_status_string": (C.c_char_p, [C.c_int]),
     "ql_last_error_message": (C.c_char_p, []),
 }

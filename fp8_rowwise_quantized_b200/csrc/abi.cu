@@ -168,6 +168,14 @@ size_t nvfp4_linear_workspace_size(int64_t M, int64_t K, int64_t N) {
   return need;
 }
 
+int ql_tile_config(int fp4, int64_t M, int64_t N, int64_t K, int* bn, int* cg) {
+  if (!bn || !cg || M < 1 || N < 1 || K < 1) return QL_ERR_INVALID_ARG;
+  const ql::GemmConfig c = ql::choose_config(fp4 != 0, M, N, K);
+  *bn = c.bn;
+  *cg = c.cg;
+  return QL_OK;
+}
+
 int ql_set_tile_override(int bn, int cg) {
   return ql::set_tile_override(bn, cg) ? QL_OK : QL_ERR_INVALID_ARG;
 }

@@ -233,6 +233,12 @@ void ql_set_fault_injection(int enable, int timeout_ms);
  * Returns QL_OK or QL_ERR_INVALID_ARG. Workspace sizes already cover every tile. */
 int ql_set_tile_override(int bn, int cg);
 
+/* The GEMM tile shape a call of this size would use now (the automatic choice, or
+ * the override): bn columns, cg = 1 (one SM per 128-row tile) or 2 (a CTA pair per
+ * 256-row tile). fp4 = 1 for the NVFP4 GEMM, 0 for fp8r. Host only; bn and cg
+ * are written only on QL_OK. QL_ERR_INVALID_ARG for null outputs or sizes < 1. */
+int ql_tile_config(int fp4, int64_t M, int64_t N, int64_t K, int* bn, int* cg);
+
 /* Text of a status code, and of the last CUDA error recorded by this thread. */
 const char* ql_status_string(int status);
 const char* ql_last_error_message(void);

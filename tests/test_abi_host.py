@@ -24,7 +24,7 @@ def declared_functions():
 def test_library_exports_every_declared_symbol():
     lib = _lib.load()
     names = declared_functions()
-    assert len(names) >= 20, names
+    assert len(names) >= 21, names
     for n in names:
         assert hasattr(lib, n), f"missing export {n}"
     assert set(names) == set(_lib.SIGNATURES), set(names) ^ set(_lib.SIGNATURES)
@@ -90,3 +90,18 @@ def test_no_device_reports_error_instead_of_crashing():
     assert lib.ql_last_error_message().decode()
     st = C.c_int(-1)
     assert lib.ql_read_device_status(C.byref(st)) in (4, 6)
+
+
+def test_tile_config_is_host_only_and_follows_override():
+    import fp8_rowwise_quantized_b200 as q
+    bn, cg = q.tile_config(4096, 12288, 3072)
+    assert bn in (128, 192, 224, 256) and cg == 2       # 256-row pair tiles once M >= 512
+    assert q.tile_config(128, 256, 256)[1] == 1        # one CTA per 128-row tile below that
+    q.set_tile_override(192, 1)
+    try:
+        assert q.tile_config(4096, 12288, 3072) == (192, 1)
+    finally:
+        q.set_tile_override(0, 0)
+    assert q.tile_config(4096, 12288, 3072) == (bn, cg)
+    lib = _lib.load()
+    assert lib.ql_tile_config(1, 0, 1, 1, None, None) == _lib.QL_ERR_INVALID_ARG
