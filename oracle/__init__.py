@@ -42,6 +42,9 @@ def lib():
         L.oracle_bf16_from_double.argtypes = [C.c_double]
         L.oracle_bf16_from_double.restype = C.c_uint16
         L.oracle_bf16_from_double_array.argtypes = [f64p, i64, u16p]
+        L.oracle_gelu.argtypes = [C.c_double]
+        L.oracle_gelu.restype = C.c_double
+        L.oracle_gelu_bf16.argtypes = [u16p, i64, C.c_double, u16p, u8p]
         L.oracle_nvfp4_global_scale.argtypes = [u16p, i64]
         L.oracle_nvfp4_global_scale.restype = C.c_float
         L.oracle_nvfp4_quantize.argtypes = [u16p, i64, i64, C.c_float, u8p, u8p]
@@ -128,6 +131,23 @@ def bf16_from_double(v) -> np.ndarray:
     out = np.empty(v.shape, np.uint16)
     lib().oracle_bf16_from_double_array(_p(v, C.c_double), v.size, _p(out, C.c_uint16))
     return out
+
+
+def gelu(v: float) -> float:
+    """Exact GELU v * Phi(v) in fp64 (oracle_gelu)."""
+    return lib().oracle_gelu(float(v))
+
+
+def gelu_bf16(y, rel_tol: float = 2.0 ** -19):
+    """bf16(GELU(y)) of a bf16 tensor (torch bf16 or uint16 bits), in fp64, plus the
+    mask of elements whose exact GELU lies within rel_tol * |value| of a bf16
+    rounding midpoint (where an fp32 evaluation may round the other way)."""
+    bits = _bits16(y)
+    h = np.empty(bits.shape, dtype=np.uint16)
+    amb = np.empty(bits.shape, dtype=np.uint8)
+    lib().oracle_gelu_bf16(_p(bits, C.c_uint16), bits.size, float(rel_tol),
+                           _p(h, C.c_uint16), _p(amb, C.c_uint8))
+    return h, amb.astype(bool)
 
 
 def nvfp4_global_scale(x) -> float:

@@ -218,6 +218,39 @@ void oracle_bf16_from_double_array(const double* v, int64_t n, uint16_t* out) {
 }
 
 // ---------------------------------------------------------------------------
+// GELU of a bf16 tensor, back to bf16: the activation between the MLP's two
+// linear layers, which the fused up-projection epilogue quantizes for the down
+// projection. The pages name "fused GELU/MLP" kernels only (Nunchaku section);
+// this file takes the exact (erf) GELU, GELU(v) = v * Phi(v), Phi the standard
+// normal CDF, written with erfc so that it stays accurate for large negative v:
+//   Phi(v) = erfc(-v / sqrt(2)) / 2,   h = bf16( v * Phi(v) ), in fp64.
+// A GPU that evaluates GELU in fp32 (error a few fp32 ulps) can round to the
+// other bf16 neighbour only when the exact value lies within that error of the
+// midpoint of two bf16 values; `ambiguous[i]` = 1 marks those elements: the fp64
+// value within rel_tol * |value| of such a midpoint.
+// ---------------------------------------------------------------------------
+double oracle_gelu(double v) { return 0.5 * v * std::erfc(-v / std::sqrt(2.0)); }
+
+void oracle_gelu_bf16(const uint16_t* y, int64_t n, double rel_tol, uint16_t* h,
+                      uint8_t* ambiguous) {
+  for (int64_t i = 0; i < n; ++i) {
+    const double g = oracle_gelu(static_cast<double>(bf16_to_float(y[i])));
+    const uint16_t b = oracle_bf16_from_double(g);
+    h[i] = b;
+    if (ambiguous) {
+      // the bf16 neighbours of g: b and the next value away from b on g's side
+      const double vb = static_cast<double>(bf16_to_float(b));
+      uint16_t other = b;
+      if (g > vb) other = (b & 0x8000) ? (b == 0x8000 ? 0x0001 : b - 1) : b + 1;
+      else if (g < vb) other = (b & 0x8000) ? b + 1 : (b == 0x0000 ? 0x8001 : b - 1);
+      const double vo = static_cast<double>(bf16_to_float(other));
+      const double mid = 0.5 * (vb + vo);
+      ambiguous[i] = (g != vb && std::fabs(g - mid) <= rel_tol * std::fabs(g)) ? 1 : 0;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Calibration rule of the workloads: global scale = amax / (6 * 448), i.e. the
 // largest magnitude maps onto the largest E2M1 value times the largest E4M3
 // scale. fp32 division, one rounding. The pages only say "calibrated".
