@@ -221,6 +221,40 @@ class Fp8rLayer:
         self.q.fp8r_linear_gemm(self.xq, self.xs, self.wq, self.wsc, bias=self.bias, y=self.y)
 
 
+class MlpBlock:
+    """Diffusion-transformer MLP block on the device: up projection (K -> H), exact
+    GELU, down projection (H -> K), both NVFP4. The down projection's input_scale
+    is calibrated once, from an unfused run (amax of GELU(up) / 2688), and then
+    held fixed, as a deployed model would."""
+
+    def __init__(self, M, K, H, device, seed=0):
+        import torch
+        import fp8_rowwise_quantized_b200 as q
+        self.up = Nvfp4Layer(M, K, H, False, device, seed=seed)
+        self.down = Nvfp4Layer(M, H, K, False, device, seed=seed + 1)
+        self.q, self.M = q, M
+        y = q.nvfp4_linear(self.up.x, self.up.wq, self.up.ws, self.up.gw, self.up.gx)
+        self.h = torch.nn.functional.gelu(y.float()).to(torch.bfloat16)
+        self.g_down = q.nvfp4_global_scale(self.h)
+        self.y = torch.empty((M, K), dtype=torch.bfloat16, device=device)
+
+    def fused(self):
+        q = self.q
+        q.nvfp4_linear_gelu_quantize(self.up.x, self.up.wq, self.up.ws, self.up.gw, self.up.gx,
+                                     self.g_down, self.down.work, workspace=self.up.work)
+        q.nvfp4_linear_quantized_input(self.M, self.down.wq, self.down.ws, self.down.gw,
+                                       self.g_down, self.down.work, y=self.y)
+
+    def unfused(self):
+        import torch
+        q = self.q
+        q.nvfp4_linear(self.up.x, self.up.wq, self.up.ws, self.up.gw, self.up.gx, y=self.up.y,
+                       workspace=self.up.work)
+        h = torch.nn.functional.gelu(self.up.y.float()).to(torch.bfloat16)
+        q.nvfp4_linear(h, self.down.wq, self.down.ws, self.down.gw, self.g_down, y=self.y,
+                       workspace=self.down.work)
+
+
 def time_events(fn, steps, warmup, flush, stream):
     """Mean device time (ms) of fn over `steps` calls, each bracketed by CUDA events
     on `stream`, with an L2 flush (outside the events) before every call."""
@@ -471,6 +505,17 @@ def run_ours(args):
                               "gemm_us": gms * 1e3, "gemm_tflops": fl / (gms / 1e3) / 1e12,
                               "gemm_frac_of_peak": fl / (gms / 1e3) / 1e12 / pk}
             del L
+        torch.cuda.empty_cache()
+        # MLP block (up 3072 -> 12288, GELU, down 12288 -> 3072): fused GELU + NVFP4
+        # requantization epilogue vs up linear, torch GELU, down linear
+        mlp = MlpBlock(4096, 3072, 12288, device)
+        f_ms, _ = time_events(mlp.fused, v_steps, 3, flush, stream)
+        u_ms, _ = time_events(mlp.unfused, v_steps, 3, flush, stream)
+        mlp_flops = 2 * nvfp4_flops(4096, 3072, 12288)
+        variants["nvfp4_mlp_block_4096x3072x12288"] = {
+            "fused_us": f_ms * 1e3, "fused_tflops": mlp_flops / (f_ms / 1e3) / 1e12,
+            "unfused_us": u_ms * 1e3, "unfused_tflops": mlp_flops / (u_ms / 1e3) / 1e12}
+        del mlp
         torch.cuda.empty_cache()
         # GEMM tile sweep on the headline layer: (128 * cg) x bn output tiles
         sweep = {}

@@ -20,7 +20,7 @@ from . import _lib
 
 __all__ = [
     "nvfp4_quantize_act", "nvfp4_linear", "nvfp4_linear_single_launch", "nvfp4_linear_noalloc",
-    "nvfp4_linear_prologue",
+    "nvfp4_linear_prologue", "nvfp4_linear_gelu_quantize", "nvfp4_linear_quantized_input",
     "nvfp4_linear_gemm",
     "nvfp4_linear_workspace_size", "nvfp4_linear_workspace_layout", "nvfp4_global_scale",
     "fp8r_quantize_rows", "fp8r_linear", "fp8r_linear_gemm", "fp8r_linear_workspace_size",
@@ -148,6 +148,59 @@ def nvfp4_linear_single_launch(x: torch.Tensor, w: torch.Tensor, w_scale: torch.
     _lib.check("nvfp4_linear_single_launch", _lib.load().nvfp4_linear_single_launch(
         _ptr(x), M, K, _ptr(w), _ptr(w_scale), N, _ptr(weight_scale_2), _ptr(input_scale),
         _ptr(bias), _ptr(y), _ptr(ws), ws.numel(), _stream()))
+    return y
+
+
+def nvfp4_linear_gelu_quantize(x: torch.Tensor, w: torch.Tensor, w_scale: torch.Tensor,
+                               weight_scale_2: torch.Tensor, input_scale: torch.Tensor,
+                               next_input_scale: torch.Tensor, next_workspace: torch.Tensor,
+                               bias: Optional[torch.Tensor] = None,
+                               workspace: Optional[torch.Tensor] = None) -> None:
+    """MLP up projection + GELU + NVFP4 quantization for the down projection: writes
+    NVFP4(GELU(linear)) (global scale next_input_scale) into the activation part of
+    next_workspace, a uint8 buffer of nvfp4_linear_workspace_size(M, N, N_down)
+    bytes, for nvfp4_linear_quantized_input. Needs N % 256 == 0."""
+    _need(x, "x", torch.bfloat16, 2)
+    _need(w, "w", torch.uint8, 2)
+    _need(w_scale, "w_scale", torch.uint8, 2)
+    _need(next_workspace, "next_workspace", torch.uint8, 1)
+    _scalar(weight_scale_2, "weight_scale_2")
+    _scalar(input_scale, "input_scale")
+    _scalar(next_input_scale, "next_input_scale")
+    M, K = x.shape
+    N = w.shape[0]
+    if w.shape[1] * 2 != K or tuple(w_scale.shape) != (N, K // 16):
+        raise ValueError("weight shapes do not match x")
+    if bias is not None:
+        _need(bias, "bias", torch.float32, 1)
+    ws = _workspace(nvfp4_linear_workspace_size(M, K, N), x.device, workspace)
+    _lib.check("nvfp4_linear_gelu_quantize", _lib.load().nvfp4_linear_gelu_quantize(
+        _ptr(x), M, K, _ptr(w), _ptr(w_scale), N, _ptr(weight_scale_2), _ptr(input_scale),
+        _ptr(bias), _ptr(next_input_scale), _ptr(next_workspace), next_workspace.numel(),
+        _ptr(ws), ws.numel(), _stream()))
+
+
+def nvfp4_linear_quantized_input(M: int, w: torch.Tensor, w_scale: torch.Tensor,
+                                 weight_scale_2: torch.Tensor, input_scale: torch.Tensor,
+                                 workspace: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                                 y: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """nvfp4_linear on activations already quantized into `workspace` (by
+    nvfp4_linear_gelu_quantize): weight-scale layout, then the GEMM."""
+    _need(w, "w", torch.uint8, 2)
+    _need(w_scale, "w_scale", torch.uint8, 2)
+    _need(workspace, "workspace", torch.uint8, 1)
+    _scalar(weight_scale_2, "weight_scale_2")
+    _scalar(input_scale, "input_scale")
+    N, K = w.shape[0], w.shape[1] * 2
+    if tuple(w_scale.shape) != (N, K // 16):
+        raise ValueError("weight scale shape does not match w")
+    if bias is not None:
+        _need(bias, "bias", torch.float32, 1)
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=w.device)
+    _lib.check("nvfp4_linear_quantized_input", _lib.load().nvfp4_linear_quantized_input(
+        M, K, _ptr(w), _ptr(w_scale), N, _ptr(weight_scale_2), _ptr(input_scale), _ptr(bias),
+        _ptr(y), _ptr(workspace), workspace.numel(), _stream()))
     return y
 
 

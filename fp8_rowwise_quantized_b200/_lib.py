@@ -30,6 +30,10 @@ SIGNATURES = {
                                _sz, _vp]),
     "nvfp4_linear_single_launch": (C.c_int, [_vp, _i64, _i64, _u8p, _u8p, _i64, _f32p, _f32p,
                                              _f32p, _vp, _vp, _sz, _vp]),
+    "nvfp4_linear_gelu_quantize": (C.c_int, [_vp, _i64, _i64, _u8p, _u8p, _i64, _f32p, _f32p,
+                                             _f32p, _f32p, _vp, _sz, _vp, _sz, _vp]),
+    "nvfp4_linear_quantized_input": (C.c_int, [_i64, _i64, _u8p, _u8p, _i64, _f32p, _f32p,
+                                               _f32p, _vp, _vp, _sz, _vp]),
     "nvfp4_linear_prologue": (C.c_int, [_vp, _i64, _i64, _u8p, _i64, _f32p, _vp, _sz, _vp]),
     "nvfp4_linear_gemm": (C.c_int, [_i64, _i64, _u8p, _i64, _f32p, _f32p, _f32p, _vp, _vp, _sz,
                                     _vp]),

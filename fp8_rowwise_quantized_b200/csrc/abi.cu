@@ -322,6 +322,83 @@ int nvfp4_linear_single_launch(const void* x, int64_t M, int64_t K, const uint8_
   return e == cudaSuccess ? QL_OK : record(e, "nvfp4_linear_single_launch");
 }
 
+int nvfp4_linear_gelu_quantize(const void* x, int64_t M, int64_t K, const uint8_t* w,
+                               const uint8_t* w_scale, int64_t N, const float* weight_scale_2,
+                               const float* input_scale, const float* bias,
+                               const float* next_input_scale, void* next_workspace,
+                               size_t next_workspace_bytes, void* workspace,
+                               size_t workspace_bytes, ql_stream_t stream) {
+  if (!x || !w || !w_scale || !weight_scale_2 || !input_scale || !next_input_scale ||
+      !next_workspace || M <= 0 || N <= 0 || K <= 0)
+    return QL_ERR_INVALID_ARG;
+  if (!nvfp4_shape_ok(M, K, N)) return fail_shape("nvfp4: needs K >= 32 and K % 32 == 0");
+  if (N % 256 != 0) return fail_shape("nvfp4_linear_gelu_quantize: needs N % 256 == 0");
+  if (!aligned16(x) || !aligned16(w) || (bias && !aligned16(bias)) || !aligned16(next_workspace))
+    return QL_ERR_ALIGN;
+  // the next layer's activations: K' = N; their part of its workspace does not
+  // depend on its N' or tile width
+  const ql::Nvfp4Workspace next = ql::nvfp4_workspace(M, N, 1, 128);
+  const size_t next_need = next.act_sf_off + static_cast<size_t>((M + 127) / 128) *
+                                                 static_cast<size_t>(N / 64) * ql::kSfAtomBytes;
+  if (next_workspace_bytes < next_need) return QL_ERR_WORKSPACE;
+  int rc = nvfp4_linear_prologue(x, M, K, w_scale, N, input_scale, workspace, workspace_bytes,
+                                 stream);
+  if (rc != QL_OK) return rc;
+  int dev = 0;
+  rc = check_device(&dev);
+  if (rc != QL_OK) return rc;
+  const ql::GemmConfig cfg = ql::choose_config(true, M, N, K);
+  const ql::Nvfp4Workspace L = ql::nvfp4_workspace(M, K, N, cfg.bn);
+  const uint8_t* ws = static_cast<const uint8_t*>(workspace);
+  uint8_t* nws = static_cast<uint8_t*>(next_workspace);
+  ql::GemmProblem p{};
+  p.fp4 = true;
+  p.bn = cfg.bn;
+  p.cg = cfg.cg;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.a = ws + L.codes_off;
+  p.b = w;
+  p.sfa = ws + L.act_sf_off;
+  p.sfb = ws + L.wgt_sf_off;
+  p.scale_a = input_scale;
+  p.scale_b = weight_scale_2;
+  p.bias = bias;
+  p.y = nullptr;
+  p.status = status_ptr(dev);
+  p.timeout_ns = timeout_ns();
+  p.inject_fault = g_inject_fault.load();
+  p.pdl = true;
+  p.gelu_quant = true;
+  p.gq_codes = nws + next.codes_off;
+  p.gq_atoms = nws + next.act_sf_off;
+  p.gq_scale = next_input_scale;
+  cudaError_t e = ql::launch_gemm(p, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QL_OK : record(e, "nvfp4_linear_gelu_quantize");
+}
+
+int nvfp4_linear_quantized_input(int64_t M, int64_t K, const uint8_t* w, const uint8_t* w_scale,
+                                 int64_t N, const float* weight_scale_2,
+                                 const float* input_scale, const float* bias, void* y,
+                                 void* workspace, size_t workspace_bytes, ql_stream_t stream) {
+  if (!w || !w_scale || !weight_scale_2 || !input_scale || !y || !workspace || M <= 0 ||
+      N <= 0 || K <= 0)
+    return QL_ERR_INVALID_ARG;
+  if (!nvfp4_shape_ok(M, K, N)) return fail_shape("nvfp4: needs K >= 32 and K % 32 == 0");
+  if (workspace_bytes < nvfp4_linear_workspace_size(M, K, N)) return QL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return QL_ERR_ALIGN;
+  int rc = check_device(nullptr);
+  if (rc != QL_OK) return rc;
+  const int bn = ql::choose_config(true, M, N, K).bn;
+  cudaError_t e = ql::launch_nvfp4_weight_layout(w_scale, M, K, N, bn, input_scale,
+                                                 static_cast<uint8_t*>(workspace),
+                                                 reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return record(e, "nvfp4_linear_quantized_input");
+  return nvfp4_gemm_impl(M, K, w, N, weight_scale_2, input_scale, bias, y, workspace,
+                         workspace_bytes, stream, true);
+}
+
 int nvfp4_global_scale(const void* x, int64_t n, float* out, ql_stream_t stream) {
   if (!x || !out || n <= 0) return QL_ERR_INVALID_ARG;
   int rc = check_device(nullptr);

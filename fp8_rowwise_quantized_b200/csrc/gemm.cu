@@ -73,6 +73,10 @@ struct GemmArgs {
   const uint8_t* w_scale;   // weight scales, row-major E4M3 [N, K/16]
   uint8_t* ws_atoms;        // weight scale atoms for tile width BN: written here, read as SFB
   uint64_t* sync;           // sync_words tagged counters (see kSyncBarrier)
+  // GELU-quantize epilogue (FP4): NVFP4 of GELU(Y) with global scale *gq_scale
+  uint8_t* gq_codes;        // packed E2M1 [M, N/2]
+  uint8_t* gq_atoms;        // E4M3 scales in the activation atom layout (K' = N)
+  const float* gq_scale;
   int sync_words;
   uint32_t tag;             // this launch's tag, odd
 };
@@ -283,13 +287,128 @@ __device__ __forceinline__ void weight_scale_job(const GemmArgs& a, int64_t job,
   }
 }
 
-template <bool FP4, int BN, int CG, bool FUSED>
-__global__ void __launch_bounds__(FUSED ? kThreadsFused : kThreads, 1)
+// GELU-quantize epilogue, one lane's row m of one slab (SLAB columns n0 ..):
+//   v = bf16(alpha * acc + bias)        (the value the plain epilogue stores as Y)
+//   h = bf16(0.5 v * erfc(-v / sqrt 2)) (exact GELU, fp32, erfc form for the tail)
+// then h in 16-column blocks as nvfp4_quantize_act quantizes a row (global scale
+// g, c = 1 / (6 g)): codes to gq_codes[m, n0/2 ..], the block scales into the atom
+// layout of the next layer's activations (K' = N, KG' = N/64 groups of 4 scales).
+// Rows in [M, 128-row padding) get zero scales and no codes.
+// The GELU of a bf16 value with 2^-8 <= |v| < 2^6 is read from a table of those
+// 3584 values (the same formula, evaluated once per CTA); other values evaluate
+// it directly. inv_of[s] = 1 / (value(s) * g) per block scale code (0: zero codes).
+constexpr int kGeluTabExpLo = 127 - 8;   // biased bf16 exponents of the table
+constexpr int kGeluTabExps = 14;
+constexpr int kGeluTabSize = 2 * kGeluTabExps * 128;
+
+__device__ __forceinline__ float gelu_bf16_formula(float v) {
+  constexpr float kRsqrt2 = 0.70710678118654752f;
+  const float e = erfcf(__fmul_rn(v, -kRsqrt2));
+  return __bfloat162float(__float2bfloat16_rn(__fmul_rn(__fmul_rn(0.5f, v), e)));
+}
+
+// Table entry i: sign i / (14 * 128), biased exponent 119 + (i / 128) % 14,
+// mantissa i % 128.
+__device__ __forceinline__ float gelu_tab_input(int i) {
+  const uint32_t sign = static_cast<uint32_t>(i / (kGeluTabExps * 128)) << 15;
+  const uint32_t e = static_cast<uint32_t>(kGeluTabExpLo + (i / 128) % kGeluTabExps);
+  const uint32_t bits = sign | (e << 7) | static_cast<uint32_t>(i % 128);
+  return __uint_as_float(bits << 16);
+}
+
+// Branch-free: outside the table, v >= 64 gives v (Phi(v) is 1 in fp32), v <= -64
+// gives -0 (v * Phi(v) is below the bf16 range), and |v| < 2^-8 takes the series
+// Phi(v) = 1/2 + (v - v^3 / 6) / sqrt(2 pi) (truncation below 2^-36 relative there).
+// Selects rather than branches keep the 16 elements of a block in one basic block,
+// so they interleave (measured: a per-lane branch costs 60% more, a table-or-formula
+// branch 2.6x). Nothing here is warp-collective: it runs after per-lane returns.
+__device__ __forceinline__ float gelu_bf16(float v, const uint16_t* tab) {
+  const uint32_t bits = __float_as_uint(v) >> 16;  // v is a bf16 value
+  const int e = static_cast<int>((bits >> 7) & 0xFF) - kGeluTabExpLo;
+  const bool in_tab = static_cast<unsigned>(e) < static_cast<unsigned>(kGeluTabExps);
+  const int i = in_tab ? static_cast<int>(bits >> 15) * (kGeluTabExps * 128) + e * 128 +
+                             static_cast<int>(bits & 127)
+                       : 0;
+  const float t = __uint_as_float(static_cast<uint32_t>(tab[i]) << 16);
+  constexpr float kInvSqrt2Pi = 0.39894228040143268f;
+  const float v2 = __fmul_rn(v, v);
+  const float phi = __fadd_rn(0.5f, __fmul_rn(__fmul_rn(v, kInvSqrt2Pi),
+                                              __fsub_rn(1.0f, __fmul_rn(v2, 1.0f / 6.0f))));
+  const float small = __bfloat162float(__float2bfloat16_rn(__fmul_rn(v, phi)));
+  const float big = v > 0.0f ? v : -0.0f;
+  return in_tab ? t : (e < 0 ? small : big);
+}
+
+template <int SLAB>
+__device__ __forceinline__ void gelu_quant_slab(const GemmArgs& a, const uint32_t (&r)[SLAB],
+                                                const float* cv_bias_slab, float alpha, int m,
+                                                int n0, const uint16_t* gelu_tab,
+                                                const float* inv_of, float cinv) {
+  const int m_pad = (a.M + 127) & ~127;
+  if (m >= m_pad) return;
+  const int64_t kg_total = a.N >> 6;
+  uint8_t* sc = a.gq_atoms + ((static_cast<int64_t>(m >> 7) * kg_total + (n0 >> 6)) * kSfAtomBytes) +
+                (m & 31) * 16 + ((m >> 5) & 3) * 4 + ((n0 & 63) >> 4);
+  if (m >= a.M) {
+    if constexpr (SLAB == 32)
+      *reinterpret_cast<uint16_t*>(sc) = 0;
+    else
+      *reinterpret_cast<uint32_t*>(sc) = 0u;
+    return;
+  }
+  uint32_t scales = 0;
+  uint32_t codes[SLAB / 8];
+#pragma unroll
+  for (int b = 0; b < SLAB / 16; ++b) {
+    float h[16];
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int j = 16 * b + i;
+      const float v =
+          __bfloat162float(__float2bfloat16_rn(__fmaf_rn(__uint_as_float(r[j]), alpha, cv_bias_slab[j])));
+      h[i] = gelu_bf16(v, gelu_tab);
+      amax = fmaxf(amax, fabsf(h[i]));
+    }
+    const uint32_t s = cvt_e4m3x4(__fmul_rn(amax, cinv), 0.0f, 0.0f, 0.0f) & 0x7Fu;
+    const float inv = inv_of[s];
+    float f0[8], f1[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      f0[i] = __fmul_rn(h[i], inv);
+      f1[i] = __fmul_rn(h[8 + i], inv);
+    }
+    codes[2 * b] = inv != 0.0f ? cvt_e2m1x8(f0) : 0u;
+    codes[2 * b + 1] = inv != 0.0f ? cvt_e2m1x8(f1) : 0u;
+    scales |= s << (8 * b);
+  }
+  uint8_t* q = a.gq_codes + static_cast<int64_t>(m) * (a.N >> 1) + (n0 >> 1);
+#pragma unroll
+  for (int i = 0; i < SLAB / 32; ++i)
+    *reinterpret_cast<uint4*>(q + 16 * i) =
+        make_uint4(codes[4 * i], codes[4 * i + 1], codes[4 * i + 2], codes[4 * i + 3]);
+  if constexpr (SLAB == 32)
+    *reinterpret_cast<uint16_t*>(sc) = static_cast<uint16_t>(scales);
+  else
+    *reinterpret_cast<uint32_t*>(sc) = scales;
+}
+
+// Kernel modes: the plain GEMM; the single-launch NVFP4 linear (quantization
+// phase, grid barrier, GEMM); the GEMM whose epilogue writes NVFP4 codes and scale
+// atoms of GELU(Y) instead of Y (the MLP up projection feeding the down projection).
+constexpr int kModePlain = 0;
+constexpr int kModeSingleLaunch = 1;
+constexpr int kModeGeluQuant = 2;
+
+template <bool FP4, int BN, int CG, int MODE>
+__global__ void __launch_bounds__(MODE == kModeSingleLaunch ? kThreadsFused : kThreads, 1)
 qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
              const __grid_constant__ CUtensorMap tmap_sfa,
              const __grid_constant__ CUtensorMap tmap_sfb,
              const __grid_constant__ CUtensorMap tmap_y, const GemmArgs args) {
   using C = Cfg<FP4, BN, CG>;
+  constexpr bool FUSED = MODE == kModeSingleLaunch;
+  constexpr bool GQ = MODE == kModeGeluQuant;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -662,6 +781,24 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     uint32_t acc_phase = 0;
     float alpha = 1.0f;
     if constexpr (FP4) alpha = __fmul_rn(__ldg(args.scale_a), __ldg(args.scale_b));
+    // GELU-quantize: 1 / (6 g), and the GELU and block-reciprocal tables in the
+    // staging memory (this mode stores no Y through it)
+    float gq_c = 0.0f;
+    uint16_t* gelu_tab = reinterpret_cast<uint16_t*>(smem_epi);
+    float* inv_of = reinterpret_cast<float*>(smem_epi + kGeluTabSize * 2);
+    if constexpr (GQ) {
+      static_assert(kGeluTabSize * 2 + 128 * 4 <= C::EPI_BYTES, "tables fit the staging memory");
+      const float g = __ldg(args.gq_scale);
+      gq_c = __frcp_rn(__fmul_rn(6.0f, g));
+      const int t = threadIdx.x - 64;  // 0 .. 127
+      for (int i = t; i < kGeluTabSize; i += 128)
+        gelu_tab[i] = static_cast<uint16_t>(__float_as_uint(gelu_bf16_formula(gelu_tab_input(i))) >> 16);
+      {
+        const float d = __fmul_rn(e4m3_to_float(static_cast<uint32_t>(t)), g);
+        inv_of[t] = d != 0.0f ? __frcp_rn(d) : 0.0f;
+      }
+      asm volatile("bar.sync 2, 128;" ::: "memory");
+    }
     int titer = 0;
     for (int tile = group; tile < args.total_tiles; tile += ngroups, ++titer) {
       int m_blk, n_blk;
@@ -714,6 +851,11 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
         }
         const int n0 = n_blk * BN + sl * C::SLAB;
         if (n0 >= args.N) continue;  // warp-uniform
+        if constexpr (GQ) {
+          gelu_quant_slab<C::SLAB>(args, r, cv_bias + sl * C::SLAB, alpha, m, n0, gelu_tab, inv_of,
+                                   gq_c);
+          continue;
+        }
         if (args.use_tma_store) {
           // columns n0 .. n0+SLAB-1 of this warp's 32 rows: scale, bias, bf16, into a
           // swizzled staging tile, then one TMA store per warp.
@@ -836,10 +978,11 @@ bool encode_2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, uin
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool FP4, int BN, int CG, bool FUSED>
+template <bool FP4, int BN, int CG, int MODE>
 cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
   using Cf = Cfg<FP4, BN, CG>;
-  auto kern = qgemm_kernel<FP4, BN, CG, FUSED>;
+  constexpr bool FUSED = MODE == kModeSingleLaunch;
+  auto kern = qgemm_kernel<FP4, BN, CG, MODE>;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -881,7 +1024,8 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
       return cudaErrorInvalidValue;
     }
   }
-  const bool tma_store = (p.N % 8) == 0 && (reinterpret_cast<uintptr_t>(p.y) & 15) == 0;
+  const bool tma_store = MODE != kModeGeluQuant && (p.N % 8) == 0 &&
+                         (reinterpret_cast<uintptr_t>(p.y) & 15) == 0;
   if (tma_store &&
       !encode_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.y, p.N, p.M, p.N * 2, Cf::SLAB, 32,
                  Cf::SLAB == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
@@ -907,6 +1051,11 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
   a.wait_prior_grid = p.pdl ? 1 : 0;
   a.use_tma_store = tma_store ? 1 : 0;
   a.raster_n = 0;
+  if (MODE == kModeGeluQuant) {
+    a.gq_codes = p.gq_codes;
+    a.gq_atoms = p.gq_atoms;
+    a.gq_scale = p.gq_scale;
+  }
   if (FUSED) {
     a.x = static_cast<const uint16_t*>(p.x);
     a.xq = static_cast<uint8_t*>(const_cast<void*>(p.a));
@@ -1014,10 +1163,26 @@ GemmConfig choose_config(bool fp4, int64_t M, int64_t N, int64_t K) {
 }
 
 cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream) {
+  if (p.gelu_quant) {
+    if (!p.fp4 || p.fused || !p.gq_codes || !p.gq_atoms || !p.gq_scale || p.N % 256 != 0)
+      return cudaErrorInvalidValue;
+#define QL_GCASE(BN_, CG_) \
+  if (p.bn == BN_ && p.cg == CG_) return launch_typed<true, BN_, CG_, kModeGeluQuant>(p, stream);
+    QL_GCASE(128, 1)
+    QL_GCASE(192, 1)
+    QL_GCASE(224, 1)
+    QL_GCASE(256, 1)
+    QL_GCASE(128, 2)
+    QL_GCASE(192, 2)
+    QL_GCASE(224, 2)
+    QL_GCASE(256, 2)
+#undef QL_GCASE
+    return cudaErrorInvalidValue;
+  }
   if (p.fused) {
     if (!p.fp4 || !p.x || !p.w_scale || !p.sync || p.K % kKTileFp4 != 0) return cudaErrorInvalidValue;
 #define QL_FCASE(BN_, CG_) \
-  if (p.bn == BN_ && p.cg == CG_) return launch_typed<true, BN_, CG_, true>(p, stream);
+  if (p.bn == BN_ && p.cg == CG_) return launch_typed<true, BN_, CG_, kModeSingleLaunch>(p, stream);
     QL_FCASE(128, 1)
     QL_FCASE(192, 1)
     QL_FCASE(224, 1)
@@ -1030,7 +1195,7 @@ cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream) {
     return cudaErrorInvalidValue;
   }
 #define QL_CASE(FP4_, BN_, CG_) \
-  if (p.fp4 == FP4_ && p.bn == BN_ && p.cg == CG_) return launch_typed<FP4_, BN_, CG_, false>(p, stream);
+  if (p.fp4 == FP4_ && p.bn == BN_ && p.cg == CG_) return launch_typed<FP4_, BN_, CG_, kModePlain>(p, stream);
   QL_CASE(true, 128, 1)
   QL_CASE(true, 192, 1)
   QL_CASE(true, 256, 1)

@@ -41,6 +41,13 @@ struct GemmProblem {
   const uint8_t* w_scale;    // E4M3 [N, K/16] row-major
   uint64_t* sync;            // 8 words (64 bytes) in the workspace
   uint32_t tag;              // odd, different from the previous launch on this workspace
+  // GELU-quantize epilogue (FP4, N % 256 == 0): instead of y, NVFP4 of GELU(Y) with
+  // global scale *gq_scale into gq_codes [M, N/2] and the activation scale atoms
+  // gq_atoms of a layer with K' = N (rows padded to 128)
+  bool gelu_quant;
+  uint8_t* gq_codes;
+  uint8_t* gq_atoms;
+  const float* gq_scale;
 };
 
 GemmConfig choose_config(bool fp4, int64_t M, int64_t N, int64_t K);
@@ -52,6 +59,10 @@ cudaError_t launch_nvfp4_quantize_rowmajor(const void* x, int64_t M, int64_t K, 
 cudaError_t launch_nvfp4_prologue(const void* x, int64_t M, int64_t K, const uint8_t* w_scale,
                                   int64_t N, int bn, const float* input_scale, uint8_t* workspace,
                                   cudaStream_t s);
+// Weight-scale layout only (the activation part of the workspace is left as is).
+cudaError_t launch_nvfp4_weight_layout(const uint8_t* w_scale, int64_t M, int64_t K, int64_t N,
+                                       int bn, const float* input_scale, uint8_t* workspace,
+                                       cudaStream_t s);
 cudaError_t launch_fp8r_quantize_rows(const void* x, int64_t M, int64_t K, uint8_t* xq,
                                       float* x_scale, cudaStream_t s);
 cudaError_t launch_global_scale(const void* x, int64_t n, float* out, cudaStream_t s);

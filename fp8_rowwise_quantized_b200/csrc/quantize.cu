@@ -385,6 +385,25 @@ cudaError_t launch_nvfp4_prologue(const void* x, int64_t M, int64_t K, const uin
   return cudaGetLastError();
 }
 
+cudaError_t launch_nvfp4_weight_layout(const uint8_t* w_scale, int64_t M, int64_t K, int64_t N,
+                                       int bn, const float* input_scale, uint8_t* workspace,
+                                       cudaStream_t s) {
+  // the prologue kernel with no activation rows: only its weight-scale jobs run
+  const Nvfp4Workspace L = nvfp4_workspace(M, K, N, bn);
+  const int64_t KG = sf_kgroups(K);
+  const int na = (bn + 127) / 128;
+  const int64_t n_tiles = ceil_div64(N, bn);
+  const int64_t w_jobs = n_tiles * na * ceil_div64(KG, kWsGroups);
+  static int64_t wave = 0;
+  if (wave == 0) wave = resident_blocks(nvfp4_prologue_kernel);
+  const int64_t blocks = w_jobs < wave ? w_jobs : wave;
+  nvfp4_prologue_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, 0, s>>>(
+      nullptr, static_cast<int>(M), static_cast<int>(K), input_scale, workspace + L.codes_off,
+      workspace + L.act_sf_off, 0u, static_cast<uint32_t>(ceil_div64(KG * 64, 1024)),
+      static_cast<int>(KG), w_scale, N, bn, na, n_tiles, w_jobs, workspace + L.wgt_sf_off);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_fp8r_quantize_rows(const void* x, int64_t M, int64_t K, uint8_t* xq,
                                       float* x_scale, cudaStream_t s) {
   const int rows_per_block = kQuantThreads / 32;

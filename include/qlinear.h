@@ -80,6 +80,34 @@ enum {
 int nvfp4_quantize_act(const void* x, int64_t M, int64_t K, const float* input_scale,
                        uint8_t* xq, uint8_t* xs, ql_stream_t stream);
 
+/* The MLP up projection with its GELU and the down projection's quantization
+ * fused into the GEMM epilogue (the "fused GELU/MLP" kernels of the Diffusers
+ * page "Nunchaku" section, for the nvfp4 scheme): instead of Y it writes
+ *   H = NVFP4( bf16( GELU( bf16(input_scale * weight_scale_2 * X W^T + bias) ) ) )
+ * with GELU(v) = v * Phi(v) (exact, erfc form, fp32) and the same 16-element block
+ * rule as nvfp4_quantize_act, under the given global scale next_input_scale (the
+ * down projection's calibrated input_scale). H goes straight into the activation
+ * part of the down projection's workspace (a buffer of at least
+ * nvfp4_linear_workspace_size(M, N, N_down) bytes): the next call is
+ * nvfp4_linear_quantized_input on that workspace. X, W, scales and bias as
+ * nvfp4_linear; `workspace` is this layer's own nvfp4_linear workspace.
+ * Requires N % 256 == 0 (the next layer's K). Two launches (prologue, GEMM). */
+int nvfp4_linear_gelu_quantize(const void* x, int64_t M, int64_t K, const uint8_t* w,
+                               const uint8_t* w_scale, int64_t N, const float* weight_scale_2,
+                               const float* input_scale, const float* bias,
+                               const float* next_input_scale, void* next_workspace,
+                               size_t next_workspace_bytes, void* workspace,
+                               size_t workspace_bytes, ql_stream_t stream);
+
+/* nvfp4_linear whose activations are already quantized in `workspace` (by
+ * nvfp4_linear_gelu_quantize of the previous layer, with input_scale as its
+ * next_input_scale): lays out this layer's weight scales, then runs the GEMM.
+ * Arguments as nvfp4_linear_gemm plus w_scale (row-major [N, K/16]). */
+int nvfp4_linear_quantized_input(int64_t M, int64_t K, const uint8_t* w, const uint8_t* w_scale,
+                                 int64_t N, const float* weight_scale_2,
+                                 const float* input_scale, const float* bias, void* y,
+                                 void* workspace, size_t workspace_bytes, ql_stream_t stream);
+
 /* Bytes of workspace nvfp4_linear needs for this problem size (0 on bad sizes). */
 size_t nvfp4_linear_workspace_size(int64_t M, int64_t K, int64_t N);
 

@@ -44,7 +44,7 @@ def lib():
         L.oracle_bf16_from_double_array.argtypes = [f64p, i64, u16p]
         L.oracle_gelu.argtypes = [C.c_double]
         L.oracle_gelu.restype = C.c_double
-        L.oracle_gelu_bf16.argtypes = [u16p, i64, C.c_double, u16p, u8p]
+        L.oracle_gelu_bf16.argtypes = [u16p, i64, C.c_double, C.c_double, u16p, u8p]
         L.oracle_nvfp4_global_scale.argtypes = [u16p, i64]
         L.oracle_nvfp4_global_scale.restype = C.c_float
         L.oracle_nvfp4_quantize.argtypes = [u16p, i64, i64, C.c_float, u8p, u8p]
@@ -138,14 +138,16 @@ def gelu(v: float) -> float:
     return lib().oracle_gelu(float(v))
 
 
-def gelu_bf16(y, rel_tol: float = 2.0 ** -19):
+def gelu_bf16(y, rel_tol: float = 2.0 ** -20, rel_tol_sq: float = 2.0 ** -22):
     """bf16(GELU(y)) of a bf16 tensor (torch bf16 or uint16 bits), in fp64, plus the
-    mask of elements whose exact GELU lies within rel_tol * |value| of a bf16
-    rounding midpoint (where an fp32 evaluation may round the other way)."""
+    mask of elements whose exact GELU lies within (rel_tol + rel_tol_sq * y^2) * |value|
+    of a bf16 rounding midpoint (where an fp32 evaluation may round the other way).
+    The defaults bound an fp32 evaluation 0.5 v * erfcf(-v * RN(1/sqrt 2)) with erfcf
+    within 4 ulp: (v^2 + |v| + 6) fp32 ulps, doubled."""
     bits = _bits16(y)
     h = np.empty(bits.shape, dtype=np.uint16)
     amb = np.empty(bits.shape, dtype=np.uint8)
-    lib().oracle_gelu_bf16(_p(bits, C.c_uint16), bits.size, float(rel_tol),
+    lib().oracle_gelu_bf16(_p(bits, C.c_uint16), bits.size, float(rel_tol), float(rel_tol_sq),
                            _p(h, C.c_uint16), _p(amb, C.c_uint8))
     return h, amb.astype(bool)
 

@@ -224,17 +224,21 @@ void oracle_bf16_from_double_array(const double* v, int64_t n, uint16_t* out) {
 // this file takes the exact (erf) GELU, GELU(v) = v * Phi(v), Phi the standard
 // normal CDF, written with erfc so that it stays accurate for large negative v:
 //   Phi(v) = erfc(-v / sqrt(2)) / 2,   h = bf16( v * Phi(v) ), in fp64.
-// A GPU that evaluates GELU in fp32 (error a few fp32 ulps) can round to the
-// other bf16 neighbour only when the exact value lies within that error of the
-// midpoint of two bf16 values; `ambiguous[i]` = 1 marks those elements: the fp64
-// value within rel_tol * |value| of such a midpoint.
+// A GPU that evaluates GELU in fp32 can round to the other bf16 neighbour only
+// when the exact value lies within its error of the midpoint of two bf16 values;
+// `ambiguous[i]` = 1 marks those elements: the fp64 value within
+// (tol_const + tol_sq * v^2) * |value| of such a midpoint. (The v^2 term: an fp32
+// rounding of v / sqrt(2) moves erfc by its logarithmic derivative, about
+// 2 |v / sqrt(2)|, times |v / sqrt(2)| relative ulps.)
 // ---------------------------------------------------------------------------
 double oracle_gelu(double v) { return 0.5 * v * std::erfc(-v / std::sqrt(2.0)); }
 
-void oracle_gelu_bf16(const uint16_t* y, int64_t n, double rel_tol, uint16_t* h,
+void oracle_gelu_bf16(const uint16_t* y, int64_t n, double tol_const, double tol_sq, uint16_t* h,
                       uint8_t* ambiguous) {
   for (int64_t i = 0; i < n; ++i) {
-    const double g = oracle_gelu(static_cast<double>(bf16_to_float(y[i])));
+    const double v = static_cast<double>(bf16_to_float(y[i]));
+    const double g = oracle_gelu(v);
+    const double rel_tol = tol_const + tol_sq * v * v;
     const uint16_t b = oracle_bf16_from_double(g);
     h[i] = b;
     if (ambiguous) {

@@ -57,12 +57,31 @@ def test_bf16_output_matches_rounded_fp64_value():
     assert oracle.bf16_bits_to_f64(h[-1:])[0] == 100.0
 
 
+def test_ambiguity_band_grows_with_v_squared():
+    # with only the v^2 term, the flag is set exactly where the fp64 GELU lies within
+    # sq * v^2 * |GELU| of the midpoint of its two bf16 neighbours
+    sq = 2.0 ** -16
+    y = np.arange(0x3E00, 0x4100, dtype=np.uint16)  # 0.125 .. 8 in bf16
+    h, amb = oracle.gelu_bf16(y, rel_tol=0.0, rel_tol_sq=sq)
+    v = oracle.bf16_bits_to_f64(y)
+    g = np.array([oracle.gelu(t) for t in v])
+    hv = oracle.bf16_bits_to_f64(h)
+    other = np.where(g > hv, h + 1, h - 1).astype(np.uint16)
+    mid = 0.5 * (hv + oracle.bf16_bits_to_f64(other))
+    want = (g != hv) & (np.abs(g - mid) <= sq * v * v * np.abs(g))
+    assert np.array_equal(amb, want)
+    assert amb.any()
+    wider = oracle.gelu_bf16(y, rel_tol=0.0, rel_tol_sq=4 * sq)[1]
+    assert np.all(wider[amb]) and wider.sum() > amb.sum()   # a wider band flags a superset
+    assert not oracle.gelu_bf16(y, rel_tol=0.0, rel_tol_sq=0.0)[1].any()
+
+
 def test_ambiguity_flag_marks_values_near_a_bf16_midpoint():
     # scan bf16 inputs; the flag must be set exactly where the fp64 GELU lies within
     # rel_tol of the midpoint of its two bf16 neighbours
     rel = 2.0 ** -12  # coarse tolerance so that the scan finds flagged values
     y = np.arange(0x3E00, 0x4100, dtype=np.uint16)  # 0.125 .. 8 in bf16
-    h, amb = oracle.gelu_bf16(y, rel_tol=rel)
+    h, amb = oracle.gelu_bf16(y, rel_tol=rel, rel_tol_sq=0.0)
     vals = oracle.bf16_bits_to_f64(y)
     g = np.array([oracle.gelu(v) for v in vals])
     hv = oracle.bf16_bits_to_f64(h)
