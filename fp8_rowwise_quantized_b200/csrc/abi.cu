@@ -341,13 +341,17 @@ int nvfp4_linear_gelu_quantize(const void* x, int64_t M, int64_t K, const uint8_
   const size_t next_need = next.act_sf_off + static_cast<size_t>((M + 127) / 128) *
                                                  static_cast<size_t>(N / 64) * ql::kSfAtomBytes;
   if (next_workspace_bytes < next_need) return QL_ERR_WORKSPACE;
-  int rc = nvfp4_linear_prologue(x, M, K, w_scale, N, input_scale, workspace, workspace_bytes,
-                                 stream);
-  if (rc != QL_OK) return rc;
+  if (!workspace || workspace_bytes < nvfp4_linear_workspace_size(M, K, N)) return QL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return QL_ERR_ALIGN;
   int dev = 0;
-  rc = check_device(&dev);
+  int rc = check_device(&dev);
   if (rc != QL_OK) return rc;
-  const ql::GemmConfig cfg = ql::choose_config(true, M, N, K);
+  // tiles whose accumulator buffers are whole (this epilogue's 8 warps split them)
+  const ql::GemmConfig cfg = ql::choose_config(true, M, N, K, true);
+  cudaError_t pe = ql::launch_nvfp4_prologue(x, M, K, w_scale, N, cfg.bn, input_scale,
+                                             static_cast<uint8_t*>(workspace),
+                                             reinterpret_cast<cudaStream_t>(stream));
+  if (pe != cudaSuccess) return record(pe, "nvfp4_linear_gelu_quantize prologue");
   const ql::Nvfp4Workspace L = ql::nvfp4_workspace(M, K, N, cfg.bn);
   const uint8_t* ws = static_cast<const uint8_t*>(workspace);
   uint8_t* nws = static_cast<uint8_t*>(next_workspace);

@@ -294,11 +294,11 @@ __device__ __forceinline__ void weight_scale_job(const GemmArgs& a, int64_t job,
 // g, c = 1 / (6 g)): codes to gq_codes[m, n0/2 ..], the block scales into the atom
 // layout of the next layer's activations (K' = N, KG' = N/64 groups of 4 scales).
 // Rows in [M, 128-row padding) get zero scales and no codes.
-// The GELU of a bf16 value with 2^-8 <= |v| < 2^6 is read from a table of those
-// 3584 values (the same formula, evaluated once per CTA); other values evaluate
-// it directly. inv_of[s] = 1 / (value(s) * g) per block scale code (0: zero codes).
-constexpr int kGeluTabExpLo = 127 - 8;   // biased bf16 exponents of the table
-constexpr int kGeluTabExps = 14;
+// The GELU of a bf16 value with 2^-16 <= |v| < 2^6 is read from a table of those
+// 5632 values (the same formula, evaluated once per CTA). inv_of[s] =
+// 1 / (value(s) * g) per block scale code (0: zero codes).
+constexpr int kGeluTabExpLo = 127 - 16;  // biased bf16 exponents of the table
+constexpr int kGeluTabExps = 22;
 constexpr int kGeluTabSize = 2 * kGeluTabExps * 128;
 
 __device__ __forceinline__ float gelu_bf16_formula(float v) {
@@ -317,26 +317,22 @@ __device__ __forceinline__ float gelu_tab_input(int i) {
 }
 
 // Branch-free: outside the table, v >= 64 gives v (Phi(v) is 1 in fp32), v <= -64
-// gives -0 (v * Phi(v) is below the bf16 range), and |v| < 2^-8 takes the series
-// Phi(v) = 1/2 + (v - v^3 / 6) / sqrt(2 pi) (truncation below 2^-36 relative there).
-// Selects rather than branches keep the 16 elements of a block in one basic block,
-// so they interleave (measured: a per-lane branch costs 60% more, a table-or-formula
-// branch 2.6x). Nothing here is warp-collective: it runs after per-lane returns.
+// gives -0 (v * Phi(v) is below the bf16 range), and |v| < 2^-16 gives 0.5 v: there
+// v * Phi(v) = 0.5 v (1 + d) with |d| < 2^-16, and 0.5 v is a bf16 value, so no bf16
+// rounding boundary lies between them (up to ties at a subnormal midpoint, which the
+// oracle marks as ambiguous). Selects rather than branches keep the 16 elements of a
+// block in one basic block, so they interleave (measured: a per-lane branch costs
+// 60% more, a table-or-formula branch 2.6x). Nothing here is warp-collective: it
+// runs after per-lane returns.
 __device__ __forceinline__ float gelu_bf16(float v, const uint16_t* tab) {
   const uint32_t bits = __float_as_uint(v) >> 16;  // v is a bf16 value
-  const int e = static_cast<int>((bits >> 7) & 0xFF) - kGeluTabExpLo;
-  const bool in_tab = static_cast<unsigned>(e) < static_cast<unsigned>(kGeluTabExps);
-  const int i = in_tab ? static_cast<int>(bits >> 15) * (kGeluTabExps * 128) + e * 128 +
-                             static_cast<int>(bits & 127)
-                       : 0;
+  const uint32_t mag = (bits & 0x7FFFu) - (static_cast<uint32_t>(kGeluTabExpLo) << 7);
+  const bool in_tab = mag < static_cast<uint32_t>(kGeluTabExps * 128);
+  const uint32_t i = in_tab ? mag + (bits >> 15) * (kGeluTabExps * 128) : 0u;
   const float t = __uint_as_float(static_cast<uint32_t>(tab[i]) << 16);
-  constexpr float kInvSqrt2Pi = 0.39894228040143268f;
-  const float v2 = __fmul_rn(v, v);
-  const float phi = __fadd_rn(0.5f, __fmul_rn(__fmul_rn(v, kInvSqrt2Pi),
-                                              __fsub_rn(1.0f, __fmul_rn(v2, 1.0f / 6.0f))));
-  const float small = __bfloat162float(__float2bfloat16_rn(__fmul_rn(v, phi)));
-  const float big = v > 0.0f ? v : -0.0f;
-  return in_tab ? t : (e < 0 ? small : big);
+  const bool tiny = (bits & 0x7FFFu) < (static_cast<uint32_t>(kGeluTabExpLo) << 7);
+  const float outside = tiny ? __fmul_rn(0.5f, v) : (v > 0.0f ? v : -0.0f);
+  return in_tab ? t : outside;
 }
 
 template <int SLAB>
@@ -362,11 +358,16 @@ __device__ __forceinline__ void gelu_quant_slab(const GemmArgs& a, const uint32_
   for (int b = 0; b < SLAB / 16; ++b) {
     float h[16];
     float amax = 0.0f;
+    float bias[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      *reinterpret_cast<float4*>(&bias[4 * i]) =
+          *reinterpret_cast<const float4*>(cv_bias_slab + 16 * b + 4 * i);
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const int j = 16 * b + i;
       const float v =
-          __bfloat162float(__float2bfloat16_rn(__fmaf_rn(__uint_as_float(r[j]), alpha, cv_bias_slab[j])));
+          __bfloat162float(__float2bfloat16_rn(__fmaf_rn(__uint_as_float(r[j]), alpha, bias[i])));
       h[i] = gelu_bf16(v, gelu_tab);
       amax = fmaxf(amax, fabsf(h[i]));
     }
@@ -400,8 +401,18 @@ constexpr int kModePlain = 0;
 constexpr int kModeSingleLaunch = 1;
 constexpr int kModeGeluQuant = 2;
 
+// Epilogue warps: 4 (one per TMEM lane quadrant); the GELU-quantize epilogue,
+// which does much more work per element and stages nothing, uses 8 (two per
+// quadrant, taking alternate slabs).
+template <int MODE>
+constexpr int epi_warps() { return MODE == kModeGeluQuant ? 8 : 4; }
+template <int MODE>
+constexpr int block_threads() {
+  return MODE == kModeSingleLaunch ? kThreadsFused : 64 + 32 * epi_warps<MODE>();
+}
+
 template <bool FP4, int BN, int CG, int MODE>
-__global__ void __launch_bounds__(MODE == kModeSingleLaunch ? kThreadsFused : kThreads, 1)
+__global__ void __launch_bounds__(block_threads<MODE>(), 1)
 qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
              const __grid_constant__ CUtensorMap tmap_sfa,
              const __grid_constant__ CUtensorMap tmap_sfb,
@@ -409,6 +420,10 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
   using C = Cfg<FP4, BN, CG>;
   constexpr bool FUSED = MODE == kModeSingleLaunch;
   constexpr bool GQ = MODE == kModeGeluQuant;
+  constexpr int EPI_WARPS = epi_warps<MODE>();
+  constexpr int EPI_THREADS = 32 * EPI_WARPS;
+  constexpr int EPI_HALVES = EPI_WARPS / 4;  // warps per TMEM lane quadrant
+  static_assert(!GQ || !C::OVERLAP, "two warps per quadrant need whole accumulator buffers");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -452,7 +467,7 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull_bar[b], 1);
-      mbar_init(&tempty_bar[b], 4 * CG);
+      mbar_init(&tempty_bar[b], EPI_WARPS * CG);
     }
     mbar_init(drain_bar, 1);
     mbar_init(never_bar, 1);
@@ -771,9 +786,10 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
         mbar_wait_bounded(drain_bar, 0, globaltimer_ns() + 100000000ull);
       }
     }
-  } else if (run && warp >= 2 && warp <= 5) {
+  } else if (run && warp >= 2 && warp < 2 + EPI_WARPS) {
     // ------------------------------------------------------------ epilogue
     const int q = warp % 4;  // TMEM lane quadrant this warp may access
+    const int half = (warp - 2) / 4;  // which of the quadrant's warps: slabs it % EPI_HALVES
     const int row_in_tile = static_cast<int>(rank) * kRowsPerCta + q * 32 + lane;
     uint8_t* stage = smem_epi + (warp - 2) * C::EPI_BUFS * kEpiBufBytes;
     int buf = 0;
@@ -790,14 +806,14 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
       static_assert(kGeluTabSize * 2 + 128 * 4 <= C::EPI_BYTES, "tables fit the staging memory");
       const float g = __ldg(args.gq_scale);
       gq_c = __frcp_rn(__fmul_rn(6.0f, g));
-      const int t = threadIdx.x - 64;  // 0 .. 127
-      for (int i = t; i < kGeluTabSize; i += 128)
+      const int t = threadIdx.x - 64;  // 0 .. EPI_THREADS - 1
+      for (int i = t; i < kGeluTabSize; i += EPI_THREADS)
         gelu_tab[i] = static_cast<uint16_t>(__float_as_uint(gelu_bf16_formula(gelu_tab_input(i))) >> 16);
-      {
+      if (t < 128) {
         const float d = __fmul_rn(e4m3_to_float(static_cast<uint32_t>(t)), g);
         inv_of[t] = d != 0.0f ? __frcp_rn(d) : 0.0f;
       }
-      asm volatile("bar.sync 2, 128;" ::: "memory");
+      asm volatile("bar.sync 2, %0;" ::"n"(EPI_THREADS) : "memory");
     }
     int titer = 0;
     for (int tile = group; tile < args.total_tiles; tile += ngroups, ++titer) {
@@ -810,7 +826,7 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
       // of them have finished the previous tile, whose buffer the next load uses)
       float* cv_bias = colvec + (titer & 1) * 512;
       float* cv_scale = cv_bias + 256;
-      for (int j = threadIdx.x - 64; j < BN; j += 128) {
+      for (int j = threadIdx.x - 64; j < BN; j += EPI_THREADS) {
         const int n = n_blk * BN + j;
         const bool in = n < args.N;
         cv_bias[j] = (args.bias && in) ? __ldg(args.bias + n) : 0.0f;
@@ -819,7 +835,7 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
       const bool ready = warp_wait_bounded(&tfull_bar[bi], acc_phase, deadline);
       // publishes the column vectors to all epilogue warps, and makes every
       // epilogue warp leave together if any wait expired
-      if (barrier1_any<128>(!ready)) {
+      if (barrier1_any<EPI_THREADS>(!ready)) {
         record_timeout(args.status);
         break;
       }
@@ -832,6 +848,7 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                              static_cast<uint32_t>(acc * C::ACC_STRIDE);
 #pragma unroll 1
       for (int it = 0; it < C::NSLAB; ++it) {
+        if (EPI_HALVES > 1 && it % EPI_HALVES != half) continue;  // warp-uniform
         // slab order: with shared slabs, buffer 0 drains its last slab (the shared
         // one) first; otherwise slabs go in order
         const int sl = (C::OVERLAP && acc == 0) ? (it + C::NSLAB - 1) % C::NSLAB : it;
@@ -843,8 +860,8 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                              *reinterpret_cast<uint32_t(*)[32]>(&r[32 * h]));
         tmem_ld_wait();
         // hand the buffer back once the MMA can no longer overwrite unread columns:
-        // after the shared slab, or after the last slab
-        if (it == (C::OVERLAP ? 0 : C::NSLAB - 1)) {
+        // after the shared slab, or after this warp's last slab
+        if (C::OVERLAP ? it == 0 : it + EPI_HALVES >= C::NSLAB) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(tempty_bar0 + bi * 8u);
@@ -1068,7 +1085,7 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
   }
 
   cudaLaunchConfig_t cfg{};
-  cfg.blockDim = dim3(FUSED ? kThreadsFused : kThreads);
+  cfg.blockDim = dim3(block_threads<MODE>());
   cfg.dynamicSmemBytes = Cf::SMEM;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
@@ -1129,11 +1146,12 @@ bool set_tile_override(int bn, int cg) {
   return true;
 }
 
-GemmConfig choose_config(bool fp4, int64_t M, int64_t N, int64_t K) {
+GemmConfig choose_config(bool fp4, int64_t M, int64_t N, int64_t K, bool whole_buffers) {
   GemmConfig c{};
   if (g_force_bn.load() != 0) {
     c.bn = g_force_bn.load();
     c.cg = g_force_cg.load();
+    if (whole_buffers && c.bn == 256) c.bn = 224;
     return c;
   }
   // CTA pairs once there are two 128-row blocks to pair. Tile width from a cost
@@ -1148,6 +1166,7 @@ GemmConfig choose_config(bool fp4, int64_t M, int64_t N, int64_t K) {
   double best = 0.0;
   c.bn = 128;
   for (int bn : {128, 192, 224, 256}) {
+    if (whole_buffers && fp4 && bn == 256) continue;  // the shared-slab tile
     const int64_t tiles = tiles_m * ceil_div64(N, bn);
     const int64_t waves = ceil_div64(tiles, groups);
     const int na = (bn + 127) / 128;
@@ -1171,11 +1190,9 @@ cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream) {
     QL_GCASE(128, 1)
     QL_GCASE(192, 1)
     QL_GCASE(224, 1)
-    QL_GCASE(256, 1)
     QL_GCASE(128, 2)
     QL_GCASE(192, 2)
     QL_GCASE(224, 2)
-    QL_GCASE(256, 2)
 #undef QL_GCASE
     return cudaErrorInvalidValue;
   }

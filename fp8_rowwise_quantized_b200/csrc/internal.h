@@ -50,7 +50,9 @@ struct GemmProblem {
   const float* gq_scale;
 };
 
-GemmConfig choose_config(bool fp4, int64_t M, int64_t N, int64_t K);
+// whole_buffers: only tile widths whose two TMEM accumulator buffers do not share
+// a slab (the GELU-quantize epilogue).
+GemmConfig choose_config(bool fp4, int64_t M, int64_t N, int64_t K, bool whole_buffers = false);
 bool set_tile_override(int bn, int cg);  // bn == 0 restores the automatic choice
 cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream);
 
