@@ -565,13 +565,16 @@ def run_ours(args):
 def run_profile(args):
     """Short fixed sequence for profilers: `--profile <piece>` runs `--steps` calls
     of one piece of the headline workload (no flushes, no timing): `step`,
-    `prologue`, `gemm`, `quant` (activation quantization alone), `fp8r_step`,
-    `fp8r_quant` or `fp8r_gemm`."""
+    `prologue`, `gemm`, `quant` (activation quantization alone), `mlp_fused` (the MLP
+    block with the GELU-quantize epilogue), `fp8r_step`, `fp8r_quant` or `fp8r_gemm`."""
     import torch
     torch.cuda.set_device(0)
     device = torch.device("cuda", 0)
     M, K, N = WORKLOAD["M"], WORKLOAD["K"], WORKLOAD["N"]
-    if args.profile.startswith("fp8r"):
+    if args.profile == "mlp_fused":
+        mlp = MlpBlock(4096, 3072, 12288, device)
+        fn = mlp.fused
+    elif args.profile.startswith("fp8r"):
         L = Fp8rLayer(4096, 3072, 3072, False, device)
         fn = {"fp8r_step": L.step, "fp8r_gemm": L.gemm,
               "fp8r_quant": lambda: L.q.fp8r_quantize_rows(L.x, L.xq, L.xs)}[args.profile]
@@ -600,7 +603,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-variants", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["step", "prologue", "gemm", "quant", "fp8r_step",
+    ap.add_argument("--profile", choices=["step", "prologue", "gemm", "quant", "mlp_fused", "fp8r_step",
                                           "fp8r_quant", "fp8r_gemm"], default=None,
                     help="run a short fixed sequence for a profiler instead of the benchmark")
     args = ap.parse_args()
