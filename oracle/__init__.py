@@ -45,6 +45,12 @@ def lib():
         L.oracle_gelu.argtypes = [C.c_double]
         L.oracle_gelu.restype = C.c_double
         L.oracle_gelu_bf16.argtypes = [u16p, i64, C.c_double, C.c_double, u16p, u8p]
+        L.oracle_smooth_bf16.argtypes = [u16p, i64, i64, f32p, u16p]
+        L.oracle_lowrank_down.argtypes = [u16p, i64, i64, u16p, i64, f64p]
+        L.oracle_svdq_nvfp4_linear.argtypes = [u8p, u8p, i64, i64, u8p, u8p, i64, C.c_float,
+                                               C.c_float, f64p, u16p, i64, f32p, u16p, f64p,
+                                               f64p, f64p]
+        L.oracle_svdq_nvfp4_linear.restype = C.c_int
         L.oracle_nvfp4_global_scale.argtypes = [u16p, i64]
         L.oracle_nvfp4_global_scale.restype = C.c_float
         L.oracle_nvfp4_quantize.argtypes = [u16p, i64, i64, C.c_float, u8p, u8p]
@@ -150,6 +156,49 @@ def gelu_bf16(y, rel_tol: float = 2.0 ** -20, rel_tol_sq: float = 2.0 ** -22):
     lib().oracle_gelu_bf16(_p(bits, C.c_uint16), bits.size, float(rel_tol), float(rel_tol_sq),
                            _p(h, C.c_uint16), _p(amb, C.c_uint8))
     return h, amb.astype(bool)
+
+
+def smooth_bf16(x, smooth) -> np.ndarray:
+    """bf16(RN32(x * smooth)) per element, smooth fp32 [K] over the last axis (uint16 bits)."""
+    bits = _bits16(x)
+    M, K = bits.shape
+    sm = np.ascontiguousarray(smooth, dtype=np.float32)
+    assert sm.shape == (K,)
+    out = np.empty_like(bits)
+    lib().oracle_smooth_bf16(_p(bits, C.c_uint16), M, K, _p(sm, C.c_float), _p(out, C.c_uint16))
+    return out
+
+
+def lowrank_down(xs, down) -> np.ndarray:
+    """D = xs @ down^T exactly (fp64); xs bf16 [M, K], down bf16 [r, K]."""
+    a, b = _bits16(xs), _bits16(down)
+    M, K = a.shape
+    r = b.shape[0]
+    assert b.shape == (r, K)
+    D = np.empty((M, r), dtype=np.float64)
+    lib().oracle_lowrank_down(_p(a, C.c_uint16), M, K, _p(b, C.c_uint16), r, _p(D, C.c_double))
+    return D
+
+
+def svdq_nvfp4_linear(xq, xs, wq, ws, input_scale, weight_scale_2, D, up, bias=None):
+    """SVDQuant-style NVFP4 linear: (y bf16 bits, y64, T, T_lr), see oracle.cpp."""
+    M, K = xq.shape[0], xq.shape[1] * 2
+    N = wq.shape[0]
+    D = np.ascontiguousarray(D, dtype=np.float64)
+    upb = _bits16(up)
+    r = D.shape[1]
+    assert upb.shape == (N, r)
+    y = np.empty((M, N), dtype=np.uint16)
+    y64, T, Tlr = (np.empty((M, N)) for _ in range(3))
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    rc = lib().oracle_svdq_nvfp4_linear(
+        _p(np.ascontiguousarray(xq), C.c_uint8), _p(np.ascontiguousarray(xs), C.c_uint8), M, K,
+        _p(np.ascontiguousarray(wq), C.c_uint8), _p(np.ascontiguousarray(ws), C.c_uint8), N,
+        float(input_scale), float(weight_scale_2), _p(D, C.c_double), _p(upb, C.c_uint16), r,
+        _p(b, C.c_float), _p(y, C.c_uint16), _p(y64, C.c_double), _p(T, C.c_double),
+        _p(Tlr, C.c_double))
+    assert rc == 0
+    return y, y64, T, Tlr
 
 
 def nvfp4_global_scale(x) -> float:

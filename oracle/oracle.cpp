@@ -255,6 +255,77 @@ void oracle_gelu_bf16(const uint16_t* y, int64_t n, double tol_const, double tol
 }
 
 // ---------------------------------------------------------------------------
+// SVDQuant-style NVFP4 linear with a 16-bit low-rank branch ("Bringing Nunchaku
+// 4-bit Diffusion Inference to Diffusers", sections "Background: SVDQuant and
+// Nunchaku" and "Introducing Nunchaku Lite", svdq_w4a4): activation outliers are
+// moved into the weights by a per-channel smoothing, the hardest part of the
+// weight is a rank-r 16-bit branch, and the residual is quantized to 4 bits.
+// The pages give no formulas; the plainest reading is taken:
+//   xs[m,k] = bf16( RN32(x[m,k] * smooth[k]) )          smoothed activations
+//   D[m,j]  = sum_k xs[m,k] * down[j,k]                  low-rank down, j < r
+//   Y[m,n]  = bf16( input_scale * weight_scale_2 * sum_k NVFP4(xs) NVFP4(R)
+//                   + sum_j D[m,j] * up[n,j] + bias[n] )
+// down [r, K] and up [N, r] are bf16 (nn.Linear weight layouts, 16-bit as the
+// pages say); NVFP4(xs) uses input_scale; R is the 4-bit residual weight. The
+// contractions are exact (fp64). T_lr[m,n] = sum_j |D[m,j] * up[n,j]| bounds the
+// low-rank term, for the tolerance of a 16-bit evaluation of that branch.
+// ---------------------------------------------------------------------------
+void oracle_smooth_bf16(const uint16_t* x, int64_t M, int64_t K, const float* smooth,
+                        uint16_t* out) {
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t k = 0; k < K; ++k) {
+      const float p = bf16_to_float(x[m * K + k]) * smooth[k];  // one fp32 RN multiply
+      out[m * K + k] = oracle_bf16_from_double(static_cast<double>(p));
+    }
+}
+
+void oracle_lowrank_down(const uint16_t* xs, int64_t M, int64_t K, const uint16_t* down,
+                         int64_t r, double* D) {
+#pragma omp parallel for schedule(static)
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t j = 0; j < r; ++j) {
+      double acc = 0.0;
+      for (int64_t k = 0; k < K; ++k)
+        acc += static_cast<double>(bf16_to_float(xs[m * K + k])) *
+               static_cast<double>(bf16_to_float(down[j * K + k]));
+      D[m * r + j] = acc;
+    }
+}
+
+int oracle_nvfp4_linear(const uint8_t* xq, const uint8_t* xs, int64_t M, int64_t K,
+                        const uint8_t* wq, const uint8_t* ws, int64_t N,
+                        float input_scale, float weight_scale_2, const float* bias,
+                        uint16_t* y, double* y64, double* T);  // below
+
+int oracle_svdq_nvfp4_linear(const uint8_t* xq, const uint8_t* xsc, int64_t M, int64_t K,
+                             const uint8_t* wq, const uint8_t* ws, int64_t N, float input_scale,
+                             float weight_scale_2, const double* D, const uint16_t* up, int64_t r,
+                             const float* bias, uint16_t* y, double* y64, double* T,
+                             double* T_lr) {
+  if (M < 0 || N < 0 || K <= 0 || K % 16 != 0 || r < 0) return -1;
+  std::vector<double> main64((size_t)M * N), mainT((size_t)M * N);
+  int rc = oracle_nvfp4_linear(xq, xsc, M, K, wq, ws, N, input_scale, weight_scale_2, nullptr,
+                               nullptr, main64.data(), mainT.data());
+  if (rc != 0) return rc;
+#pragma omp parallel for schedule(static)
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t n = 0; n < N; ++n) {
+      double lr = 0.0, lr_abs = 0.0;
+      for (int64_t j = 0; j < r; ++j) {
+        const double t = D[m * r + j] * static_cast<double>(bf16_to_float(up[n * r + j]));
+        lr += t;
+        lr_abs += std::fabs(t);
+      }
+      const double v = main64[m * N + n] + lr + (bias ? static_cast<double>(bias[n]) : 0.0);
+      if (y) y[m * N + n] = oracle_bf16_from_double(v);
+      if (y64) y64[m * N + n] = v;
+      if (T) T[m * N + n] = mainT[m * N + n];
+      if (T_lr) T_lr[m * N + n] = lr_abs;
+    }
+  return 0;
+}
+
+// ---------------------------------------------------------------------------
 // Calibration rule of the workloads: global scale = amax / (6 * 448), i.e. the
 // largest magnitude maps onto the largest E2M1 value times the largest E4M3
 // scale. fp32 division, one rounding. The pages only say "calibrated".
