@@ -21,6 +21,7 @@ from . import _lib
 __all__ = [
     "nvfp4_quantize_act", "nvfp4_linear", "nvfp4_linear_single_launch", "nvfp4_linear_noalloc",
     "nvfp4_linear_prologue", "nvfp4_linear_gelu_quantize", "nvfp4_linear_quantized_input",
+    "nvfp4_linear_gemm_lowrank",
     "nvfp4_linear_gemm",
     "nvfp4_linear_workspace_size", "nvfp4_linear_workspace_layout", "nvfp4_global_scale",
     "fp8r_quantize_rows", "fp8r_linear", "fp8r_linear_gemm", "fp8r_linear_workspace_size",
@@ -201,6 +202,33 @@ def nvfp4_linear_quantized_input(M: int, w: torch.Tensor, w_scale: torch.Tensor,
     _lib.check("nvfp4_linear_quantized_input", _lib.load().nvfp4_linear_quantized_input(
         M, K, _ptr(w), _ptr(w_scale), N, _ptr(weight_scale_2), _ptr(input_scale), _ptr(bias),
         _ptr(y), _ptr(workspace), workspace.numel(), _stream()))
+    return y
+
+
+def nvfp4_linear_gemm_lowrank(M: int, w: torch.Tensor, weight_scale_2: torch.Tensor,
+                              input_scale: torch.Tensor, workspace: torch.Tensor,
+                              lr_act: torch.Tensor, lr_up: torch.Tensor,
+                              bias: Optional[torch.Tensor] = None,
+                              y: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """nvfp4_linear_gemm plus the low-rank branch alpha * lr_act @ lr_up^T: lr_act bf16
+    [M, r] (the branch's activations divided by alpha), lr_up bf16 [N, r]."""
+    _need(w, "w", torch.uint8, 2)
+    _need(workspace, "workspace", torch.uint8, 1)
+    _need(lr_act, "lr_act", torch.bfloat16, 2)
+    _need(lr_up, "lr_up", torch.bfloat16, 2)
+    _scalar(weight_scale_2, "weight_scale_2")
+    _scalar(input_scale, "input_scale")
+    N, K = w.shape[0], w.shape[1] * 2
+    r = lr_act.shape[1]
+    if lr_act.shape[0] != M or tuple(lr_up.shape) != (N, r):
+        raise ValueError("low-rank operand shapes do not match")
+    if bias is not None:
+        _need(bias, "bias", torch.float32, 1)
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=w.device)
+    _lib.check("nvfp4_linear_gemm_lowrank", _lib.load().nvfp4_linear_gemm_lowrank(
+        M, K, _ptr(w), N, _ptr(weight_scale_2), _ptr(input_scale), _ptr(bias), _ptr(lr_act),
+        _ptr(lr_up), r, _ptr(y), _ptr(workspace), workspace.numel(), _stream()))
     return y
 
 

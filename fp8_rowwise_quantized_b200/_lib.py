@@ -34,6 +34,8 @@ SIGNATURES = {
                                              _f32p, _f32p, _vp, _sz, _vp, _sz, _vp]),
     "nvfp4_linear_quantized_input": (C.c_int, [_i64, _i64, _u8p, _u8p, _i64, _f32p, _f32p,
                                                _f32p, _vp, _vp, _sz, _vp]),
+    "nvfp4_linear_gemm_lowrank": (C.c_int, [_i64, _i64, _u8p, _i64, _f32p, _f32p, _f32p, _vp,
+                                            _vp, _i64, _vp, _vp, _sz, _vp]),
     "nvfp4_linear_prologue": (C.c_int, [_vp, _i64, _i64, _u8p, _i64, _f32p, _vp, _sz, _vp]),
     "nvfp4_linear_gemm": (C.c_int, [_i64, _i64, _u8p, _i64, _f32p, _f32p, _f32p, _vp, _vp, _sz,
                                     _vp]),

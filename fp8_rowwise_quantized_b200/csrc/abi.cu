@@ -211,7 +211,9 @@ int nvfp4_linear_prologue(const void* x, int64_t M, int64_t K, const uint8_t* w_
 static int nvfp4_gemm_impl(int64_t M, int64_t K, const uint8_t* w, int64_t N,
                            const float* weight_scale_2, const float* input_scale,
                            const float* bias, void* y, const void* workspace,
-                           size_t workspace_bytes, ql_stream_t stream, bool pdl) {
+                           size_t workspace_bytes, ql_stream_t stream, bool pdl,
+                           const void* lr_act = nullptr, const void* lr_up = nullptr,
+                           int lr_rank = 0) {
   if (!w || !weight_scale_2 || !input_scale || !y || M <= 0 || N <= 0 || K <= 0)
     return QL_ERR_INVALID_ARG;
   if (!nvfp4_shape_ok(M, K, N)) return fail_shape("nvfp4: needs K >= 32 and K % 32 == 0");
@@ -244,6 +246,9 @@ static int nvfp4_gemm_impl(int64_t M, int64_t K, const uint8_t* w, int64_t N,
   p.timeout_ns = timeout_ns();
   p.inject_fault = g_inject_fault.load();
   p.pdl = pdl;
+  p.lr_act = lr_act;
+  p.lr_up = lr_up;
+  p.lr_rank = lr_rank;
   cudaError_t e = ql::launch_gemm(p, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? QL_OK : record(e, "nvfp4 gemm launch");
 }
@@ -253,6 +258,19 @@ int nvfp4_linear_gemm(int64_t M, int64_t K, const uint8_t* w, int64_t N,
                       void* y, const void* workspace, size_t workspace_bytes, ql_stream_t stream) {
   return nvfp4_gemm_impl(M, K, w, N, weight_scale_2, input_scale, bias, y, workspace,
                          workspace_bytes, stream, false);
+}
+
+int nvfp4_linear_gemm_lowrank(int64_t M, int64_t K, const uint8_t* w, int64_t N,
+                              const float* weight_scale_2, const float* input_scale,
+                              const float* bias, const void* lr_act, const void* lr_up,
+                              int64_t rank, void* y, const void* workspace,
+                              size_t workspace_bytes, ql_stream_t stream) {
+  if (!lr_act || !lr_up) return QL_ERR_INVALID_ARG;
+  if (rank < 8 || rank > 64 || rank % 8 != 0)
+    return fail_shape("low-rank branch: needs rank in 8..64, rank % 8 == 0");
+  if (!aligned16(lr_act) || !aligned16(lr_up)) return QL_ERR_ALIGN;
+  return nvfp4_gemm_impl(M, K, w, N, weight_scale_2, input_scale, bias, y, workspace,
+                         workspace_bytes, stream, false, lr_act, lr_up, static_cast<int>(rank));
 }
 
 int nvfp4_linear(const void* x, int64_t M, int64_t K, const uint8_t* w, const uint8_t* w_scale,

@@ -79,6 +79,10 @@ struct GemmArgs {
   const float* gq_scale;
   int sync_words;
   uint32_t tag;             // this launch's tag, odd
+  // low-rank branch (FP4, plain mode): after a tile's K tiles, one more stage of
+  // bf16 operands (tmap_lra: [M, r] activations pre-divided by alpha; tmap_lrb:
+  // [N, r]) and lr_k16 = ceil(r / 16) MMAs of K = 16 into the same accumulator
+  int lr_k16;
 };
 
 template <bool FP4, int BN, int CG>
@@ -112,6 +116,9 @@ struct Cfg {
   static constexpr uint32_t IDESC =
       FP4 ? ((1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(TILE_M >> 4) << 24))
           : ((1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(TILE_M >> 4) << 24));
+  // the low-rank branch's bf16 x bf16 MMAs (K = 16 each) into the same accumulator
+  static constexpr uint32_t IDESC_BF16 = (1u << 4) | (1u << 7) | (1u << 10) |
+                                         (uint32_t(BN >> 3) << 17) | (uint32_t(TILE_M >> 4) << 24);
   static_assert(STAGES >= 2, "shared memory too small for two stages");
   static_assert(SFA_COL + SF_COLS <= kTmemCols, "TMEM budget");
   static_assert(!OVERLAP || BN == 256, "only the 256-column tile shares a slab");
@@ -416,7 +423,9 @@ __global__ void __launch_bounds__(block_threads<MODE>(), 1)
 qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
              const __grid_constant__ CUtensorMap tmap_sfa,
              const __grid_constant__ CUtensorMap tmap_sfb,
-             const __grid_constant__ CUtensorMap tmap_y, const GemmArgs args) {
+             const __grid_constant__ CUtensorMap tmap_y,
+             const __grid_constant__ CUtensorMap tmap_lra,
+             const __grid_constant__ CUtensorMap tmap_lrb, const GemmArgs args) {
   using C = Cfg<FP4, BN, CG>;
   constexpr bool FUSED = MODE == kModeSingleLaunch;
   constexpr bool GQ = MODE == kModeGeluQuant;
@@ -461,6 +470,10 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
       prefetch_tmap(&tmap_sfb);
     }
     if (args.use_tma_store) prefetch_tmap(&tmap_y);
+    if (args.lr_k16 > 0) {
+      prefetch_tmap(&tmap_lra);
+      prefetch_tmap(&tmap_lrb);
+    }
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
@@ -659,6 +672,34 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
           phase ^= 1u;
         }
       }
+      if (ok && args.lr_k16 > 0) {
+        // the low-rank branch's operands, one stage in the A and B areas (same
+        // 128-byte rows and swizzle as a K tile; columns r .. 63 read as zeros)
+        if (!warp_wait_bounded(&empty_bar[stage], phase ^ 1u, deadline)) {
+          ok = false;
+          break;
+        }
+        if (elect_one()) {
+          const uint32_t fb = full_bar0 + stage * 8u;
+          uint8_t* sa = smem_a + stage * C::A_BYTES;
+          uint8_t* sb = smem_b + stage * C::B_BYTES;
+          if constexpr (CG == 2) {
+            if (leader) mbar_arrive_expect_tx(&full_bar[stage], CG * (C::A_BYTES + C::B_BYTES));
+            tma_load_2d_pair(sa, &tmap_lra, fb, 0, a_row);
+            tma_load_2d_pair(sb, &tmap_lrb, fb, 0, b_row);
+          } else {
+            mbar_arrive_expect_tx(&full_bar[stage], C::A_BYTES + C::B_BYTES);
+            tma_load_2d(sa, &tmap_lra, &full_bar[stage], 0, a_row);
+            tma_load_2d(sb, &tmap_lrb, &full_bar[stage], 0, b_row);
+          }
+        }
+        __syncwarp();
+        ++issued;
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
     }
     if (!ok) {
       record_timeout(args.status);
@@ -760,6 +801,36 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
         if (++stage == C::STAGES) {
           stage = 0;
           phase ^= 1u;
+        }
+      }
+      if (ok && FP4 && args.lr_k16 > 0) {
+        // low-rank up projection: (D / alpha) x up^T, bf16, K = 16 per MMA, into the
+        // same accumulator (always accumulating: the K tiles came first)
+        if (!warp_wait_bounded(&full_bar[stage], phase, deadline)) {
+          ok = false;
+        } else {
+          tc_fence_after();
+          if (elect_one()) {
+            const uint32_t a_addr = smem_u32(smem_a + stage * C::A_BYTES);
+            const uint32_t b_addr = smem_u32(smem_b + stage * C::B_BYTES);
+            for (int kb = 0; kb < args.lr_k16; ++kb) {
+              const uint64_t ad = smem_desc(a_addr + kb * 32, 16, 1024, 2);
+              const uint64_t bd = smem_desc(b_addr + kb * 32, 16, 1024, 2);
+              if constexpr (CG == 2)
+                mma_bf16_pair(d_tmem, ad, bd, C::IDESC_BF16, 1u);
+              else
+                mma_bf16(d_tmem, ad, bd, C::IDESC_BF16, 1u);
+            }
+            if constexpr (CG == 2)
+              tc_commit_pair(&empty_bar[stage], 0x3);
+            else
+              tc_commit(&empty_bar[stage]);
+          }
+          __syncwarp();
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
       }
       if (!ok) break;
@@ -1017,7 +1088,9 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
 
   const int64_t k_bytes = FP4 ? p.K / 2 : p.K;
-  CUtensorMap ta, tb, tsa, tsb, ty;
+  CUtensorMap ta, tb, tsa, tsb, ty, tla, tlb;
+  std::memset(&tla, 0, sizeof(tla));
+  std::memset(&tlb, 0, sizeof(tlb));
   std::memset(&tsa, 0, sizeof(tsa));
   std::memset(&tsb, 0, sizeof(tsb));
   std::memset(&ty, 0, sizeof(ty));
@@ -1049,7 +1122,21 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
                  CU_TENSOR_MAP_L2_PROMOTION_NONE))
     return cudaErrorInvalidValue;
 
+  const bool lowrank = FP4 && MODE == kModePlain && p.lr_rank > 0;
+  if (lowrank) {
+    // bf16 [rows, r] with 128-byte boxes of 64 elements: columns r .. 63 read as zeros
+    if (p.lr_rank > 64 || p.lr_rank % 8 != 0 || !p.lr_act || !p.lr_up ||
+        !encode_2d(&tla, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.lr_act, p.lr_rank, p.M,
+                   p.lr_rank * 2, 64, kRowsPerCta, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
+        !encode_2d(&tlb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.lr_up, p.lr_rank, p.N,
+                   p.lr_rank * 2, 64, Cf::B_ROWS, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
+      return cudaErrorInvalidValue;
+  }
+
   GemmArgs a{};
+  a.lr_k16 = lowrank ? (p.lr_rank + 15) / 16 : 0;
   a.M = static_cast<int>(p.M);
   a.N = static_cast<int>(p.N);
   a.K = static_cast<int>(p.K);
@@ -1124,7 +1211,7 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
   }
   cfg.attrs = attr;
   cfg.numAttrs = nattr;
-  return cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, ty, a);
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, ty, tla, tlb, a);
 }
 
 }  // namespace

@@ -48,6 +48,12 @@ struct GemmProblem {
   uint8_t* gq_codes;
   uint8_t* gq_atoms;
   const float* gq_scale;
+  // low-rank branch (FP4, plain mode, 8 <= lr_rank <= 64, lr_rank % 8 == 0):
+  // Y += alpha * lr_act x lr_up^T with lr_act bf16 [M, r] (the low-rank activations
+  // divided by alpha) and lr_up bf16 [N, r]
+  const void* lr_act;
+  const void* lr_up;
+  int lr_rank;
 };
 
 // whole_buffers: only tile widths whose two TMEM accumulator buffers do not share

@@ -80,6 +80,21 @@ enum {
 int nvfp4_quantize_act(const void* x, int64_t M, int64_t K, const float* input_scale,
                        uint8_t* xq, uint8_t* xs, ql_stream_t stream);
 
+/* nvfp4_linear_gemm plus a 16-bit low-rank branch (SVDQuant, "Background: SVDQuant
+ * and Nunchaku": the low-rank up projection fused with the 4-bit compute kernel):
+ *   Y = bf16( alpha * (sum_k NVFP4(x) NVFP4(w) + sum_j lr_act[m,j] * lr_up[n,j]) + bias )
+ * with alpha = input_scale * weight_scale_2, i.e. lr_act is the low-rank branch's
+ * activations D divided by alpha (so that alpha * lr_act = D), bf16 [M, rank]
+ * row-major; lr_up bf16 [N, rank] row-major. The branch runs on the tensor cores
+ * as one more K step (bf16 x bf16, fp32 accumulation) into the FP4 accumulator.
+ * Requires 8 <= rank <= 64, rank % 8 == 0, 16-byte aligned lr_act / lr_up; the
+ * workspace is the one nvfp4_linear_prologue filled. */
+int nvfp4_linear_gemm_lowrank(int64_t M, int64_t K, const uint8_t* w, int64_t N,
+                              const float* weight_scale_2, const float* input_scale,
+                              const float* bias, const void* lr_act, const void* lr_up,
+                              int64_t rank, void* y, const void* workspace,
+                              size_t workspace_bytes, ql_stream_t stream);
+
 /* The MLP up projection with its GELU and the down projection's quantization
  * fused into the GEMM epilogue (the "fused GELU/MLP" kernels of the Diffusers
  * page "Nunchaku" section, for the nvfp4 scheme): instead of Y it writes
