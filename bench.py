@@ -221,6 +221,31 @@ class Fp8rLayer:
         self.q.fp8r_linear_gemm(self.xq, self.xs, self.wq, self.wsc, bias=self.bias, y=self.y)
 
 
+class SvdqLayer:
+    """svdq_w4a4 NVFP4 layer (smoothing, rank-r bf16 branch, 4-bit residual) with
+    synthetic operands of the Nvfp4Layer's shapes."""
+
+    def __init__(self, M, K, N, rank, device, seed=0):
+        import torch
+        import fp8_rowwise_quantized_b200 as q
+        base = Nvfp4Layer(M, K, N, False, device, seed=seed)
+        g = torch.Generator().manual_seed(seed + 7)
+        self.q, self.base = q, base
+        self.down = (torch.randn(rank, K, generator=g) * 0.02).to(torch.bfloat16).to(device)
+        self.up = (torch.randn(N, rank, generator=g) * 0.05).to(torch.bfloat16).to(device)
+        amax = base.x.float().abs().amax(dim=0).clamp(min=1e-3)
+        self.smooth = (1.0 / amax.sqrt()).float().contiguous()
+        xs = (base.x.float() * self.smooth).to(torch.bfloat16)
+        self.gx = q.nvfp4_global_scale(xs)
+        self.work = torch.empty(q.svdq_nvfp4_linear_workspace_size(M, K, N, rank),
+                                dtype=torch.uint8, device=device)
+
+    def step(self):
+        b = self.base
+        self.q.svdq_nvfp4_linear(b.x, b.wq, b.ws, b.gw, self.gx, self.down, self.up,
+                                 smooth=self.smooth, y=b.y, workspace=self.work)
+
+
 class MlpBlock:
     """Diffusion-transformer MLP block on the device: up projection (K -> H), exact
     GELU, down projection (H -> K), both NVFP4. The down projection's input_scale
@@ -506,6 +531,14 @@ def run_ours(args):
                               "gemm_frac_of_peak": fl / (gms / 1e3) / 1e12 / pk}
             del L
         torch.cuda.empty_cache()
+        # svdq_w4a4 NVFP4 layer (rank 32) on the headline shape
+        sv = SvdqLayer(M, K, N, 32, device)
+        s_ms, _ = time_events(sv.step, v_steps, 3, flush, stream)
+        variants["svdq_nvfp4_r32_4096x3072x12288"] = {
+            "us": s_ms * 1e3, "tflops": flops / (s_ms / 1e3) / 1e12,
+            "lowrank_extra_flops_pct": 100.0 * 2 * 32 * (K + N) / (2 * K * N)}
+        del sv
+        torch.cuda.empty_cache()
         # MLP block (up 3072 -> 12288, GELU, down 12288 -> 3072): fused GELU + NVFP4
         # requantization epilogue vs up linear, torch GELU, down linear
         mlp = MlpBlock(4096, 3072, 12288, device)
@@ -566,7 +599,8 @@ def run_profile(args):
     """Short fixed sequence for profilers: `--profile <piece>` runs `--steps` calls
     of one piece of the headline workload (no flushes, no timing): `step`,
     `prologue`, `gemm`, `quant` (activation quantization alone), `mlp_fused` (the MLP
-    block with the GELU-quantize epilogue), `fp8r_step`, `fp8r_quant` or `fp8r_gemm`."""
+    block with the GELU-quantize epilogue), `svdq` (the rank-32 svdq layer), `fp8r_step`,
+    `fp8r_quant` or `fp8r_gemm`."""
     import torch
     torch.cuda.set_device(0)
     device = torch.device("cuda", 0)
@@ -574,6 +608,9 @@ def run_profile(args):
     if args.profile == "mlp_fused":
         mlp = MlpBlock(4096, 3072, 12288, device)
         fn = mlp.fused
+    elif args.profile == "svdq":
+        sv = SvdqLayer(4096, 3072, 12288, 32, device)
+        fn = sv.step
     elif args.profile.startswith("fp8r"):
         L = Fp8rLayer(4096, 3072, 3072, False, device)
         fn = {"fp8r_step": L.step, "fp8r_gemm": L.gemm,
@@ -603,7 +640,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-variants", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["step", "prologue", "gemm", "quant", "mlp_fused", "fp8r_step",
+    ap.add_argument("--profile", choices=["step", "prologue", "gemm", "quant", "mlp_fused", "svdq",
+                                          "fp8r_step",
                                           "fp8r_quant", "fp8r_gemm"], default=None,
                     help="run a short fixed sequence for a profiler instead of the benchmark")
     args = ap.parse_args()

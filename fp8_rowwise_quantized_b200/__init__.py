@@ -21,7 +21,7 @@ from . import _lib
 __all__ = [
     "nvfp4_quantize_act", "nvfp4_linear", "nvfp4_linear_single_launch", "nvfp4_linear_noalloc",
     "nvfp4_linear_prologue", "nvfp4_linear_gelu_quantize", "nvfp4_linear_quantized_input",
-    "nvfp4_linear_gemm_lowrank",
+    "nvfp4_linear_gemm_lowrank", "svdq_nvfp4_linear", "svdq_nvfp4_linear_workspace_size",
     "nvfp4_linear_gemm",
     "nvfp4_linear_workspace_size", "nvfp4_linear_workspace_layout", "nvfp4_global_scale",
     "fp8r_quantize_rows", "fp8r_linear", "fp8r_linear_gemm", "fp8r_linear_workspace_size",
@@ -229,6 +229,47 @@ def nvfp4_linear_gemm_lowrank(M: int, w: torch.Tensor, weight_scale_2: torch.Ten
     _lib.check("nvfp4_linear_gemm_lowrank", _lib.load().nvfp4_linear_gemm_lowrank(
         M, K, _ptr(w), N, _ptr(weight_scale_2), _ptr(input_scale), _ptr(bias), _ptr(lr_act),
         _ptr(lr_up), r, _ptr(y), _ptr(workspace), workspace.numel(), _stream()))
+    return y
+
+
+def svdq_nvfp4_linear_workspace_size(M: int, K: int, N: int, rank: int) -> int:
+    return int(_lib.load().svdq_nvfp4_linear_workspace_size(M, K, N, rank))
+
+
+def svdq_nvfp4_linear(x: torch.Tensor, w: torch.Tensor, w_scale: torch.Tensor,
+                      weight_scale_2: torch.Tensor, input_scale: torch.Tensor,
+                      lora_down: torch.Tensor, lora_up: torch.Tensor,
+                      smooth: Optional[torch.Tensor] = None, bias: Optional[torch.Tensor] = None,
+                      y: Optional[torch.Tensor] = None,
+                      workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """SVDQuant-style NVFP4 linear: Y = bf16(alpha * NVFP4(xs) NVFP4(w)^T
+    + (xs lora_down^T) lora_up^T + bias), xs = bf16(x * smooth). lora_down bf16 [r, K],
+    lora_up bf16 [N, r], smooth fp32 [K] or None; input_scale calibrated on xs."""
+    _need(x, "x", torch.bfloat16, 2)
+    _need(w, "w", torch.uint8, 2)
+    _need(w_scale, "w_scale", torch.uint8, 2)
+    _need(lora_down, "lora_down", torch.bfloat16, 2)
+    _need(lora_up, "lora_up", torch.bfloat16, 2)
+    _scalar(weight_scale_2, "weight_scale_2")
+    _scalar(input_scale, "input_scale")
+    M, K = x.shape
+    N = w.shape[0]
+    r = lora_down.shape[0]
+    if w.shape[1] * 2 != K or tuple(w_scale.shape) != (N, K // 16):
+        raise ValueError("weight shapes do not match x")
+    if tuple(lora_down.shape) != (r, K) or tuple(lora_up.shape) != (N, r):
+        raise ValueError("low-rank shapes do not match")
+    if smooth is not None:
+        _need(smooth, "smooth", torch.float32, 1)
+    if bias is not None:
+        _need(bias, "bias", torch.float32, 1)
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    ws = _workspace(svdq_nvfp4_linear_workspace_size(M, K, N, r), x.device, workspace)
+    _lib.check("svdq_nvfp4_linear", _lib.load().svdq_nvfp4_linear(
+        _ptr(x), M, K, _ptr(smooth), _ptr(lora_down), _ptr(lora_up), r, _ptr(w), _ptr(w_scale),
+        N, _ptr(weight_scale_2), _ptr(input_scale), _ptr(bias), _ptr(y), _ptr(ws), ws.numel(),
+        _stream()))
     return y
 
 

@@ -36,6 +36,9 @@ SIGNATURES = {
                                                _f32p, _vp, _vp, _sz, _vp]),
     "nvfp4_linear_gemm_lowrank": (C.c_int, [_i64, _i64, _u8p, _i64, _f32p, _f32p, _f32p, _vp,
                                             _vp, _i64, _vp, _vp, _sz, _vp]),
+    "svdq_nvfp4_linear_workspace_size": (C.c_size_t, [_i64, _i64, _i64, _i64]),
+    "svdq_nvfp4_linear": (C.c_int, [_vp, _i64, _i64, _f32p, _vp, _vp, _i64, _u8p, _u8p, _i64,
+                                    _f32p, _f32p, _f32p, _vp, _vp, _sz, _vp]),
     "nvfp4_linear_prologue": (C.c_int, [_vp, _i64, _i64, _u8p, _i64, _f32p, _vp, _sz, _vp]),
     "nvfp4_linear_gemm": (C.c_int, [_i64, _i64, _u8p, _i64, _f32p, _f32p, _f32p, _vp, _vp, _sz,
                                     _vp]),

@@ -273,6 +273,48 @@ int nvfp4_linear_gemm_lowrank(int64_t M, int64_t K, const uint8_t* w, int64_t N,
                          workspace_bytes, stream, false, lr_act, lr_up, static_cast<int>(rank));
 }
 
+size_t svdq_nvfp4_linear_workspace_size(int64_t M, int64_t K, int64_t N, int64_t rank) {
+  const size_t base = nvfp4_linear_workspace_size(M, K, N);
+  if (base == 0 || rank < 8 || rank > 64 || rank % 8 != 0) return 0;
+  return base + ql::align_up(static_cast<size_t>(M) * static_cast<size_t>(rank) * 2, 1024);
+}
+
+int svdq_nvfp4_linear(const void* x, int64_t M, int64_t K, const float* smooth,
+                      const void* lora_down, const void* lora_up, int64_t rank, const uint8_t* w,
+                      const uint8_t* w_scale, int64_t N, const float* weight_scale_2,
+                      const float* input_scale, const float* bias, void* y, void* workspace,
+                      size_t workspace_bytes, ql_stream_t stream) {
+  if (!x || !lora_down || !lora_up || !w || !w_scale || !weight_scale_2 || !input_scale || !y ||
+      M <= 0 || N <= 0 || K <= 0)
+    return QL_ERR_INVALID_ARG;
+  if (!nvfp4_shape_ok(M, K, N)) return fail_shape("nvfp4: needs K >= 32 and K % 32 == 0");
+  if (rank < 8 || rank > 64 || rank % 8 != 0)
+    return fail_shape("low-rank branch: needs rank in 8..64, rank % 8 == 0");
+  if (!aligned16(x) || (smooth && !aligned16(smooth)) || !aligned16(lora_down) ||
+      !aligned16(lora_up) || !aligned16(w) || !aligned16(y) || (bias && !aligned16(bias)))
+    return QL_ERR_ALIGN;
+  const size_t base = nvfp4_linear_workspace_size(M, K, N);
+  if (!workspace || workspace_bytes < svdq_nvfp4_linear_workspace_size(M, K, N, rank))
+    return QL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return QL_ERR_ALIGN;
+  int rc = check_device(nullptr);
+  if (rc != QL_OK) return rc;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int bn = ql::choose_config(true, M, N, K).bn;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* lr_act = ws + base;
+  // 1. smoothing + NVFP4 quantization of the smoothed activations, weight-scale layout
+  cudaError_t e = ql::launch_nvfp4_prologue(x, M, K, w_scale, N, bn, input_scale, ws, s, smooth);
+  if (e != cudaSuccess) return record(e, "svdq_nvfp4_linear prologue");
+  // 2. low-rank down projection of the smoothed activations (divided by alpha)
+  e = ql::launch_lowrank_down(x, M, K, smooth, lora_down, static_cast<int>(rank), input_scale,
+                              weight_scale_2, lr_act, s);
+  if (e != cudaSuccess) return record(e, "svdq_nvfp4_linear low-rank down");
+  // 3. the 4-bit GEMM with the low-rank up projection as one more K step
+  return nvfp4_gemm_impl(M, K, w, N, weight_scale_2, input_scale, bias, y, workspace,
+                         workspace_bytes, stream, true, lr_act, lora_up, static_cast<int>(rank));
+}
+
 int nvfp4_linear(const void* x, int64_t M, int64_t K, const uint8_t* w, const uint8_t* w_scale,
                  int64_t N, const float* weight_scale_2, const float* input_scale,
                  const float* bias, void* y, void* workspace, size_t workspace_bytes,

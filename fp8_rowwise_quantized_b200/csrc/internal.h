@@ -64,13 +64,20 @@ cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream);
 
 cudaError_t launch_nvfp4_quantize_rowmajor(const void* x, int64_t M, int64_t K, const float* g,
                                            uint8_t* xq, uint8_t* xs, cudaStream_t s);
+// smooth: per-column fp32 multipliers applied (bf16(RN32(x * smooth))) before
+// quantization, or null
 cudaError_t launch_nvfp4_prologue(const void* x, int64_t M, int64_t K, const uint8_t* w_scale,
                                   int64_t N, int bn, const float* input_scale, uint8_t* workspace,
-                                  cudaStream_t s);
+                                  cudaStream_t s, const float* smooth = nullptr);
 // Weight-scale layout only (the activation part of the workspace is left as is).
 cudaError_t launch_nvfp4_weight_layout(const uint8_t* w_scale, int64_t M, int64_t K, int64_t N,
                                        int bn, const float* input_scale, uint8_t* workspace,
                                        cudaStream_t s);
+// SVDQuant low-rank down projection: out bf16 [M, rank] = bf16((xs down^T) / alpha),
+// xs = bf16(RN32(x * smooth)) (smooth may be null), alpha = *scale_a * *scale_b.
+cudaError_t launch_lowrank_down(const void* x, int64_t M, int64_t K, const float* smooth,
+                                const void* down, int rank, const float* scale_a,
+                                const float* scale_b, void* out, cudaStream_t s);
 cudaError_t launch_fp8r_quantize_rows(const void* x, int64_t M, int64_t K, uint8_t* xq,
                                       float* x_scale, cudaStream_t s);
 cudaError_t launch_global_scale(const void* x, int64_t n, float* out, cudaStream_t s);

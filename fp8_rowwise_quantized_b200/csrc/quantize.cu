@@ -8,6 +8,7 @@
 //   * element encoder diagnostics.
 // The scheme is the one of the Diffusers page "BFL (fp8r / nvfp4)" (scheme list:
 // nvfp4 and fp8r entries; "Kernels" table: run-time activation quantization).
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cstdint>
 
@@ -56,20 +57,42 @@ __device__ __forceinline__ void nvfp4_load_item(uint32_t item, int lane,
   }
 }
 
+// SVDQuant smoothing of 8 bf16 values: bf16(RN32(x * smooth)) for the columns
+// e .. e+7 (smooth: fp32 per column of x).
+__device__ __forceinline__ uint4 smooth8(const uint4 u, const float* __restrict__ smooth) {
+  const float4 s0 = __ldg(reinterpret_cast<const float4*>(smooth));
+  const float4 s1 = __ldg(reinterpret_cast<const float4*>(smooth + 4));
+  const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat162 p = __floats2bfloat162_rn(__fmul_rn(bf16_lo(w[i]), sv[2 * i]),
+                                                   __fmul_rn(bf16_hi(w[i]), sv[2 * i + 1]));
+    o[i] = *reinterpret_cast<const uint32_t*>(&p);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 template <bool SF_MMA>
-__device__ __forceinline__ void nvfp4_encode_item(uint32_t item, int lane, const QuantItem& q,
+__device__ __forceinline__ void nvfp4_encode_item(uint32_t item, int lane, const QuantItem& qin,
                                                   int M, int K, float g, float c,
                                                   uint8_t* __restrict__ xq,
-                                                  uint8_t* __restrict__ xs, uint32_t segs, int KG) {
+                                                  uint8_t* __restrict__ xs, uint32_t segs, int KG,
+                                                  const float* __restrict__ smooth) {
   const int r = static_cast<int>(item / segs);
   const int seg = static_cast<int>(item - static_cast<uint32_t>(r) * segs);
   const int nblk = K >> 4;
   uint8_t* qr = xq + static_cast<int64_t>(r) * (K >> 1);
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
-    const uint4 u = q.raw[2 * i], v = q.raw[2 * i + 1];
     const int e = seg * 1024 + i * 512 + lane * 16;
     const bool valid = (r < M) && (e < K);
+    uint4 u = qin.raw[2 * i], v = qin.raw[2 * i + 1];
+    if (smooth && valid) {  // the smoothed activations are what gets quantized
+      u = smooth8(u, smooth + e);
+      v = smooth8(v, smooth + e + 8);
+    }
     const float amax = fmaxf(bf16x8_amax(u.x, u.y, u.z, u.w), bf16x8_amax(v.x, v.y, v.z, v.w));
     const float sf = __fmul_rn(amax, c);
     const uint32_t s = cvt_e4m3x4(sf, 0.0f, 0.0f, 0.0f) & 0xFFu;
@@ -124,7 +147,8 @@ __device__ __forceinline__ void nvfp4_quantize_items(uint32_t warp_id, uint32_t 
                                                      const uint16_t* __restrict__ x, int M, int K,
                                                      float g, float c, uint8_t* __restrict__ xq,
                                                      uint8_t* __restrict__ xs, uint32_t total,
-                                                     uint32_t segs, int KG) {
+                                                     uint32_t segs, int KG,
+                                                     const float* __restrict__ smooth = nullptr) {
   if (warp_id >= total) return;  // warp-uniform
   QuantItem cur;
   nvfp4_load_item(warp_id, lane, x, M, K, segs, cur);
@@ -132,7 +156,7 @@ __device__ __forceinline__ void nvfp4_quantize_items(uint32_t warp_id, uint32_t 
     QuantItem nxt;
     const uint32_t next = item + nwarps;
     if (next < total) nvfp4_load_item(next, lane, x, M, K, segs, nxt);
-    nvfp4_encode_item<SF_MMA>(item, lane, cur, M, K, g, c, xq, xs, segs, KG);
+    nvfp4_encode_item<SF_MMA>(item, lane, cur, M, K, g, c, xq, xs, segs, KG, smooth);
     cur = nxt;
   }
 }
@@ -212,13 +236,15 @@ nvfp4_prologue_kernel(const uint16_t* __restrict__ x, int M, int K,
                       const float* __restrict__ g_ptr, uint8_t* __restrict__ xq,
                       uint8_t* __restrict__ xs, uint32_t rows_total, uint32_t segs, int KG,
                       const uint8_t* __restrict__ ws, int64_t N, int bn, int na, int64_t n_tiles,
-                      int64_t w_jobs, uint8_t* __restrict__ wout) {
+                      int64_t w_jobs, uint8_t* __restrict__ wout,
+                      const float* __restrict__ smooth) {
   __shared__ uint32_t tile[128][kWsGroups + 1];
   const float g = __ldg(g_ptr);
   const float c = __frcp_rn(__fmul_rn(6.0f, g));
   constexpr uint32_t kWarps = kQuantThreads / 32;
   nvfp4_quantize_items<true>(blockIdx.x * kWarps + threadIdx.x / 32, gridDim.x * kWarps,
-                             threadIdx.x % 32, x, M, K, g, c, xq, xs, rows_total * segs, segs, KG);
+                             threadIdx.x % 32, x, M, K, g, c, xq, xs, rows_total * segs, segs, KG,
+                             smooth);
   for (int64_t job = blockIdx.x; job < w_jobs; job += gridDim.x) {
     nvfp4_weight_scale_atoms(job, threadIdx.x, ws, N, K, bn, na, n_tiles, KG, wout, tile);
     __syncthreads();  // the tile buffer is reused by the next job
@@ -364,7 +390,7 @@ cudaError_t launch_nvfp4_quantize_rowmajor(const void* x, int64_t M, int64_t K, 
 
 cudaError_t launch_nvfp4_prologue(const void* x, int64_t M, int64_t K, const uint8_t* w_scale,
                                   int64_t N, int bn, const float* input_scale, uint8_t* workspace,
-                                  cudaStream_t s) {
+                                  cudaStream_t s, const float* smooth) {
   const Nvfp4Workspace L = nvfp4_workspace(M, K, N, bn);
   const int64_t KG = sf_kgroups(K);
   const int64_t rows = ceil_div64(M, 128) * 128;
@@ -381,7 +407,7 @@ cudaError_t launch_nvfp4_prologue(const void* x, int64_t M, int64_t K, const uin
       static_cast<const uint16_t*>(x), static_cast<int>(M), static_cast<int>(K), input_scale,
       workspace + L.codes_off, workspace + L.act_sf_off, static_cast<uint32_t>(rows),
       static_cast<uint32_t>(segs), static_cast<int>(KG), w_scale, N, bn, na, n_tiles, w_jobs,
-      workspace + L.wgt_sf_off);
+      workspace + L.wgt_sf_off, smooth);
   return cudaGetLastError();
 }
 
@@ -400,7 +426,8 @@ cudaError_t launch_nvfp4_weight_layout(const uint8_t* w_scale, int64_t M, int64_
   nvfp4_prologue_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, 0, s>>>(
       nullptr, static_cast<int>(M), static_cast<int>(K), input_scale, workspace + L.codes_off,
       workspace + L.act_sf_off, 0u, static_cast<uint32_t>(ceil_div64(KG * 64, 1024)),
-      static_cast<int>(KG), w_scale, N, bn, na, n_tiles, w_jobs, workspace + L.wgt_sf_off);
+      static_cast<int>(KG), w_scale, N, bn, na, n_tiles, w_jobs, workspace + L.wgt_sf_off,
+      nullptr);
   return cudaGetLastError();
 }
 

@@ -95,6 +95,30 @@ int nvfp4_linear_gemm_lowrank(int64_t M, int64_t K, const uint8_t* w, int64_t N,
                               int64_t rank, void* y, const void* workspace,
                               size_t workspace_bytes, ql_stream_t stream);
 
+/* SVDQuant-style NVFP4 linear (svdq_w4a4, NVFP4 variant, of the Diffusers page
+ * "Bringing Nunchaku 4-bit Diffusion Inference to Diffusers": activation outliers
+ * moved into the weights, a 16-bit low-rank branch, the residual in 4 bits):
+ *   xs = bf16(RN32(x * smooth))                 (per input column; smooth may be NULL)
+ *   Y  = bf16( input_scale * weight_scale_2 * NVFP4(xs) NVFP4(w)^T
+ *              + (xs lora_down^T) lora_up^T + bias )
+ *   x          bf16 [M, K]
+ *   smooth     fp32 [K] multipliers, or NULL (xs = x)
+ *   lora_down  bf16 [rank, K]; lora_up bf16 [N, rank]; 8 <= rank <= 64, rank % 8 == 0
+ *   w, w_scale, weight_scale_2, bias, y  as nvfp4_linear (w: the 4-bit residual)
+ *   input_scale  the calibrated global scale of xs
+ *   workspace  >= svdq_nvfp4_linear_workspace_size(M, K, N, rank) bytes
+ * Three launches: the prologue (smoothing, quantization of xs, weight-scale
+ * layout); the low-rank down projection (warp-level bf16 tensor-core MMA) into the
+ * workspace; the 4-bit GEMM with the low-rank up projection as one more bf16 K step
+ * into the same accumulator (the fusion the page describes for the up projection).
+ * Requires the nvfp4_linear shapes and 16-byte aligned pointers. */
+size_t svdq_nvfp4_linear_workspace_size(int64_t M, int64_t K, int64_t N, int64_t rank);
+int svdq_nvfp4_linear(const void* x, int64_t M, int64_t K, const float* smooth,
+                      const void* lora_down, const void* lora_up, int64_t rank, const uint8_t* w,
+                      const uint8_t* w_scale, int64_t N, const float* weight_scale_2,
+                      const float* input_scale, const float* bias, void* y, void* workspace,
+                      size_t workspace_bytes, ql_stream_t stream);
+
 /* The MLP up projection with its GELU and the down projection's quantization
  * fused into the GEMM epilogue (the "fused GELU/MLP" kernels of the Diffusers
  * page "Nunchaku" section, for the nvfp4 scheme): instead of Y it writes

@@ -68,3 +68,86 @@ def test_gemm_lowrank_rejects_bad_rank():
         with pytest.raises(q.QLinearError):
             q.nvfp4_linear_gemm_lowrank(128, d["w"], d["weight_scale_2"], d["input_scale"], ws,
                                         act, up)
+
+
+class SvdqCase:
+    """Seeded svdq layer: outlier activations, per-column smoothing multipliers
+    (1 / sqrt of the column's amax, so outlier columns are scaled down), a rank-r
+    bf16 branch and an oracle-quantized 4-bit residual weight."""
+
+    def __init__(self, M, K, N, r, seed, bias=True):
+        c = Nvfp4Case(M, K, N, seed=seed, bias=bias)
+        self.M, self.K, self.N, self.r = M, K, N, r
+        self.x, self.wq, self.ws, self.gw, self.bias = c.x, c.wq, c.ws, c.gw, c.bias
+        amax = c.x.float().abs().amax(dim=0).clamp(min=1e-3)
+        self.smooth = (1.0 / amax.sqrt()).numpy().astype(np.float32)
+        self.down, self.up = lowrank_operands(K, N, r, seed=seed + 1)
+        self.xs = oracle.smooth_bf16(self.x, self.smooth)
+        self.gx = np.float32(oracle.nvfp4_global_scale(self.xs))
+
+    def device_args(self):
+        return dict(x=to_dev(self.x), w=to_dev(self.wq), w_scale=to_dev(self.ws),
+                    weight_scale_2=scalar_dev(self.gw), input_scale=scalar_dev(float(self.gx)),
+                    lora_down=to_dev(self.down), lora_up=to_dev(self.up),
+                    smooth=to_dev(torch.from_numpy(self.smooth)),
+                    bias=None if self.bias is None else to_dev(self.bias))
+
+    def reference(self):
+        xq, xsc = oracle.nvfp4_quantize(self.xs, self.gx)
+        D = oracle.lowrank_down(self.xs, self.down)
+        return (xq, xsc, D) + oracle.svdq_nvfp4_linear(xq, xsc, self.wq, self.ws, self.gx,
+                                                       self.gw, D, self.up, self.bias)
+
+
+@pytest.mark.parametrize("M,K,N,r", [
+    (600, 512, 520, 32),
+    (130, 1024, 1536, 16),
+    (1024, 3072, 3072, 32),
+])
+def test_svdq_linear_end_to_end(M, K, N, r):
+    from gpu_helpers import unpack_act_scale_atoms
+    c = SvdqCase(M, K, N, r, seed=M + r)
+    d = c.device_args()
+    ws = torch.full((q.svdq_nvfp4_linear_workspace_size(M, K, N, r),), 0xCD, dtype=torch.uint8,
+                    device="cuda")
+    y = q.svdq_nvfp4_linear(d["x"], d["w"], d["w_scale"], d["weight_scale_2"], d["input_scale"],
+                            d["lora_down"], d["lora_up"], smooth=d["smooth"], bias=d["bias"],
+                            workspace=ws)
+    torch.cuda.synchronize()
+    xq, xsc, D, _, y64, T, Tlr = c.reference()
+    # the smoothed activations' codes and scales: bit-exact
+    codes_off, sf_off, _ = q.nvfp4_linear_workspace_layout(M, K, N)
+    buf = ws.cpu().numpy()
+    assert np.array_equal(buf[codes_off:codes_off + M * K // 2].reshape(M, K // 2), xq)
+    atoms = buf[sf_off:sf_off + -(-M // 128) * (-(-K // 256) * 4) * 512]
+    assert np.array_equal(unpack_act_scale_atoms(atoms, M, K), xsc)
+    # the branch activations bf16(D / alpha), from fp32 tensor-core sums: within one ulp
+    alpha = float(np.float32(c.gx) * np.float32(c.gw))
+    base = q.nvfp4_linear_workspace_size(M, K, N)
+    lr = oracle.bf16_bits_to_f64(buf[base:base + M * r * 2].view(np.uint16).reshape(M, r))
+    want = D / alpha
+    assert np.all(np.abs(lr - want) <= 2.0 * oracle.bf16_ulp(want) + 1e-30)
+    check_linear(y, y64, T, f"svdq {M}x{K}x{N} r{r}", extra=LR_TOL * Tlr)
+
+
+def test_svdq_without_smoothing_equals_gemm_lowrank_path():
+    M, K, N, r = 512, 768, 1000, 32
+    c = SvdqCase(M, K, N, r, seed=9)
+    d = c.device_args()
+    gx = scalar_dev(float(np.float32(oracle.nvfp4_global_scale(c.x))))
+    y1 = q.svdq_nvfp4_linear(d["x"], d["w"], d["w_scale"], d["weight_scale_2"], gx,
+                             d["lora_down"], d["lora_up"], bias=d["bias"])
+    torch.cuda.synchronize()
+    # the same branch activations through the split calls
+    ws = torch.empty(q.nvfp4_linear_workspace_size(M, K, N), dtype=torch.uint8, device="cuda")
+    q.nvfp4_linear_prologue(d["x"], d["w_scale"], gx, ws)
+    wsv = torch.empty(q.svdq_nvfp4_linear_workspace_size(M, K, N, r), dtype=torch.uint8,
+                      device="cuda")
+    q.svdq_nvfp4_linear(d["x"], d["w"], d["w_scale"], d["weight_scale_2"], gx, d["lora_down"],
+                        d["lora_up"], bias=d["bias"], workspace=wsv)
+    base = q.nvfp4_linear_workspace_size(M, K, N)
+    lr_act = wsv[base:base + M * r * 2].view(torch.bfloat16).reshape(M, r)
+    y2 = q.nvfp4_linear_gemm_lowrank(M, d["w"], d["weight_scale_2"], gx, ws, lr_act.clone(),
+                                     d["lora_up"], bias=d["bias"])
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
