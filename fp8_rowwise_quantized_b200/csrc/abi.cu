@@ -297,20 +297,20 @@ int svdq_nvfp4_linear(const void* x, int64_t M, int64_t K, const float* smooth,
   if (!workspace || workspace_bytes < svdq_nvfp4_linear_workspace_size(M, K, N, rank))
     return QL_ERR_WORKSPACE;
   if (!aligned16(workspace)) return QL_ERR_ALIGN;
-  int rc = check_device(nullptr);
+  int dev = 0;
+  int rc = check_device(&dev);
   if (rc != QL_OK) return rc;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int bn = ql::choose_config(true, M, N, K).bn;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* lr_act = ws + base;
-  // 1. smoothing + NVFP4 quantization of the smoothed activations, weight-scale layout
-  cudaError_t e = ql::launch_nvfp4_prologue(x, M, K, w_scale, N, bn, input_scale, ws, s, smooth);
+  // 1. one pass over x: smoothing, NVFP4 of the smoothed activations, the low-rank
+  //    down projection (divided by alpha), weight-scale layout
+  const cudaError_t e = ql::launch_svdq_prologue(
+      x, M, K, smooth, lora_down, static_cast<int>(rank), w_scale, N, bn, input_scale,
+      weight_scale_2, ws, lr_act, status_ptr(dev), timeout_ns(), s);
   if (e != cudaSuccess) return record(e, "svdq_nvfp4_linear prologue");
-  // 2. low-rank down projection of the smoothed activations (divided by alpha)
-  e = ql::launch_lowrank_down(x, M, K, smooth, lora_down, static_cast<int>(rank), input_scale,
-                              weight_scale_2, lr_act, s);
-  if (e != cudaSuccess) return record(e, "svdq_nvfp4_linear low-rank down");
-  // 3. the 4-bit GEMM with the low-rank up projection as one more K step
+  // 2. the 4-bit GEMM with the low-rank up projection as one more K step
   return nvfp4_gemm_impl(M, K, w, N, weight_scale_2, input_scale, bias, y, workspace,
                          workspace_bytes, stream, true, lr_act, lora_up, static_cast<int>(rank));
 }

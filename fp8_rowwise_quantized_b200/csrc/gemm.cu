@@ -1033,12 +1033,14 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
 
 // ---------------------------------------------------------------- host side
 
+}  // namespace
+
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-EncodeTiledFn get_encode_fn() {
+static EncodeTiledFn get_encode_fn() {
   static EncodeTiledFn fn = nullptr;
   static std::once_flag once;
   std::call_once(once, [] {
@@ -1065,6 +1067,8 @@ bool encode_2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, uin
              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, promo,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+namespace {
 
 template <bool FP4, int BN, int CG, int MODE>
 cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {

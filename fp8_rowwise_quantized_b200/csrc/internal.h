@@ -1,5 +1,6 @@
 // Host-side declarations shared by the translation units of the library.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstddef>
 #include <cstdint>
@@ -64,24 +65,34 @@ cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream);
 
 cudaError_t launch_nvfp4_quantize_rowmajor(const void* x, int64_t M, int64_t K, const float* g,
                                            uint8_t* xq, uint8_t* xs, cudaStream_t s);
-// smooth: per-column fp32 multipliers applied (bf16(RN32(x * smooth))) before
-// quantization, or null
 cudaError_t launch_nvfp4_prologue(const void* x, int64_t M, int64_t K, const uint8_t* w_scale,
                                   int64_t N, int bn, const float* input_scale, uint8_t* workspace,
-                                  cudaStream_t s, const float* smooth = nullptr);
+                                  cudaStream_t s);
 // Weight-scale layout only (the activation part of the workspace is left as is).
 cudaError_t launch_nvfp4_weight_layout(const uint8_t* w_scale, int64_t M, int64_t K, int64_t N,
                                        int bn, const float* input_scale, uint8_t* workspace,
                                        cudaStream_t s);
-// SVDQuant low-rank down projection: out bf16 [M, rank] = bf16((xs down^T) / alpha),
-// xs = bf16(RN32(x * smooth)) (smooth may be null), alpha = *scale_a * *scale_b.
-cudaError_t launch_lowrank_down(const void* x, int64_t M, int64_t K, const float* smooth,
-                                const void* down, int rank, const float* scale_a,
-                                const float* scale_b, void* out, cudaStream_t s);
+// Prologue of the SVDQuant-style linear in one launch: NVFP4 codes and scale atoms
+// of xs = bf16(RN32(x * smooth)) (smooth may be null) into the nvfp4_linear
+// workspace, lr_act bf16 [M, rank] = bf16((xs down^T) / alpha) with alpha =
+// *input_scale * *weight_scale_2 (rank % 8 == 0, rank <= 64; rank 0 skips it), and
+// the weight scales in atom layout for tiles of bn rows. x 16-byte aligned, K % 32 == 0.
+cudaError_t launch_svdq_prologue(const void* x, int64_t M, int64_t K, const float* smooth,
+                                 const void* down, int rank, const uint8_t* w_scale, int64_t N,
+                                 int bn, const float* input_scale, const float* weight_scale_2,
+                                 uint8_t* workspace, void* lr_act, int* status,
+                                 uint64_t timeout_ns, cudaStream_t s);
 cudaError_t launch_fp8r_quantize_rows(const void* x, int64_t M, int64_t K, uint8_t* xq,
                                       float* x_scale, cudaStream_t s);
 cudaError_t launch_global_scale(const void* x, int64_t n, float* out, cudaStream_t s);
 cudaError_t launch_encode(const float* in, uint8_t* out, int64_t n, bool fp4, cudaStream_t s);
+
+// 2-D tiled tensor map over a row-major matrix (rows x inner elements, rows
+// `row_bytes` apart) with boxes of box_rows x box_inner; false when the driver
+// entry point is missing or rejects the arguments. Out-of-range elements load as 0.
+bool encode_2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, uint64_t inner,
+               uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows,
+               CUtensorMapSwizzle swz, CUtensorMapL2promotion promo);
 
 // Sets the text ql_last_error_message() returns on this thread.
 void set_error_text(const char* text);

@@ -15,6 +15,7 @@
 #include "internal.h"
 #include "layout.cuh"
 #include "ptx.cuh"
+#include "quant.cuh"
 
 namespace ql {
 
@@ -42,11 +43,9 @@ struct QuantItem {
   uint4 raw[4];
 };
 
-__device__ __forceinline__ void nvfp4_load_item(uint32_t item, int lane,
+__device__ __forceinline__ void nvfp4_load_item(int r, int seg, int lane,
                                                 const uint16_t* __restrict__ x, int M, int K,
-                                                uint32_t segs, QuantItem& q) {
-  const int r = static_cast<int>(item / segs);
-  const int seg = static_cast<int>(item - static_cast<uint32_t>(r) * segs);
+                                                QuantItem& q) {
   const uint16_t* xr = x + static_cast<int64_t>(r) * K;
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
@@ -57,60 +56,20 @@ __device__ __forceinline__ void nvfp4_load_item(uint32_t item, int lane,
   }
 }
 
-// SVDQuant smoothing of 8 bf16 values: bf16(RN32(x * smooth)) for the columns
-// e .. e+7 (smooth: fp32 per column of x).
-__device__ __forceinline__ uint4 smooth8(const uint4 u, const float* __restrict__ smooth) {
-  const float4 s0 = __ldg(reinterpret_cast<const float4*>(smooth));
-  const float4 s1 = __ldg(reinterpret_cast<const float4*>(smooth + 4));
-  const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-  uint32_t o[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const __nv_bfloat162 p = __floats2bfloat162_rn(__fmul_rn(bf16_lo(w[i]), sv[2 * i]),
-                                                   __fmul_rn(bf16_hi(w[i]), sv[2 * i + 1]));
-    o[i] = *reinterpret_cast<const uint32_t*>(&p);
-  }
-  return make_uint4(o[0], o[1], o[2], o[3]);
-}
-
 template <bool SF_MMA>
-__device__ __forceinline__ void nvfp4_encode_item(uint32_t item, int lane, const QuantItem& qin,
+__device__ __forceinline__ void nvfp4_encode_item(int r, int seg, int lane, const QuantItem& qin,
                                                   int M, int K, float g, float c,
                                                   uint8_t* __restrict__ xq,
-                                                  uint8_t* __restrict__ xs, uint32_t segs, int KG,
-                                                  const float* __restrict__ smooth) {
-  const int r = static_cast<int>(item / segs);
-  const int seg = static_cast<int>(item - static_cast<uint32_t>(r) * segs);
+                                                  uint8_t* __restrict__ xs, int KG) {
   const int nblk = K >> 4;
   uint8_t* qr = xq + static_cast<int64_t>(r) * (K >> 1);
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
     const int e = seg * 1024 + i * 512 + lane * 16;
     const bool valid = (r < M) && (e < K);
-    uint4 u = qin.raw[2 * i], v = qin.raw[2 * i + 1];
-    if (smooth && valid) {  // the smoothed activations are what gets quantized
-      u = smooth8(u, smooth + e);
-      v = smooth8(v, smooth + e + 8);
-    }
-    const float amax = fmaxf(bf16x8_amax(u.x, u.y, u.z, u.w), bf16x8_amax(v.x, v.y, v.z, v.w));
-    const float sf = __fmul_rn(amax, c);
-    const uint32_t s = cvt_e4m3x4(sf, 0.0f, 0.0f, 0.0f) & 0xFFu;
-    const float d = __fmul_rn(e4m3_to_float(s), g);
-    uint2 codes = make_uint2(0u, 0u);
-    if (d != 0.0f) {
-      const float inv = __frcp_rn(d);
-      const uint32_t w[8] = {u.x, u.y, u.z, u.w, v.x, v.y, v.z, v.w};
-      float fa[8], fb[8];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        fa[2 * j] = __fmul_rn(bf16_lo(w[j]), inv);
-        fa[2 * j + 1] = __fmul_rn(bf16_hi(w[j]), inv);
-        fb[2 * j] = __fmul_rn(bf16_lo(w[4 + j]), inv);
-        fb[2 * j + 1] = __fmul_rn(bf16_hi(w[4 + j]), inv);
-      }
-      codes = make_uint2(cvt_e2m1x8(fa), cvt_e2m1x8(fb));
-    }
+    const uint4 u = qin.raw[2 * i], v = qin.raw[2 * i + 1];
+    uint32_t s;
+    const uint2 codes = nvfp4_block16(u, v, g, c, s);
     if (valid) *reinterpret_cast<uint2*>(qr + (e >> 1)) = codes;
     // gather the scales of blocks lane .. lane+3 into lanes 0, 4, ..., 28
     const uint32_t s1 = __shfl_down_sync(0xffffffffu, s, 1);
@@ -147,17 +106,27 @@ __device__ __forceinline__ void nvfp4_quantize_items(uint32_t warp_id, uint32_t 
                                                      const uint16_t* __restrict__ x, int M, int K,
                                                      float g, float c, uint8_t* __restrict__ xq,
                                                      uint8_t* __restrict__ xs, uint32_t total,
-                                                     uint32_t segs, int KG,
-                                                     const float* __restrict__ smooth = nullptr) {
+                                                     uint32_t segs, int KG) {
   if (warp_id >= total) return;  // warp-uniform
+  // item = r * segs + seg, advanced by nwarps per iteration without dividing
+  const uint32_t dr = nwarps / segs, ds = nwarps - (nwarps / segs) * segs;
+  uint32_t r = warp_id / segs, seg = warp_id - (warp_id / segs) * segs;
   QuantItem cur;
-  nvfp4_load_item(warp_id, lane, x, M, K, segs, cur);
+  nvfp4_load_item(static_cast<int>(r), static_cast<int>(seg), lane, x, M, K, cur);
   for (uint32_t item = warp_id; item < total; item += nwarps) {
+    uint32_t rn = r + dr, sn = seg + ds;
+    if (sn >= segs) {
+      sn -= segs;
+      ++rn;
+    }
     QuantItem nxt;
-    const uint32_t next = item + nwarps;
-    if (next < total) nvfp4_load_item(next, lane, x, M, K, segs, nxt);
-    nvfp4_encode_item<SF_MMA>(item, lane, cur, M, K, g, c, xq, xs, segs, KG, smooth);
+    if (item + nwarps < total)
+      nvfp4_load_item(static_cast<int>(rn), static_cast<int>(sn), lane, x, M, K, nxt);
+    nvfp4_encode_item<SF_MMA>(static_cast<int>(r), static_cast<int>(seg), lane, cur, M, K, g, c,
+                              xq, xs, KG);
     cur = nxt;
+    r = rn;
+    seg = sn;
   }
 }
 
@@ -174,56 +143,6 @@ nvfp4_quantize_kernel(const uint16_t* __restrict__ x, int M, int K,
                                KG);
 }
 
-// Row-major weight scales [N, K/16] -> atom layout for tiles of `bn` rows, through
-// shared memory so that both the reads (64 contiguous bytes per row) and the
-// writes (whole 512-byte atoms) are coalesced. One block per (tile, 128-row atom
-// a, 16 consecutive 64-element groups).
-constexpr int kWsGroups = 16;
-__device__ __forceinline__ void nvfp4_weight_scale_atoms(int64_t job, int tid,
-                                                         const uint8_t* __restrict__ ws, int64_t N,
-                                                         int64_t K, int bn, int na, int64_t n_tiles,
-                                                         int64_t KG, uint8_t* __restrict__ out,
-                                                         uint32_t (*tile)[kWsGroups + 1]) {
-  const int64_t kg_chunks = ceil_div64(KG, kWsGroups);
-  const int64_t kc = job % kg_chunks;
-  const int a = static_cast<int>((job / kg_chunks) % na);
-  const int64_t t = job / (kg_chunks * na);
-  const int64_t nblk = K / 16;
-  // load: 128 rows x 16 groups; thread -> (row = tid / 2, groups 8 * (tid % 2) .. +8)
-  {
-    const int rr = tid / 2;
-    const int g0 = (tid % 2) * 8;
-    const int64_t nn = static_cast<int64_t>(a) * 128 + rr;
-    const int64_t n = t * bn + nn;
-    const bool row_ok = nn < bn && n < N;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int64_t kg = kc * kWsGroups + g0 + j;
-      uint32_t word = 0;
-      if (row_ok && 4 * kg < nblk) {
-        const uint8_t* src = ws + n * nblk + kg * 4;
-        if (4 * kg + 4 <= nblk && (reinterpret_cast<uintptr_t>(src) & 3) == 0) {
-          word = __ldg(reinterpret_cast<const uint32_t*>(src));
-        } else {
-          for (int b = 0; b < 4; ++b)
-            if (4 * kg + b < nblk) word |= static_cast<uint32_t>(__ldg(src + b)) << (8 * b);
-        }
-      }
-      tile[rr][g0 + j] = word;
-    }
-  }
-  __syncthreads();
-  // store: per group, one 512-byte atom = 128 words; thread tid writes word tid % 128
-  for (int j = tid / 128; j < kWsGroups; j += 2) {
-    const int64_t kg = kc * kWsGroups + j;
-    if (kg >= KG) continue;
-    const int w = tid % 128;
-    const int rr = (w % 4) * 32 + w / 4;  // word w holds row rr of the atom
-    uint8_t* atom = out + static_cast<size_t>(((t * KG) + kg) * na + a) * kSfAtomBytes;
-    reinterpret_cast<uint32_t*>(atom)[w] = tile[rr][j];
-  }
-}
-
 // The prologue of nvfp4_linear in one launch, one wave of resident blocks: each
 // block's warps first quantize activation items (codes row-major, scales in atom
 // layout) in a grid-stride loop, then the block takes weight-scale layout jobs.
@@ -236,17 +155,17 @@ nvfp4_prologue_kernel(const uint16_t* __restrict__ x, int M, int K,
                       const float* __restrict__ g_ptr, uint8_t* __restrict__ xq,
                       uint8_t* __restrict__ xs, uint32_t rows_total, uint32_t segs, int KG,
                       const uint8_t* __restrict__ ws, int64_t N, int bn, int na, int64_t n_tiles,
-                      int64_t w_jobs, uint8_t* __restrict__ wout,
-                      const float* __restrict__ smooth) {
-  __shared__ uint32_t tile[128][kWsGroups + 1];
+                      int64_t w_jobs, uint8_t* __restrict__ wout) {
+  __shared__ WsTile tile;
   const float g = __ldg(g_ptr);
   const float c = __frcp_rn(__fmul_rn(6.0f, g));
   constexpr uint32_t kWarps = kQuantThreads / 32;
   nvfp4_quantize_items<true>(blockIdx.x * kWarps + threadIdx.x / 32, gridDim.x * kWarps,
-                             threadIdx.x % 32, x, M, K, g, c, xq, xs, rows_total * segs, segs, KG,
-                             smooth);
+                             threadIdx.x % 32, x, M, K, g, c, xq, xs, rows_total * segs, segs, KG);
   for (int64_t job = blockIdx.x; job < w_jobs; job += gridDim.x) {
-    nvfp4_weight_scale_atoms(job, threadIdx.x, ws, N, K, bn, na, n_tiles, KG, wout, tile);
+    weight_scale_atoms_load(job, threadIdx.x, ws, N, K, bn, na, KG, tile);
+    __syncthreads();
+    weight_scale_atoms_store(job, threadIdx.x, na, KG, wout, tile);
     __syncthreads();  // the tile buffer is reused by the next job
   }
   grid_dependents_launch();
@@ -390,7 +309,7 @@ cudaError_t launch_nvfp4_quantize_rowmajor(const void* x, int64_t M, int64_t K, 
 
 cudaError_t launch_nvfp4_prologue(const void* x, int64_t M, int64_t K, const uint8_t* w_scale,
                                   int64_t N, int bn, const float* input_scale, uint8_t* workspace,
-                                  cudaStream_t s, const float* smooth) {
+                                  cudaStream_t s) {
   const Nvfp4Workspace L = nvfp4_workspace(M, K, N, bn);
   const int64_t KG = sf_kgroups(K);
   const int64_t rows = ceil_div64(M, 128) * 128;
@@ -407,7 +326,7 @@ cudaError_t launch_nvfp4_prologue(const void* x, int64_t M, int64_t K, const uin
       static_cast<const uint16_t*>(x), static_cast<int>(M), static_cast<int>(K), input_scale,
       workspace + L.codes_off, workspace + L.act_sf_off, static_cast<uint32_t>(rows),
       static_cast<uint32_t>(segs), static_cast<int>(KG), w_scale, N, bn, na, n_tiles, w_jobs,
-      workspace + L.wgt_sf_off, smooth);
+      workspace + L.wgt_sf_off);
   return cudaGetLastError();
 }
 
@@ -426,8 +345,7 @@ cudaError_t launch_nvfp4_weight_layout(const uint8_t* w_scale, int64_t M, int64_
   nvfp4_prologue_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, 0, s>>>(
       nullptr, static_cast<int>(M), static_cast<int>(K), input_scale, workspace + L.codes_off,
       workspace + L.act_sf_off, 0u, static_cast<uint32_t>(ceil_div64(KG * 64, 1024)),
-      static_cast<int>(KG), w_scale, N, bn, na, n_tiles, w_jobs, workspace + L.wgt_sf_off,
-      nullptr);
+      static_cast<int>(KG), w_scale, N, bn, na, n_tiles, w_jobs, workspace + L.wgt_sf_off);
   return cudaGetLastError();
 }
 
