@@ -68,6 +68,11 @@ def lib():
         L.oracle_fp8r_linear.argtypes = [u8p, f32p, i64, i64, u8p, f32p, i64, f32p,
                                          u16p, f64p, f64p]
         L.oracle_fp8r_linear.restype = C.c_int
+        L.oracle_w4a16_dequantize_bf16.argtypes = [u8p, u8p, i64, i64, C.c_float, u16p]
+        L.oracle_w4a16_dequantize_bf16.restype = C.c_int
+        L.oracle_w4a16_linear.argtypes = [u16p, i64, i64, u8p, u8p, i64, C.c_float, f32p, u16p,
+                                          f64p, f64p]
+        L.oracle_w4a16_linear.restype = C.c_int
         _lib = L
     return _lib
 
@@ -267,6 +272,41 @@ def nvfp4_linear_unquantized_act(x, wq, ws, weight_scale_2, bias=None):
     if rc != 0:
         raise ValueError("bad shape")
     return y64
+
+
+def w4a16_dequantize_bf16(q, s, weight_scale_2) -> np.ndarray:
+    """bf16 bits [R, K] of bf16(fp32(E2M1(q) * E4M3(s) * weight_scale_2))."""
+    q = np.ascontiguousarray(q, np.uint8)
+    s = np.ascontiguousarray(s, np.uint8)
+    R, K = q.shape[0], q.shape[1] * 2
+    out = np.empty((R, K), np.uint16)
+    rc = lib().oracle_w4a16_dequantize_bf16(_p(q, C.c_uint8), _p(s, C.c_uint8), R, K,
+                                            np.float32(weight_scale_2), _p(out, C.c_uint16))
+    if rc != 0:
+        raise ValueError("oracle_w4a16_dequantize_bf16: bad shape")
+    return out
+
+
+def w4a16_linear(x, wq, ws, weight_scale_2, bias=None):
+    """W4A16 linear on bf16 activations x [M, K] and NVFP4 weights: returns (y bf16
+    bits [M, N], y fp64 [M, N], tolerance scale T fp64 [M, N])."""
+    xb = _bits16(x)
+    wq = np.ascontiguousarray(wq, np.uint8)
+    ws = np.ascontiguousarray(ws, np.uint8)
+    M, K = xb.shape
+    N = wq.shape[0]
+    assert wq.shape[1] * 2 == K and ws.shape == (N, K // 16)
+    b = None if bias is None else np.ascontiguousarray(bias, np.float32)
+    y = np.empty((M, N), np.uint16)
+    y64 = np.empty((M, N), np.float64)
+    T = np.empty((M, N), np.float64)
+    rc = lib().oracle_w4a16_linear(_p(xb, C.c_uint16), M, K, _p(wq, C.c_uint8),
+                                   _p(ws, C.c_uint8), N, np.float32(weight_scale_2),
+                                   _p(b, C.c_float), _p(y, C.c_uint16), _p(y64, C.c_double),
+                                   _p(T, C.c_double))
+    if rc != 0:
+        raise ValueError("oracle_w4a16_linear: bad shape")
+    return y, y64, T
 
 
 def fp8r_quantize_rows(x):

@@ -513,4 +513,51 @@ int oracle_fp8r_linear(const uint8_t* xq, const float* xs, int64_t M, int64_t K,
   return 0;
 }
 
+// ---------------------------------------------------------------------------
+// W4A16: NVFP4 weights with 16-bit activations. The 4-bit weight kernel family
+// of "Bringing Nunchaku 4-bit Diffusion Inference to Diffusers" (section
+// "Introducing Nunchaku Lite", the W4A16 family: memory-bound modulation layers),
+// taken with the weight format of "BFL (fp8r / nvfp4)" and the semantics that page
+// gives for devices without the fused kernel ("Kernels", last paragraph): the
+// weight is dequantized to the compute dtype (bf16) and the layer runs as a plain
+// linear on unquantized activations.
+//   what[n, k] = bf16( fp32( E2M1(q[n,k]) * E4M3(s[n, k/16]) * weight_scale_2 ) )
+// The triple product is exact in fp64 (at most 2 + 4 + 24 significant bits); it is
+// rounded once to fp32 (the dequantization arithmetic) and then to bf16 (the cast
+// to the compute dtype).
+// ---------------------------------------------------------------------------
+int oracle_w4a16_dequantize_bf16(const uint8_t* q, const uint8_t* s, int64_t R, int64_t K,
+                                 float weight_scale_2, uint16_t* out) {
+  if (R < 0 || K <= 0 || K % 16 != 0) return -1;
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < R; ++r) {
+    for (int64_t k = 0; k < K; ++k) {
+      const uint8_t byte = q[r * (K / 2) + k / 2];
+      const uint8_t nib = (k % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+      const double exact = oracle_e2m1_decode(nib) * oracle_e4m3_decode(s[r * (K / 16) + k / 16]) *
+                           (double)weight_scale_2;
+      const float w32 = (float)exact;  // one RN to fp32
+      out[r * K + k] = oracle_bf16_from_double((double)w32);
+    }
+  }
+  return 0;
+}
+
+// W4A16 linear: Y[m, n] = bf16( sum_k x[m,k] * what[n,k] + bias[n] ), the sum in
+// fp64 in increasing k (the products of two bf16 values are exact), with the
+// tolerance scale T[m, n] = sum_k |x[m,k] * what[n,k]|.
+int oracle_w4a16_linear(const uint16_t* x, int64_t M, int64_t K, const uint8_t* wq,
+                        const uint8_t* ws, int64_t N, float weight_scale_2, const float* bias,
+                        uint16_t* y, double* y64, double* T) {
+  if (M < 0 || N < 0 || K <= 0 || K % 16 != 0) return -1;
+  std::vector<uint16_t> wb((size_t)N * K);
+  oracle_w4a16_dequantize_bf16(wq, ws, N, K, weight_scale_2, wb.data());
+  std::vector<double> A((size_t)M * K), B((size_t)N * K);
+  for (int64_t i = 0; i < M * K; ++i) A[i] = (double)bf16_to_float(x[i]);
+  for (int64_t i = 0; i < N * K; ++i) B[i] = (double)bf16_to_float(wb[i]);
+  std::vector<double> am((size_t)M, 1.0), an((size_t)N, 1.0);
+  contract(A.data(), B.data(), M, K, N, am.data(), an.data(), bias, y, y64, T);
+  return 0;
+}
+
 }  // extern "C"
