@@ -300,6 +300,201 @@ def time_events(fn, steps, warmup, flush, stream):
     return statistics.fmean(times), times
 
 
+L2_BYTES = 126 << 20
+ROTATION_BYTES = 4 * L2_BYTES
+
+
+class Nvfp4Rotation:
+    """R copies of one NVFP4 layer's device buffers (x, weight codes and scales,
+    bias, y, workspace), R chosen so that all copies together hold at least four
+    times the L2. Stepping through them in turn makes every call find its
+    operands in HBM, not in L2, as in a stack of distinct layers; nothing is
+    written between calls, so no flush write-back lands in the timed region."""
+
+    def __init__(self, layer, min_bytes=ROTATION_BYTES):
+        import torch
+        self.L = layer
+        per = sum(t.numel() * t.element_size() for t in
+                  (layer.x, layer.wq, layer.ws, layer.y, layer.work) if t is not None)
+        if layer.bias is not None:
+            per += layer.bias.numel() * 4
+        self.R = max(2, -(-min_bytes // per))
+        self.bytes_per_set = per
+
+        def clone(t):
+            return None if t is None else t.clone()
+        self.sets = [(layer.x, layer.wq, layer.ws, layer.bias, layer.y, layer.work)]
+        for _ in range(self.R - 1):
+            self.sets.append((clone(layer.x), clone(layer.wq), clone(layer.ws), clone(layer.bias),
+                              torch.empty_like(layer.y), torch.empty_like(layer.work)))
+        self.i = 0
+
+    def _next(self):
+        s = self.sets[self.i]
+        self.i = (self.i + 1) % self.R
+        return s
+
+    def step(self):
+        x, wq, ws, b, y, work = self._next()
+        self.L.q.nvfp4_linear(x, wq, ws, self.L.gw, self.L.gx, bias=b, y=y, workspace=work)
+
+    def prologue_all(self):
+        for x, wq, ws, b, y, work in self.sets:
+            self.L.q.nvfp4_linear_prologue(x, ws, self.L.gx, work)
+
+    def gemm(self):
+        x, wq, ws, b, y, work = self._next()
+        self.L.q.nvfp4_linear_gemm(self.L.M, wq, self.L.gw, self.L.gx, work, bias=b, y=y)
+
+    def prologue(self):
+        x, wq, ws, b, y, work = self._next()
+        self.L.q.nvfp4_linear_prologue(x, ws, self.L.gx, work)
+
+    def quantize_act(self):
+        # codes and scales into the set's workspace (row-major, as the call returns them)
+        x, wq, ws, b, y, work = self._next()
+        M, K = self.L.M, self.L.K
+        xq = work[:M * K // 2].view(M, K // 2)
+        xs = work[M * K // 2:M * K // 2 + M * K // 16].view(M, K // 16)
+        self.L.q.nvfp4_quantize_act(x, self.L.gx, xq, xs)
+
+
+def time_graph_rotation(fn, calls, reps, stream):
+    """Mean device time (ms) of one call of fn, where fn cycles through buffer sets
+    larger than L2: `calls` consecutive calls (one per set) are captured in a CUDA
+    graph, the graph is replayed `reps` times with CUDA events around each replay,
+    and the mean replay time is divided by `calls`. No host launch gap and no
+    flush lands inside the timed region."""
+    import torch
+    for _ in range(calls):  # warm-up: every set once
+        fn()
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            for _ in range(calls):
+                fn()
+    torch.cuda.current_stream().wait_stream(side)
+    graph.replay()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+    for i in range(reps):
+        starts[i].record(stream)
+        graph.replay()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    ms = statistics.fmean(a.elapsed_time(b) for a, b in zip(starts, ends)) / calls
+    del graph
+    return ms
+
+
+class W4a16Rotation:
+    """W4A16 modulation layer (NVFP4 weight quantized on the GPU, bf16 activations)
+    in R copies whose weights together hold at least four times the L2."""
+
+    def __init__(self, M, K, N, device, seed=0, min_bytes=ROTATION_BYTES):
+        import torch
+        import fp8_rowwise_quantized_b200 as q
+        from synthetic import make_linear_inputs
+        inp = make_linear_inputs(M, K, N, seed=seed, with_bias=True)
+        self.q, self.M, self.K, self.N = q, M, K, N
+        x = inp.x.to(device)
+        wq, ws, self.gw = q.prepare_nvfp4_weight(inp.w.to(device))
+        bias = inp.bias.to(device)
+        per = wq.numel() + ws.numel() + x.numel() * 2 + M * N * 2 + N * 4
+        self.R = max(2, -(-min_bytes // per))
+        self.sets = [(x.clone(), wq.clone(), ws.clone(), bias.clone(),
+                      torch.empty((M, N), dtype=torch.bfloat16, device=device))
+                     for _ in range(self.R)]
+        self.i = 0
+
+    def step(self):
+        x, wq, ws, b, y = self.sets[self.i]
+        self.i = (self.i + 1) % self.R
+        self.q.w4a16_linear(x, wq, ws, self.gw, bias=b, y=y)
+
+
+def w4a16_bytes(M, K, N):
+    """Algorithmic bytes of one W4A16 call: weight codes and scales, x, bias, y."""
+    return N * K // 2 + N * K // 16 + 2 * M * K + 4 * N + 2 * M * N
+
+
+def w4a16_sweep(device, stream, peaks, steps):
+    """Modulation projections of a diffusion transformer (hidden 3072): the
+    six-way adaptive-norm modulation (N = 6 x 3072) and the three-way one of the
+    single-stream blocks (N = 3 x 3072), for batches of 1, 2 and 4 conditioning
+    vectors; graph-replayed over rotating weight copies (cold L2 every call)."""
+    import torch
+    hbm = peaks["hbm_gbs"]
+    out = {}
+    for N in (18432, 9216):
+        for M in (1, 2, 4):
+            K = 3072
+            L = W4a16Rotation(M, K, N, device)
+            reps = max(3, min(steps // L.R, 20))
+            ms = time_graph_rotation(L.step, L.R, reps, stream)
+            b = w4a16_bytes(M, K, N)
+            out[f"M{M}_K{K}_N{N}"] = {"us": ms * 1e3, "gbs": b / (ms / 1e3) / 1e9,
+                                      "hbm_frac": b / (ms / 1e3) / 1e9 / hbm,
+                                      "alg_bytes": b, "rotation_sets": L.R}
+            del L
+            torch.cuda.empty_cache()
+    return out
+
+
+# Skinny / batched sweep of the NVFP4 layer (K = 3072): M from a few text tokens
+# to four 4096-token latents, N of the attention projection and the MLP up projection.
+SKINNY_M = (16, 256, 1024, 8192, 16384)
+SKINNY_N = (3072, 12288)
+
+
+def nvfp4_gemm_alg_bytes(M, K, N):
+    """Algorithmic bytes of the GEMM kernel alone: activation codes and scales,
+    weight codes and scales in, bf16 Y out."""
+    return M * K // 2 + M * K // 16 + N * K // 2 + N * K // 16 + 2 * M * N
+
+
+def skinny_sweep(device, stream, peaks, steps):
+    """Per shape: the nvfp4_linear step and its GEMM alone, timed over rotating
+    buffer sets, against the roofline max(FLOPs / FP4 peak, bytes / HBM peak)."""
+    import torch
+    fp4_peak = peaks["bf16_tflops"] * NOMINAL_FP4_OVER_BF16
+    hbm = peaks["hbm_gbs"]
+    out = {}
+    for N in SKINNY_N:
+        for M in SKINNY_M:
+            K = 3072
+            L = Nvfp4Layer(M, K, N, False, device)
+            rot = Nvfp4Rotation(L)
+            reps = max(3, min(steps // rot.R, 20))
+            st_ms = time_graph_rotation(rot.step, rot.R, reps, stream)
+            rot.prologue_all()
+            g_ms = time_graph_rotation(rot.gemm, rot.R, reps, stream)
+            fl = nvfp4_flops(M, K, N)
+            b_step = nvfp4_alg_bytes(M, K, N)
+            b_gemm = nvfp4_gemm_alg_bytes(M, K, N)
+            t_fl = fl / (fp4_peak * 1e12)
+            t_gemm_b = b_gemm / (hbm * 1e9)
+            t_step_b = b_step / (hbm * 1e9)
+            bn, cg = L.q.tile_config(M, N, K)
+            out[f"M{M}_N{N}"] = {
+                "step_us": st_ms * 1e3, "step_tflops": fl / (st_ms / 1e3) / 1e12,
+                "step_gbs": b_step / (st_ms / 1e3) / 1e9,
+                "step_roofline_frac": max(t_fl, t_step_b) / (st_ms / 1e3),
+                "gemm_us": g_ms * 1e3, "gemm_tflops": fl / (g_ms / 1e3) / 1e12,
+                "gemm_gbs": b_gemm / (g_ms / 1e3) / 1e9,
+                "gemm_bound": "hbm" if t_gemm_b > t_fl else "tensor",
+                "gemm_roofline_frac": max(t_fl, t_gemm_b) / (g_ms / 1e3),
+                "tile": f"{128 * cg}x{bn}", "rotation_sets": rot.R,
+            }
+            del rot, L
+            torch.cuda.empty_cache()
+    return out
+
+
 def traffic_from_profiles(kernel_key: str):
     """Per-launch DRAM bytes of a kernel from the committed ncu summary, or None
     when the kernel source changed since the capture."""
@@ -460,6 +655,13 @@ def run_ours(args):
     value = value_flops / 1e12
     status = q.read_device_status()
 
+    # the same step with inputs larger than L2 instead of a flush: consecutive
+    # steps cycle through buffer sets four times the L2, replayed from a CUDA graph
+    # (device time only, no host launch gaps)
+    rot = Nvfp4Rotation(layer)
+    rot_ms = time_graph_rotation(rot.step, rot.R, max(3, min(args.steps // rot.R, 50)), stream)
+    rot_ms, rot_val = aggregate(rot_ms, flops, world, device)
+
     # --------------------------------------------------- roofline of the GEMM kernel
     fp4_peak = peaks["bf16_tflops"] * NOMINAL_FP4_OVER_BF16
     tile_bn, tile_cg = q.tile_config(M, N, K)
@@ -482,12 +684,14 @@ def run_ours(args):
         "traffic": traffic_from_profiles("nvfp4_gemm_mlp_up"),
         "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {NOMINAL_FP4_OVER_BF16} "
                        "(nominal dense FP4:bf16 ratio)",
+        "algorithmic": "2*M*K*N flops per launch",
         "gemm_us": gemm_ms * 1e3,
         "prologue_us": prol_ms * 1e3,
         "prologue_gbs": prologue_bytes / (prol_ms / 1e3) / 1e9,
         "prologue_hbm_frac": prologue_bytes / (prol_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
         "quantize_act_us": quant_ms * 1e3,
         "quantize_act_gbs": quant_bytes / (quant_ms / 1e3) / 1e9,
+        "quantize_act_hbm_frac": quant_bytes / (quant_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
         "frac_of_nominal_9pf": gemm_tflops / 9000.0,
         "step_frac_of_fp4_peak": value / world / fp4_peak,
     }
@@ -562,6 +766,9 @@ def run_ours(args):
             sweep[f"bn{bn}_cg{cg}"] = {"gemm_us": gms * 1e3,
                                       "gemm_tflops": flops / (gms / 1e3) / 1e12}
         variants["mlp_up_gemm_tile_sweep"] = sweep
+        torch.cuda.empty_cache()
+        variants["nvfp4_skinny_sweep_K3072"] = skinny_sweep(device, stream, peaks, v_steps)
+        variants["w4a16_modulation_sweep"] = w4a16_sweep(device, stream, peaks, v_steps)
 
     # --------------------------------------------------- CPU oracle baseline (rank 0, N=1)
     cpu = None
@@ -579,6 +786,10 @@ def run_ours(args):
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "flushed (256 MB write) before every step, outside the events"},
         "frac_of_fp4_peak": value / world / fp4_peak,
+        "l2_rotating_graph": {"value": rot_val / 1e12, "ms_per_step": rot_ms,
+                              "how": f"{rot.R} buffer sets of {rot.bytes_per_set / 1e6:.0f} MB (x, "
+                                     "weights, y, workspace) cycled, one per step, all steps of a "
+                                     "cycle in one CUDA graph; mean over replays"},
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
@@ -600,7 +811,9 @@ def run_profile(args):
     of one piece of the headline workload (no flushes, no timing): `step`,
     `prologue`, `gemm`, `quant` (activation quantization alone), `mlp_fused` (the MLP
     block with the GELU-quantize epilogue), `svdq` (the rank-32 svdq layer), `fp8r_step`,
-    `fp8r_quant` or `fp8r_gemm`."""
+    `fp8r_quant`, `fp8r_gemm`, `w4a16` (the 1 x 3072 x 18432 modulation layer over
+    rotating weight copies) or `skinny_<M>_<N>` (nvfp4_linear at K = 3072 over
+    rotating copies)."""
     import torch
     torch.cuda.set_device(0)
     device = torch.device("cuda", 0)
@@ -611,6 +824,14 @@ def run_profile(args):
     elif args.profile == "svdq":
         sv = SvdqLayer(4096, 3072, 12288, 32, device)
         fn = sv.step
+    elif args.profile == "w4a16":
+        W = W4a16Rotation(1, 3072, 18432, device)
+        fn = W.step
+    elif args.profile.startswith("skinny"):
+        # skinny_<M>_<N>: the nvfp4_linear step at K = 3072 over rotating copies
+        _, Ms, Ns = args.profile.split("_")
+        rot = Nvfp4Rotation(Nvfp4Layer(int(Ms), 3072, int(Ns), False, device))
+        fn = rot.step
     elif args.profile.startswith("fp8r"):
         L = Fp8rLayer(4096, 3072, 3072, False, device)
         fn = {"fp8r_step": L.step, "fp8r_gemm": L.gemm,
@@ -641,8 +862,9 @@ def main():
     ap.add_argument("--no-variants", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", choices=["step", "prologue", "gemm", "quant", "mlp_fused", "svdq",
-                                          "fp8r_step",
-                                          "fp8r_quant", "fp8r_gemm"], default=None,
+                                          "fp8r_step", "fp8r_quant", "fp8r_gemm", "w4a16",
+                                          "skinny_16_3072", "skinny_16_12288",
+                                          "skinny_256_12288"], default=None,
                     help="run a short fixed sequence for a profiler instead of the benchmark")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps

@@ -22,6 +22,7 @@ __all__ = [
     "nvfp4_quantize_act", "nvfp4_linear", "nvfp4_linear_single_launch", "nvfp4_linear_noalloc",
     "nvfp4_linear_prologue", "nvfp4_linear_gelu_quantize", "nvfp4_linear_quantized_input",
     "nvfp4_linear_gemm_lowrank", "svdq_nvfp4_linear", "svdq_nvfp4_linear_workspace_size",
+    "w4a16_linear",
     "nvfp4_linear_gemm",
     "nvfp4_linear_workspace_size", "nvfp4_linear_workspace_layout", "nvfp4_global_scale",
     "fp8r_quantize_rows", "fp8r_linear", "fp8r_linear_gemm", "fp8r_linear_workspace_size",
@@ -269,6 +270,32 @@ def svdq_nvfp4_linear(x: torch.Tensor, w: torch.Tensor, w_scale: torch.Tensor,
     _lib.check("svdq_nvfp4_linear", _lib.load().svdq_nvfp4_linear(
         _ptr(x), M, K, _ptr(smooth), _ptr(lora_down), _ptr(lora_up), r, _ptr(w), _ptr(w_scale),
         N, _ptr(weight_scale_2), _ptr(input_scale), _ptr(bias), _ptr(y), _ptr(ws), ws.numel(),
+        _stream()))
+    return y
+
+
+def w4a16_linear(x: torch.Tensor, w: torch.Tensor, w_scale: torch.Tensor,
+                 weight_scale_2: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                 y: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Y = bf16(x @ what^T + bias) with what = bf16(fp32(E2M1(w) * E4M3(w_scale) *
+    weight_scale_2)): 4-bit weights, bf16 activations (modulation layers).
+
+    x bf16 [M, K]; w uint8 [N, K/2]; w_scale uint8 [N, K/16]; weight_scale_2 fp32
+    scalar; bias fp32 [N] or None."""
+    _need(x, "x", torch.bfloat16, 2)
+    _need(w, "w", torch.uint8, 2)
+    _need(w_scale, "w_scale", torch.uint8, 2)
+    _scalar(weight_scale_2, "weight_scale_2")
+    M, K = x.shape
+    N = w.shape[0]
+    if w.shape[1] * 2 != K or tuple(w_scale.shape) != (N, K // 16):
+        raise ValueError("weight shapes do not match x")
+    if bias is not None:
+        _need(bias, "bias", torch.float32, 1)
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _lib.check("w4a16_linear", _lib.load().w4a16_linear(
+        _ptr(x), M, K, _ptr(w), _ptr(w_scale), N, _ptr(weight_scale_2), _ptr(bias), _ptr(y),
         _stream()))
     return y
 

@@ -39,6 +39,7 @@ SIGNATURES = {
     "svdq_nvfp4_linear_workspace_size": (C.c_size_t, [_i64, _i64, _i64, _i64]),
     "svdq_nvfp4_linear": (C.c_int, [_vp, _i64, _i64, _f32p, _vp, _vp, _i64, _u8p, _u8p, _i64,
                                     _f32p, _f32p, _f32p, _vp, _vp, _sz, _vp]),
+    "w4a16_linear": (C.c_int, [_vp, _i64, _i64, _u8p, _u8p, _i64, _f32p, _f32p, _vp, _vp]),
     "nvfp4_linear_prologue": (C.c_int, [_vp, _i64, _i64, _u8p, _i64, _f32p, _vp, _sz, _vp]),
     "nvfp4_linear_gemm": (C.c_int, [_i64, _i64, _u8p, _i64, _f32p, _f32p, _f32p, _vp, _vp, _sz,
                                     _vp]),

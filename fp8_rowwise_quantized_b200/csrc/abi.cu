@@ -463,6 +463,23 @@ int nvfp4_linear_quantized_input(int64_t M, int64_t K, const uint8_t* w, const u
                          workspace_bytes, stream, true);
 }
 
+int w4a16_linear(const void* x, int64_t M, int64_t K, const uint8_t* w, const uint8_t* w_scale,
+                 int64_t N, const float* weight_scale_2, const float* bias, void* y,
+                 ql_stream_t stream) {
+  if (!x || !w || !w_scale || !weight_scale_2 || !y || M <= 0 || N <= 0 || K <= 0)
+    return QL_ERR_INVALID_ARG;
+  if (!nvfp4_shape_ok(M, K, N)) return fail_shape("w4a16: needs K >= 32 and K % 32 == 0");
+  if (!aligned16(x) || !aligned16(w) || !aligned16(y) ||
+      (reinterpret_cast<uintptr_t>(w_scale) & 1u) != 0 ||
+      (reinterpret_cast<uintptr_t>(bias) & 3u) != 0)
+    return QL_ERR_ALIGN;
+  int rc = check_device(nullptr);
+  if (rc != QL_OK) return rc;
+  cudaError_t e = ql::launch_w4a16_linear(x, M, K, w, w_scale, N, weight_scale_2, bias, y,
+                                          reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QL_OK : record(e, "w4a16_linear");
+}
+
 int nvfp4_global_scale(const void* x, int64_t n, float* out, ql_stream_t stream) {
   if (!x || !out || n <= 0) return QL_ERR_INVALID_ARG;
   int rc = check_device(nullptr);

@@ -107,10 +107,11 @@ int nvfp4_linear_gemm_lowrank(int64_t M, int64_t K, const uint8_t* w, int64_t N,
  *   w, w_scale, weight_scale_2, bias, y  as nvfp4_linear (w: the 4-bit residual)
  *   input_scale  the calibrated global scale of xs
  *   workspace  >= svdq_nvfp4_linear_workspace_size(M, K, N, rank) bytes
- * Three launches: the prologue (smoothing, quantization of xs, weight-scale
- * layout); the low-rank down projection (warp-level bf16 tensor-core MMA) into the
- * workspace; the 4-bit GEMM with the low-rank up projection as one more bf16 K step
- * into the same accumulator (the fusion the page describes for the up projection).
+ * Two launches: a prologue that reads x once (smoothing, quantization of xs, the
+ * low-rank down projection on warp-level bf16 tensor-core MMAs into the workspace,
+ * weight-scale layout: the fusion the page describes for the down projection); the
+ * 4-bit GEMM with the low-rank up projection as one more bf16 K step into the same
+ * accumulator (the fusion the page describes for the up projection).
  * Requires the nvfp4_linear shapes and 16-byte aligned pointers. */
 size_t svdq_nvfp4_linear_workspace_size(int64_t M, int64_t K, int64_t N, int64_t rank);
 int svdq_nvfp4_linear(const void* x, int64_t M, int64_t K, const float* smooth,
@@ -118,6 +119,26 @@ int svdq_nvfp4_linear(const void* x, int64_t M, int64_t K, const float* smooth,
                       const uint8_t* w_scale, int64_t N, const float* weight_scale_2,
                       const float* input_scale, const float* bias, void* y, void* workspace,
                       size_t workspace_bytes, ql_stream_t stream);
+
+/* W4A16 linear: 4-bit weights, 16-bit activations (the awq_w4a16 kernel family of
+ * the Diffusers page "Bringing Nunchaku 4-bit Diffusion Inference to Diffusers",
+ * section "Introducing Nunchaku Lite", used there for the memory-bound adaptive
+ * normalization and modulation projections), with the nvfp4 weight of this
+ * library. The weight is dequantized to the compute dtype and the activations are
+ * not quantized (the unfused path of "BFL (fp8r / nvfp4)", section "Kernels"):
+ *   what[n, k] = bf16( RN32( E2M1(w[n, k]) * E4M3(w_scale[n, k/16]) * weight_scale_2 ) )
+ *   Y[m, n]    = bf16( sum_k x[m, k] * what[n, k] + bias[n] )   (fp32 accumulation)
+ *   x               bf16 [M, K] (a few rows: one per conditioning vector)
+ *   w, w_scale      as nvfp4_linear: uint8 [N, K/2] packed E2M1, uint8 [N, K/16] E4M3
+ *   weight_scale_2  device fp32 scalar
+ *   bias            fp32 [N] or NULL
+ *   y               bf16 [M, N] (output)
+ * One launch, no workspace: a GEMV that streams the weight once per 8 rows of x
+ * (made for M <= 8; larger M works and re-reads the weight, mostly from L2).
+ * Requires K >= 32, K % 32 == 0; x, w, y 16-byte aligned, w_scale 2-byte aligned. */
+int w4a16_linear(const void* x, int64_t M, int64_t K, const uint8_t* w,
+                 const uint8_t* w_scale, int64_t N, const float* weight_scale_2,
+                 const float* bias, void* y, ql_stream_t stream);
 
 /* The MLP up projection with its GELU and the down projection's quantization
  * fused into the GEMM epilogue (the "fused GELU/MLP" kernels of the Diffusers

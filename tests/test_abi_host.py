@@ -77,6 +77,11 @@ def test_argument_errors_before_device():
     assert lib.nvfp4_quantize_act(fake, M, 24, fake, fake, fake, None) == 2
     assert lib.nvfp4_quantize_act(odd, M, K, fake, fake, fake, None) == 3
     assert lib.ql_encode_e4m3(None, fake, 10, None) == 1
+    # w4a16: null weight, K % 32, misaligned x, odd w_scale
+    assert lib.w4a16_linear(fake, 1, K, None, fake, N, fake, None, fake, None) == 1
+    assert lib.w4a16_linear(fake, 1, 48, fake, fake, N, fake, None, fake, None) == 2
+    assert lib.w4a16_linear(odd, 1, K, fake, fake, N, fake, None, fake, None) == 3
+    assert lib.w4a16_linear(fake, 1, K, fake, fake + 1, N, fake, None, fake, None) == 3
 
 
 def test_no_device_reports_error_instead_of_crashing():

@@ -70,6 +70,22 @@ def test_nvfp4_linear_dit_sizes_sampled(name, M, K, N, bias):
     assert np.abs(yb).max() < 1e4 and (yb != 0).mean() > 0.99
 
 
+# Skinny / batched sweep of the layer at K = 3072: a few text tokens up to four
+# 4096-token latents, with the attention-projection and MLP-up widths.
+@pytest.mark.parametrize("M,N", [(16, 3072), (16, 12288), (256, 3072), (256, 12288)])
+def test_nvfp4_linear_skinny_full(M, N):
+    run_nvfp4(Nvfp4Case(M, 3072, N, seed=M + N))
+
+
+@pytest.mark.parametrize("M,N", [(1024, 3072), (1024, 12288), (8192, 3072), (8192, 12288),
+                                 (16384, 3072), (16384, 12288)])
+def test_nvfp4_linear_batched_sampled(M, N):
+    c = Nvfp4Case(M, 3072, N, seed=M + N)
+    y, _ = run_nvfp4(c, sample_rows(M, 16, seed=M))
+    yb = oracle.bf16_bits_to_f64(bf16_bits(y))
+    assert np.abs(yb).max() < 1e4 and (yb != 0).mean() > 0.99
+
+
 def test_nvfp4_mlp_down_from_gelu_of_up():
     # the down projection's input is GELU of the up projection's GPU output,
     # re-quantized at run time with a re-calibrated input scale
