@@ -83,6 +83,10 @@ struct GemmArgs {
   // bf16 operands (tmap_lra: [M, r] activations pre-divided by alpha; tmap_lrb:
   // [N, r]) and lr_k16 = ceil(r / 16) MMAs of K = 16 into the same accumulator
   int lr_k16;
+  // rows of A one CTA loads per K tile: 128, or M rounded up to 8 when a lone CTA's
+  // tile has fewer valid rows (rows past it keep stale shared memory, which only
+  // reaches accumulator rows that are never stored; their scale atoms are zero)
+  int a_box_rows;
 };
 
 template <bool FP4, int BN, int CG>
@@ -646,7 +650,7 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
           const int sfb_atom = static_cast<int>((static_cast<int64_t>(n_blk) * args.kg + kt * 4) *
                                                 C::NA);
 
-          constexpr uint32_t kTx = C::STAGE_BYTES;
+          const uint32_t kTx = C::STAGE_BYTES - C::A_BYTES + args.a_box_rows * 128;
           if constexpr (CG == 2) {
             if (leader) mbar_arrive_expect_tx(&full_bar[stage], CG * kTx);
             tma_load_2d_pair(sa, &tmap_a, fb, kt * 128, a_row);
@@ -1098,9 +1102,15 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
   std::memset(&tsa, 0, sizeof(tsa));
   std::memset(&tsb, 0, sizeof(tsb));
   std::memset(&ty, 0, sizeof(ty));
-  // A / B: uint8 rows of K* bytes, boxes of [rows, 128 bytes], 128-byte swizzle
-  if (!encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.a, k_bytes, p.M, k_bytes, 128, kRowsPerCta,
-                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
+  // A / B: uint8 rows of K* bytes, boxes of [rows, 128 bytes], 128-byte swizzle; a
+  // lone CTA with fewer than 128 rows of A loads only those (whole 8-row swizzle
+  // atoms), the plain FP4 mode only (its A scale atoms zero the rows past M)
+  const int a_box_rows = (CG == 1 && FP4 && MODE == kModePlain && p.M < kRowsPerCta)
+                             ? static_cast<int>((p.M + 7) / 8 * 8)
+                             : kRowsPerCta;
+  if (!encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.a, k_bytes, p.M, k_bytes, 128,
+                 static_cast<uint32_t>(a_box_rows), CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
       !encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.b, k_bytes, p.N, k_bytes, 128, Cf::B_ROWS,
                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
     return cudaErrorInvalidValue;
@@ -1140,6 +1150,7 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
   }
 
   GemmArgs a{};
+  a.a_box_rows = a_box_rows;
   a.lr_k16 = lowrank ? (p.lr_rank + 15) / 16 : 0;
   a.M = static_cast<int>(p.M);
   a.N = static_cast<int>(p.N);
