@@ -109,16 +109,18 @@ __device__ __forceinline__ uint2 nvfp4_block16(const uint4 u, const uint4 v, flo
 constexpr int kWsGroups = 16;
 using WsTile = uint32_t[128][kWsGroups + 1];
 
-__device__ __forceinline__ void weight_scale_atoms_load(int64_t job, int tid,
-                                                        const uint8_t* __restrict__ ws, int64_t N,
-                                                        int64_t K, int bn, int na, int64_t KG,
-                                                        WsTile& tile) {
+// The 8 words of weight_scale_atoms_load held in registers (word j of row tid / 2,
+// group 8 * (tid % 2) + j), so that the loads can be issued long before the words
+// are written to shared memory.
+__device__ __forceinline__ void weight_scale_words(int64_t job, int tid,
+                                                   const uint8_t* __restrict__ ws, int64_t N,
+                                                   int64_t K, int bn, int na, int64_t KG,
+                                                   uint32_t (&words)[8]) {
   const int64_t kg_chunks = ceil_div64(KG, kWsGroups);
   const int64_t kc = job % kg_chunks;
   const int a = static_cast<int>((job / kg_chunks) % na);
   const int64_t t = job / (kg_chunks * na);
   const int64_t nblk = K / 16;
-  // thread -> (row = tid / 2, groups 8 * (tid % 2) .. +8)
   const int rr = tid / 2;
   const int g0 = (tid % 2) * 8;
   const int64_t nn = static_cast<int64_t>(a) * 128 + rr;
@@ -137,8 +139,23 @@ __device__ __forceinline__ void weight_scale_atoms_load(int64_t job, int tid,
           if (4 * kg + b < nblk) word |= static_cast<uint32_t>(__ldg(src + b)) << (8 * b);
       }
     }
-    tile[rr][g0 + j] = word;
+    words[j] = word;
   }
+}
+
+__device__ __forceinline__ void weight_scale_words_to_tile(int tid, const uint32_t (&words)[8],
+                                                           WsTile& tile) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) tile[tid / 2][(tid % 2) * 8 + j] = words[j];
+}
+
+__device__ __forceinline__ void weight_scale_atoms_load(int64_t job, int tid,
+                                                        const uint8_t* __restrict__ ws, int64_t N,
+                                                        int64_t K, int bn, int na, int64_t KG,
+                                                        WsTile& tile) {
+  uint32_t words[8];
+  weight_scale_words(job, tid, ws, N, K, bn, na, KG, words);
+  weight_scale_words_to_tile(tid, words, tile);
 }
 
 // One 512-byte atom = 128 words per group; thread tid writes word tid % 128 of the

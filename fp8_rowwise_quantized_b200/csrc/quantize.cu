@@ -157,12 +157,23 @@ nvfp4_prologue_kernel(const uint16_t* __restrict__ x, int M, int K,
                       const uint8_t* __restrict__ ws, int64_t N, int bn, int na, int64_t n_tiles,
                       int64_t w_jobs, uint8_t* __restrict__ wout) {
   __shared__ WsTile tile;
+  // the block's first weight-scale job: its loads are in flight during the activation
+  // items, so their latency is off the block's critical path
+  uint32_t first[8];
+  const bool has_job = blockIdx.x < w_jobs;
+  if (has_job) weight_scale_words(blockIdx.x, threadIdx.x, ws, N, K, bn, na, KG, first);
   const float g = __ldg(g_ptr);
   const float c = __frcp_rn(__fmul_rn(6.0f, g));
   constexpr uint32_t kWarps = kQuantThreads / 32;
   nvfp4_quantize_items<true>(blockIdx.x * kWarps + threadIdx.x / 32, gridDim.x * kWarps,
                              threadIdx.x % 32, x, M, K, g, c, xq, xs, rows_total * segs, segs, KG);
-  for (int64_t job = blockIdx.x; job < w_jobs; job += gridDim.x) {
+  if (has_job) {
+    weight_scale_words_to_tile(threadIdx.x, first, tile);
+    __syncthreads();
+    weight_scale_atoms_store(blockIdx.x, threadIdx.x, na, KG, wout, tile);
+    __syncthreads();
+  }
+  for (int64_t job = blockIdx.x + gridDim.x; job < w_jobs; job += gridDim.x) {
     weight_scale_atoms_load(job, threadIdx.x, ws, N, K, bn, na, KG, tile);
     __syncthreads();
     weight_scale_atoms_store(job, threadIdx.x, na, KG, wout, tile);
