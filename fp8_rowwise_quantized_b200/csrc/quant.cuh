@@ -100,6 +100,31 @@ __device__ __forceinline__ uint2 nvfp4_block16(const uint4 u, const uint4 v, flo
   return make_uint2(zero ? 0u : lo, zero ? 0u : hi);
 }
 
+// The same block rule with the per-block reciprocal read from a table: inv_of[s] =
+// RN32(1 / RN32(value(s) * g)) for the 128 non-negative scale codes s (0 where
+// value(s) * g == 0), computed once per CTA with the same operations, so the codes
+// are the same bits as nvfp4_block16's.
+__device__ __forceinline__ uint2 nvfp4_block16_tab(const uint4 u, const uint4 v, float c,
+                                                   const float* inv_of, uint32_t& scale_code) {
+  const float amax = bf16x16_amax(u, v);
+  const uint32_t s = cvt_e4m3x2(0.0f, __fmul_rn(amax, c)) & 0x7Fu;  // amax >= 0: sign bit 0
+  scale_code = s;
+  const float inv = inv_of[s];
+  const uint32_t lo = e2m1x8_of_bf16_scaled(u.x, u.y, u.z, u.w, inv);
+  const uint32_t hi = e2m1x8_of_bf16_scaled(v.x, v.y, v.z, v.w, inv);
+  const bool zero = inv == 0.0f;
+  return make_uint2(zero ? 0u : lo, zero ? 0u : hi);
+}
+
+// Fills inv_of[0..127] for global scale g (threads 0..127 of the block, one entry
+// each); the caller synchronises the block before use.
+__device__ __forceinline__ void fill_block_reciprocals(float* inv_of, float g, int tid) {
+  if (tid < 128) {
+    const float d = __fmul_rn(e4m3_to_float(static_cast<uint32_t>(tid)), g);
+    inv_of[tid] = d != 0.0f ? __frcp_rn(d) : 0.0f;
+  }
+}
+
 // Row-major weight scales [N, K/16] -> atom layout for tiles of `bn` rows, through
 // shared memory so that both the reads (64 contiguous bytes per row) and the
 // writes (whole 512-byte atoms) are coalesced. One job = (tile, 128-row atom a,

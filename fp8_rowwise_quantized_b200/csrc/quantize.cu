@@ -58,7 +58,7 @@ __device__ __forceinline__ void nvfp4_load_item(int r, int seg, int lane,
 
 template <bool SF_MMA>
 __device__ __forceinline__ void nvfp4_encode_item(int r, int seg, int lane, const QuantItem& qin,
-                                                  int M, int K, float g, float c,
+                                                  int M, int K, const float* inv_of, float c,
                                                   uint8_t* __restrict__ xq,
                                                   uint8_t* __restrict__ xs, int KG) {
   const int nblk = K >> 4;
@@ -69,7 +69,7 @@ __device__ __forceinline__ void nvfp4_encode_item(int r, int seg, int lane, cons
     const bool valid = (r < M) && (e < K);
     const uint4 u = qin.raw[2 * i], v = qin.raw[2 * i + 1];
     uint32_t s;
-    const uint2 codes = nvfp4_block16(u, v, g, c, s);
+    const uint2 codes = nvfp4_block16_tab(u, v, c, inv_of, s);
     if (valid) *reinterpret_cast<uint2*>(qr + (e >> 1)) = codes;
     // gather the scales of blocks lane .. lane+3 into lanes 0, 4, ..., 28
     const uint32_t s1 = __shfl_down_sync(0xffffffffu, s, 1);
@@ -104,7 +104,8 @@ __device__ __forceinline__ void nvfp4_encode_item(int r, int seg, int lane, cons
 template <bool SF_MMA>
 __device__ __forceinline__ void nvfp4_quantize_items(uint32_t warp_id, uint32_t nwarps, int lane,
                                                      const uint16_t* __restrict__ x, int M, int K,
-                                                     float g, float c, uint8_t* __restrict__ xq,
+                                                     const float* inv_of, float c,
+                                                     uint8_t* __restrict__ xq,
                                                      uint8_t* __restrict__ xs, uint32_t total,
                                                      uint32_t segs, int KG) {
   if (warp_id >= total) return;  // warp-uniform
@@ -122,8 +123,8 @@ __device__ __forceinline__ void nvfp4_quantize_items(uint32_t warp_id, uint32_t 
     QuantItem nxt;
     if (item + nwarps < total)
       nvfp4_load_item(static_cast<int>(rn), static_cast<int>(sn), lane, x, M, K, nxt);
-    nvfp4_encode_item<SF_MMA>(static_cast<int>(r), static_cast<int>(seg), lane, cur, M, K, g, c,
-                              xq, xs, KG);
+    nvfp4_encode_item<SF_MMA>(static_cast<int>(r), static_cast<int>(seg), lane, cur, M, K,
+                              inv_of, c, xq, xs, KG);
     cur = nxt;
     r = rn;
     seg = sn;
@@ -135,12 +136,15 @@ __global__ void __launch_bounds__(kQuantThreads)
 nvfp4_quantize_kernel(const uint16_t* __restrict__ x, int M, int K,
                       const float* __restrict__ g_ptr, uint8_t* __restrict__ xq,
                       uint8_t* __restrict__ xs, uint32_t rows_total, uint32_t segs, int KG) {
+  __shared__ float inv_of[128];
   const float g = __ldg(g_ptr);
   const float c = __frcp_rn(__fmul_rn(6.0f, g));
+  fill_block_reciprocals(inv_of, g, threadIdx.x);
+  __syncthreads();
   constexpr uint32_t kWarps = kQuantThreads / 32;
   nvfp4_quantize_items<SF_MMA>(blockIdx.x * kWarps + threadIdx.x / 32, gridDim.x * kWarps,
-                               threadIdx.x % 32, x, M, K, g, c, xq, xs, rows_total * segs, segs,
-                               KG);
+                               threadIdx.x % 32, x, M, K, inv_of, c, xq, xs, rows_total * segs,
+                               segs, KG);
 }
 
 // The prologue of nvfp4_linear in one launch, one wave of resident blocks: each
@@ -162,11 +166,15 @@ nvfp4_prologue_kernel(const uint16_t* __restrict__ x, int M, int K,
   uint32_t first[8];
   const bool has_job = blockIdx.x < w_jobs;
   if (has_job) weight_scale_words(blockIdx.x, threadIdx.x, ws, N, K, bn, na, KG, first);
+  __shared__ float inv_of[128];
   const float g = __ldg(g_ptr);
   const float c = __frcp_rn(__fmul_rn(6.0f, g));
+  fill_block_reciprocals(inv_of, g, threadIdx.x);
+  __syncthreads();
   constexpr uint32_t kWarps = kQuantThreads / 32;
   nvfp4_quantize_items<true>(blockIdx.x * kWarps + threadIdx.x / 32, gridDim.x * kWarps,
-                             threadIdx.x % 32, x, M, K, g, c, xq, xs, rows_total * segs, segs, KG);
+                             threadIdx.x % 32, x, M, K, inv_of, c, xq, xs, rows_total * segs, segs,
+                             KG);
   if (has_job) {
     weight_scale_words_to_tile(threadIdx.x, first, tile);
     __syncthreads();
