@@ -13,8 +13,11 @@ the time is the max over ranks.
 
 Prints one JSON line (rank 0). Extra keys: roofline of the GEMM kernel,
 cpu_baseline (the CPU oracle on a bounded sample), e2e (host buffers, copies
-inside the timed region), clocks sampled during the timed region, and the other
-layer shapes under "variants".
+inside the timed region), clocks sampled during the timed region,
+l2_rotating_graph (the same step timed over buffer sets four times the L2, replayed
+from a CUDA graph), and under "variants" the other layer shapes (flushed L2), the
+skinny / batched NVFP4 sweep and the W4A16 modulation sweep (both rotating-graph
+timed, against the HBM and FP4 rooflines).
 """
 import argparse
 import hashlib
