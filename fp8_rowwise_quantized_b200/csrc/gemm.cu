@@ -367,21 +367,35 @@ __device__ __forceinline__ void gelu_quant_slab(const GemmArgs& a, const uint32_
   uint32_t codes[SLAB / 8];
 #pragma unroll
   for (int b = 0; b < SLAB / 16; ++b) {
-    float h[16];
-    float amax = 0.0f;
+    float h[16], v[16];
     float bias[16];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
       *reinterpret_cast<float4*>(&bias[4 * i]) =
           *reinterpret_cast<const float4*>(cv_bias_slab + 16 * b + 4 * i);
+    // fast path: every element's GELU from the table (index clamped into it), with
+    // a flag for elements outside the table's range
+    bool outside = false;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const int j = 16 * b + i;
-      const float v =
+      v[i] =
           __bfloat162float(__float2bfloat16_rn(__fmaf_rn(__uint_as_float(r[j]), alpha, bias[i])));
-      h[i] = gelu_bf16(v, gelu_tab);
-      amax = fmaxf(amax, fabsf(h[i]));
+      const uint32_t bits = __float_as_uint(v[i]) >> 16;
+      const uint32_t mag = (bits & 0x7FFFu) - (static_cast<uint32_t>(kGeluTabExpLo) << 7);
+      outside |= mag >= static_cast<uint32_t>(kGeluTabExps * 128);
+      const uint32_t idx = min(mag, static_cast<uint32_t>(kGeluTabExps * 128 - 1)) +
+                           (bits >> 15) * static_cast<uint32_t>(kGeluTabExps * 128);
+      h[i] = __uint_as_float(static_cast<uint32_t>(gelu_tab[idx]) << 16);
     }
+    // rare (|v| < 2^-16 or >= 64 somewhere in the block): the exact rule for all 16
+    if (outside) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) h[i] = gelu_bf16(v[i], gelu_tab);
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(h[i]));
     const uint32_t s = cvt_e4m3x4(__fmul_rn(amax, cinv), 0.0f, 0.0f, 0.0f) & 0x7Fu;
     const float inv = inv_of[s];
     float f0[8], f1[8];
