@@ -367,21 +367,37 @@ __device__ __forceinline__ void gelu_quant_slab(const GemmArgs& a, const uint32_
   uint32_t codes[SLAB / 8];
 #pragma unroll
   for (int b = 0; b < SLAB / 16; ++b) {
-    float h[16], v[16];
+    float h[16];
     float bias[16];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
       *reinterpret_cast<float4*>(&bias[4 * i]) =
           *reinterpret_cast<const float4*>(cv_bias_slab + 16 * b + 4 * i);
+    // v = bf16(alpha * acc + bias), two elements per packed fma and conversion
+    uint32_t vb[16];  // bf16 bits of v
+#pragma unroll
+    for (int p2 = 0; p2 < 8; ++p2) {
+      const int j = 16 * b + 2 * p2;
+      uint32_t pair;
+      asm("{\n\t.reg .b64 a, s, c;\n\t.reg .b32 lo, hi;\n\t"
+          "mov.b64 a, {%1, %2};\n\t"
+          "mov.b64 s, {%3, %3};\n\t"
+          "mov.b64 c, {%4, %5};\n\t"
+          "fma.rn.f32x2 a, a, s, c;\n\t"
+          "mov.b64 {lo, hi}, a;\n\t"
+          "cvt.rn.bf16x2.f32 %0, hi, lo;\n\t}"
+          : "=r"(pair)
+          : "f"(__uint_as_float(r[j])), "f"(__uint_as_float(r[j + 1])), "f"(alpha),
+            "f"(bias[2 * p2]), "f"(bias[2 * p2 + 1]));
+      vb[2 * p2] = pair & 0xFFFFu;
+      vb[2 * p2 + 1] = pair >> 16;
+    }
     // fast path: every element's GELU from the table (index clamped into it), with
     // a flag for elements outside the table's range
     bool outside = false;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const int j = 16 * b + i;
-      v[i] =
-          __bfloat162float(__float2bfloat16_rn(__fmaf_rn(__uint_as_float(r[j]), alpha, bias[i])));
-      const uint32_t bits = __float_as_uint(v[i]) >> 16;
+      const uint32_t bits = vb[i];
       const uint32_t mag = (bits & 0x7FFFu) - (static_cast<uint32_t>(kGeluTabExpLo) << 7);
       outside |= mag >= static_cast<uint32_t>(kGeluTabExps * 128);
       const uint32_t idx = min(mag, static_cast<uint32_t>(kGeluTabExps * 128 - 1)) +
@@ -391,7 +407,7 @@ __device__ __forceinline__ void gelu_quant_slab(const GemmArgs& a, const uint32_
     // rare (|v| < 2^-16 or >= 64 somewhere in the block): the exact rule for all 16
     if (outside) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) h[i] = gelu_bf16(v[i], gelu_tab);
+      for (int i = 0; i < 16; ++i) h[i] = gelu_bf16(__uint_as_float(vb[i] << 16), gelu_tab);
     }
     float amax = 0.0f;
 #pragma unroll
@@ -400,9 +416,21 @@ __device__ __forceinline__ void gelu_quant_slab(const GemmArgs& a, const uint32_
     const float inv = inv_of[s];
     float f0[8], f1[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      f0[i] = __fmul_rn(h[i], inv);
-      f1[i] = __fmul_rn(h[8 + i], inv);
+    for (int i = 0; i < 8; i += 2) {  // RN products, two lanes per packed multiply
+      asm("{\n\t.reg .b64 a, s;\n\t"
+          "mov.b64 s, {%4, %4};\n\t"
+          "mov.b64 a, {%2, %3};\n\t"
+          "mul.rn.f32x2 a, a, s;\n\t"
+          "mov.b64 {%0, %1}, a;\n\t}"
+          : "=f"(f0[i]), "=f"(f0[i + 1])
+          : "f"(h[i]), "f"(h[i + 1]), "f"(inv));
+      asm("{\n\t.reg .b64 a, s;\n\t"
+          "mov.b64 s, {%4, %4};\n\t"
+          "mov.b64 a, {%2, %3};\n\t"
+          "mul.rn.f32x2 a, a, s;\n\t"
+          "mov.b64 {%0, %1}, a;\n\t}"
+          : "=f"(f1[i]), "=f"(f1[i + 1])
+          : "f"(h[8 + i]), "f"(h[8 + i + 1]), "f"(inv));
     }
     codes[2 * b] = inv != 0.0f ? cvt_e2m1x8(f0) : 0u;
     codes[2 * b + 1] = inv != 0.0f ? cvt_e2m1x8(f1) : 0u;
