@@ -378,19 +378,20 @@ __device__ __forceinline__ void gelu_quant_slab(const GemmArgs& a, const uint32_
 #pragma unroll
     for (int p2 = 0; p2 < 8; ++p2) {
       const int j = 16 * b + 2 * p2;
-      uint32_t pair;
-      asm("{\n\t.reg .b64 a, s, c;\n\t.reg .b32 lo, hi;\n\t"
-          "mov.b64 a, {%1, %2};\n\t"
-          "mov.b64 s, {%3, %3};\n\t"
-          "mov.b64 c, {%4, %5};\n\t"
+      uint32_t o0, o1;
+      asm("{\n\t.reg .b64 a, s, c;\n\t"
+          "mov.b64 a, {%2, %3};\n\t"
+          "mov.b64 s, {%4, %4};\n\t"
+          "mov.b64 c, {%5, %6};\n\t"
           "fma.rn.f32x2 a, a, s, c;\n\t"
-          "mov.b64 {lo, hi}, a;\n\t"
-          "cvt.rn.bf16x2.f32 %0, hi, lo;\n\t}"
-          : "=r"(pair)
+          "mov.b64 {%0, %1}, a;\n\t}"
+          : "=r"(o0), "=r"(o1)
           : "f"(__uint_as_float(r[j])), "f"(__uint_as_float(r[j + 1])), "f"(alpha),
             "f"(bias[2 * p2]), "f"(bias[2 * p2 + 1]));
-      vb[2 * p2] = pair & 0xFFFFu;
-      vb[2 * p2 + 1] = pair >> 16;
+      // RN-even to bf16 in integer arithmetic (finite values): the conversion pipe is
+      // the epilogue's bottleneck, the integer pipe has room
+      vb[2 * p2] = (o0 + 0x7FFFu + ((o0 >> 16) & 1u)) >> 16;
+      vb[2 * p2 + 1] = (o1 + 0x7FFFu + ((o1 >> 16) & 1u)) >> 16;
     }
     // fast path: every element's GELU from the table (index clamped into it), with
     // a flag for elements outside the table's range
