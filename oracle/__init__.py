@@ -73,6 +73,11 @@ def lib():
         L.oracle_w4a16_linear.argtypes = [u16p, i64, i64, u8p, u8p, i64, C.c_float, f32p, u16p,
                                           f64p, f64p]
         L.oracle_w4a16_linear.restype = C.c_int
+        L.oracle_int4_quantize.argtypes = [u16p, i64, i64, u8p, f32p]
+        L.oracle_int4_quantize.restype = C.c_int
+        L.oracle_int4_linear.argtypes = [u8p, f32p, i64, i64, u8p, f32p, i64, f32p, u16p, f64p,
+                                         f64p]
+        L.oracle_int4_linear.restype = C.c_int
         _lib = L
     return _lib
 
@@ -356,3 +361,37 @@ def bf16_ulp(v) -> np.ndarray:
 def bf16_bits_to_f64(bits) -> np.ndarray:
     b = np.ascontiguousarray(bits, np.uint16).astype(np.uint32) << 16
     return b.view(np.float32).astype(np.float64)
+
+
+def int4_quantize(x):
+    """bf16 [R, K] -> (INT4 codes uint8 [R, K/2], element 2j in the low nibble, two's
+    complement; fp32 group scales [R, K/64]). K % 64 == 0."""
+    xb = _bits16(x)
+    R, K = xb.shape
+    q = np.empty((R, K // 2), np.uint8)
+    s = np.empty((R, K // 64), np.float32)
+    rc = lib().oracle_int4_quantize(_p(xb, C.c_uint16), R, K, _p(q, C.c_uint8), _p(s, C.c_float))
+    if rc != 0:
+        raise ValueError("oracle_int4_quantize: bad shape")
+    return q, s
+
+
+def int4_linear(xq, xs, wq, ws, bias=None):
+    """INT4 W4A4 linear: returns (y bf16 bits [M, N], y fp64, tolerance scale T)."""
+    xq = np.ascontiguousarray(xq, np.uint8)
+    xs = np.ascontiguousarray(xs, np.float32)
+    wq = np.ascontiguousarray(wq, np.uint8)
+    ws = np.ascontiguousarray(ws, np.float32)
+    M, K = xq.shape[0], xq.shape[1] * 2
+    N = wq.shape[0]
+    assert wq.shape[1] * 2 == K and xs.shape == (M, K // 64) and ws.shape == (N, K // 64)
+    b = None if bias is None else np.ascontiguousarray(bias, np.float32)
+    y = np.empty((M, N), np.uint16)
+    y64 = np.empty((M, N), np.float64)
+    T = np.empty((M, N), np.float64)
+    rc = lib().oracle_int4_linear(_p(xq, C.c_uint8), _p(xs, C.c_float), M, K, _p(wq, C.c_uint8),
+                                  _p(ws, C.c_float), N, _p(b, C.c_float), _p(y, C.c_uint16),
+                                  _p(y64, C.c_double), _p(T, C.c_double))
+    if rc != 0:
+        raise ValueError("oracle_int4_linear: bad shape")
+    return y, y64, T

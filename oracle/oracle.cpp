@@ -14,6 +14,10 @@
 //   * "BFL (fp8r / nvfp4)", section "Kernels", table: the nvfp4 forward quantizes
 //     the activations at run time (nvfp4_quantize) and runs a block-scaled FP4
 //     GEMM (mm_fp4); fp8r runs a GEMM with row-wise scales (_scaled_mm).
+//   * "Bringing Nunchaku 4-bit Diffusion Inference to Diffusers": the SVDQuant-style
+//     layer (smoothing, 16-bit low-rank branch, 4-bit residual), the W4A16 family
+//     (4-bit weights, bf16 activations) and the INT4 variant of the 4-bit layer;
+//     their readings are stated at each function below.
 //   The pages name the element formats but print no bit layout. This file takes the
 //   public OCP definitions of the two formats: E4M3 "FN" (bias 7, no infinity,
 //   S.1111.111 is NaN, largest finite 448) and E2M1 (bias 1, magnitudes
@@ -557,6 +561,96 @@ int oracle_w4a16_linear(const uint16_t* x, int64_t M, int64_t K, const uint8_t* 
   for (int64_t i = 0; i < N * K; ++i) B[i] = (double)bf16_to_float(wb[i]);
   std::vector<double> am((size_t)M, 1.0), an((size_t)N, 1.0);
   contract(A.data(), B.data(), M, K, N, am.data(), an.data(), bias, y, y64, T);
+  return 0;
+}
+
+// ---------------------------------------------------------------------------
+// INT4 W4A4: the INT4 variant of the svdq_w4a4 kernel family ("Bringing Nunchaku
+// 4-bit Diffusion Inference to Diffusers", section "Introducing Nunchaku Lite":
+// 4-bit weights and activations, "available in INT4 and NVFP4 variants"), without
+// the low-rank branch. The page gives no format; the reading: signed 4-bit integer
+// codes in [-8, 7] with one fp32 scale per 64-element group along K, for the
+// activations (quantized at run time) and the weights:
+//   amax  = max over the group of |x|
+//   scale = RN32(amax / 7)                    (the largest magnitude maps to 7)
+//   scale == 0 -> all codes 0
+//   else       -> q = clamp(RNE(RN32(x * RN32(1 / scale))), -8, 7)
+// Codes are packed two per byte, element 2j in bits 3..0 of byte j (two's
+// complement nibbles); scales are row-major [R, K/64].
+// ---------------------------------------------------------------------------
+int oracle_int4_quantize(const uint16_t* x, int64_t R, int64_t K, uint8_t* q, float* scale) {
+  if (R < 0 || K <= 0 || K % 64 != 0) return -1;
+  const int64_t G = K / 64;
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < R; ++r) {
+    for (int64_t g = 0; g < G; ++g) {
+      const uint16_t* xg = x + r * K + g * 64;
+      float amax = 0.0f;
+      for (int i = 0; i < 64; ++i) {
+        const float a = std::fabs(bf16_to_float(xg[i]));
+        if (a > amax) amax = a;
+      }
+      const float sc = amax / 7.0f;  // one fp32 division
+      scale[r * G + g] = sc;
+      const float inv = sc == 0.0f ? 0.0f : 1.0f / sc;
+      uint8_t* qg = q + r * (K / 2) + g * 32;
+      for (int i = 0; i < 64; i += 2) {
+        int c[2] = {0, 0};
+        for (int e = 0; e < 2; ++e) {
+          if (sc == 0.0f) continue;
+          const float t = bf16_to_float(xg[i + e]) * inv;  // one fp32 multiply
+          double rq = std::nearbyint(static_cast<double>(t));  // ties to even
+          if (rq < -8.0) rq = -8.0;
+          if (rq > 7.0) rq = 7.0;
+          c[e] = static_cast<int>(rq);
+        }
+        qg[i / 2] = static_cast<uint8_t>((c[0] & 0xF) | ((c[1] & 0xF) << 4));
+      }
+    }
+  }
+  return 0;
+}
+
+static inline int int4_code(const uint8_t* q, int64_t k) {
+  const int nib = (k % 2 == 0) ? (q[k / 2] & 0xF) : (q[k / 2] >> 4);
+  return nib >= 8 ? nib - 16 : nib;
+}
+
+// INT4 linear:
+//   Y[m, n] = bf16( sum_g xs[m,g] ws[n,g] sum_{k in group g} qx[m,k] qw[n,k] + bias[n] )
+// the integer group sums exact, the scaled sum in fp64 in increasing g, with the
+// tolerance scale T[m, n] = sum_g |xs[m,g] ws[n,g]| sum_{k in g} |qx qw|.
+int oracle_int4_linear(const uint8_t* xq, const float* xs, int64_t M, int64_t K,
+                       const uint8_t* wq, const float* ws, int64_t N, const float* bias,
+                       uint16_t* y, double* y64, double* T) {
+  if (M < 0 || N < 0 || K <= 0 || K % 64 != 0) return -1;
+  const int64_t G = K / 64;
+  std::vector<int8_t> A((size_t)M * K), B((size_t)N * K);
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t k = 0; k < K; ++k) A[m * K + k] = static_cast<int8_t>(int4_code(xq + m * (K / 2), k));
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k) B[n * K + k] = static_cast<int8_t>(int4_code(wq + n * (K / 2), k));
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t m = 0; m < M; ++m) {
+    for (int64_t n = 0; n < N; ++n) {
+      double acc = 0.0, absacc = 0.0;
+      for (int64_t g = 0; g < G; ++g) {
+        int64_t isum = 0, iabs = 0;
+        for (int64_t k = g * 64; k < g * 64 + 64; ++k) {
+          const int64_t p = static_cast<int64_t>(A[m * K + k]) * B[n * K + k];
+          isum += p;
+          iabs += p < 0 ? -p : p;
+        }
+        const double sc = static_cast<double>(xs[m * G + g]) * static_cast<double>(ws[n * G + g]);
+        acc += sc * static_cast<double>(isum);
+        absacc += std::fabs(sc) * static_cast<double>(iabs);
+      }
+      const double v = acc + (bias ? static_cast<double>(bias[n]) : 0.0);
+      if (y64) y64[m * N + n] = v;
+      if (T) T[m * N + n] = absacc;
+      if (y) y[m * N + n] = oracle_bf16_from_double(v);
+    }
+  }
   return 0;
 }
 
