@@ -224,6 +224,30 @@ class Fp8rLayer:
         self.q.fp8r_linear_gemm(self.xq, self.xs, self.wq, self.wsc, bias=self.bias, y=self.y)
 
 
+class Int4Layer:
+    """INT4 W4A4 layer (weights quantized on the GPU by int4_quantize_rows)."""
+
+    def __init__(self, M, K, N, bias, device, seed=0):
+        import torch
+        import fp8_rowwise_quantized_b200 as q
+        from synthetic import make_linear_inputs
+        inp = make_linear_inputs(M, K, N, seed=seed, with_bias=bias)
+        self.q, self.M, self.K, self.N = q, M, K, N
+        self.x = inp.x.to(device)
+        self.wq, self.ws = q.prepare_int4_weight(inp.w.to(device))
+        self.bias = None if inp.bias is None else inp.bias.to(device)
+        self.y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        self.work = torch.empty(q.int4_linear_workspace_size(M, K, N), dtype=torch.uint8,
+                                device=device)
+        self.xq, self.xs = q.int4_quantize_rows(self.x)
+
+    def step(self):
+        self.q.int4_linear(self.x, self.wq, self.ws, bias=self.bias, y=self.y, workspace=self.work)
+
+    def gemm(self):
+        self.q.int4_linear_gemm(self.xq, self.xs, self.wq, self.ws, bias=self.bias, y=self.y)
+
+
 class SvdqLayer:
     """svdq_w4a4 NVFP4 layer (smoothing, rank-r bf16 branch, 4-bit residual) with
     synthetic operands of the Nvfp4Layer's shapes."""
@@ -738,6 +762,21 @@ def run_ours(args):
                               "gemm_frac_of_peak": fl / (gms / 1e3) / 1e12 / pk}
             del L
         torch.cuda.empty_cache()
+        # INT4 W4A4 layer on the headline shape: per-group fp32 scales are applied on the
+        # CUDA cores, 4 fp32 operations per output and 64-element group
+        i4 = Int4Layer(M, K, N, False, device)
+        i_ms, _ = time_events(i4.step, v_steps, 3, flush, stream)
+        ig_ms, _ = time_events(i4.gemm, v_steps, 3, flush, stream)
+        alu_ops = 4.0 * M * N * (K // 64)
+        sms = torch.cuda.get_device_properties(device).multi_processor_count
+        alu_peak = sms * 128 * peaks.get("sm_max_mhz", 1965.0) * 1e6  # fp32 lanes per second
+        variants["int4_w4a4_4096x3072x12288"] = {
+            "us": i_ms * 1e3, "tops": flops / (i_ms / 1e3) / 1e12,
+            "gemm_us": ig_ms * 1e3, "gemm_tops": flops / (ig_ms / 1e3) / 1e12,
+            "gemm_scaling_bound_us": alu_ops / alu_peak * 1e6,
+            "note": "roofline: 4 fp32 ops per output per group on 128 lanes/clk/SM"}
+        del i4
+        torch.cuda.empty_cache()
         # svdq_w4a4 NVFP4 layer (rank 32) on the headline shape
         sv = SvdqLayer(M, K, N, 32, device)
         s_ms, _ = time_events(sv.step, v_steps, 3, flush, stream)
@@ -814,7 +853,8 @@ def run_profile(args):
     of one piece of the headline workload (no flushes, no timing): `step`,
     `prologue`, `gemm`, `quant` (activation quantization alone), `mlp_fused` (the MLP
     block with the GELU-quantize epilogue), `svdq` (the rank-32 svdq layer), `fp8r_step`,
-    `fp8r_quant`, `fp8r_gemm`, `w4a16` (the 1 x 3072 x 18432 modulation layer over
+    `fp8r_quant`, `fp8r_gemm`, `int4` (the INT4 W4A4 layer on the headline shape),
+    `w4a16` (the 1 x 3072 x 18432 modulation layer over
     rotating weight copies) or `skinny_<M>_<N>` (nvfp4_linear at K = 3072 over
     rotating copies)."""
     import torch
@@ -827,6 +867,9 @@ def run_profile(args):
     elif args.profile == "svdq":
         sv = SvdqLayer(4096, 3072, 12288, 32, device)
         fn = sv.step
+    elif args.profile == "int4":
+        L4 = Int4Layer(M, K, N, False, device)
+        fn = L4.step
     elif args.profile == "w4a16":
         W = W4a16Rotation(1, 3072, 18432, device)
         fn = W.step
@@ -865,7 +908,7 @@ def main():
     ap.add_argument("--no-variants", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", choices=["step", "prologue", "gemm", "quant", "mlp_fused", "svdq",
-                                          "fp8r_step", "fp8r_quant", "fp8r_gemm", "w4a16",
+                                          "fp8r_step", "fp8r_quant", "fp8r_gemm", "w4a16", "int4",
                                           "skinny_16_3072", "skinny_16_12288",
                                           "skinny_256_12288"], default=None,
                     help="run a short fixed sequence for a profiler instead of the benchmark")

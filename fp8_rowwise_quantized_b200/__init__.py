@@ -22,7 +22,8 @@ __all__ = [
     "nvfp4_quantize_act", "nvfp4_linear", "nvfp4_linear_single_launch", "nvfp4_linear_noalloc",
     "nvfp4_linear_prologue", "nvfp4_linear_gelu_quantize", "nvfp4_linear_quantized_input",
     "nvfp4_linear_gemm_lowrank", "svdq_nvfp4_linear", "svdq_nvfp4_linear_workspace_size",
-    "w4a16_linear",
+    "w4a16_linear", "int4_quantize_rows", "int4_linear", "int4_linear_gemm",
+    "int4_linear_workspace_size", "prepare_int4_weight",
     "nvfp4_linear_gemm",
     "nvfp4_linear_workspace_size", "nvfp4_linear_workspace_layout", "nvfp4_global_scale",
     "fp8r_quantize_rows", "fp8r_linear", "fp8r_linear_gemm", "fp8r_linear_workspace_size",
@@ -371,6 +372,70 @@ def prepare_nvfp4_weight(w: torch.Tensor):
 
 
 # ----------------------------------------------------------------------------- fp8r
+
+# ----------------------------------------------------------------------------- INT4
+
+def int4_quantize_rows(x: torch.Tensor, q: Optional[torch.Tensor] = None,
+                       scale: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """bf16 [M, K] -> (INT4 codes uint8 [M, K/2], fp32 group scales [M, K/64])."""
+    _need(x, "x", torch.bfloat16, 2)
+    M, K = x.shape
+    if q is None:
+        q = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device)
+    if scale is None:
+        scale = torch.empty((M, K // 64), dtype=torch.float32, device=x.device)
+    _lib.check("int4_quantize_rows", _lib.load().int4_quantize_rows(
+        _ptr(x), M, K, _ptr(q), _ptr(scale), _stream()))
+    return q, scale
+
+
+def prepare_int4_weight(w: torch.Tensor):
+    """bf16 weight [N, K] -> (INT4 codes [N, K/2], group scales [N, K/64])."""
+    return int4_quantize_rows(w.contiguous())
+
+
+def int4_linear_workspace_size(M: int, K: int, N: int) -> int:
+    return int(_lib.load().int4_linear_workspace_size(M, K, N))
+
+
+def int4_linear(x: torch.Tensor, w: torch.Tensor, w_scale: torch.Tensor,
+                bias: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
+                workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """INT4 W4A4 linear: Y = bf16(sum_g xs ws sum_k qx qw + bias), x quantized at run time."""
+    _need(x, "x", torch.bfloat16, 2)
+    _need(w, "w", torch.uint8, 2)
+    _need(w_scale, "w_scale", torch.float32, 2)
+    M, K = x.shape
+    N = w.shape[0]
+    if w.shape[1] * 2 != K or tuple(w_scale.shape) != (N, K // 64):
+        raise ValueError("weight shapes do not match x")
+    if bias is not None:
+        _need(bias, "bias", torch.float32, 1)
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    ws = _workspace(int4_linear_workspace_size(M, K, N), x.device, workspace)
+    _lib.check("int4_linear", _lib.load().int4_linear(
+        _ptr(x), M, K, _ptr(w), _ptr(w_scale), N, _ptr(bias), _ptr(y), _ptr(ws), ws.numel(),
+        _stream()))
+    return y
+
+
+def int4_linear_gemm(xq: torch.Tensor, x_scale: torch.Tensor, w: torch.Tensor,
+                     w_scale: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                     y: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _need(xq, "xq", torch.uint8, 2)
+    _need(x_scale, "x_scale", torch.float32, 2)
+    _need(w, "w", torch.uint8, 2)
+    _need(w_scale, "w_scale", torch.float32, 2)
+    M, K = xq.shape[0], xq.shape[1] * 2
+    N = w.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    _lib.check("int4_linear_gemm", _lib.load().int4_linear_gemm(
+        _ptr(xq), _ptr(x_scale), M, K, _ptr(w), _ptr(w_scale), N, _ptr(bias), _ptr(y),
+        _stream()))
+    return y
+
 
 def fp8r_quantize_rows(x: torch.Tensor, xq: Optional[torch.Tensor] = None,
                        x_scale: Optional[torch.Tensor] = None):

@@ -12,7 +12,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libqlinear.so")
-SOURCES = ["abi.cu", "quantize.cu", "gemm.cu", "noalloc.cu", "svdq.cu", "w4a16.cu"]
+SOURCES = ["abi.cu", "quantize.cu", "gemm.cu", "noalloc.cu", "svdq.cu", "w4a16.cu", "int4.cu"]
 HEADERS = ["internal.h", "layout.cuh", "ptx.cuh", "quant.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

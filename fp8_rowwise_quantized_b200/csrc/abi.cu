@@ -563,6 +563,63 @@ int fp8r_linear(const void* x, int64_t M, int64_t K, const uint8_t* w, const flo
   return fp8r_gemm_impl(xq, xs, M, K, w, w_scale, N, bias, y, stream, true);
 }
 
+// ------------------------------------------------------------------ INT4 W4A4
+
+static bool int4_shape_ok(int64_t M, int64_t K, int64_t N) {
+  return M >= 1 && N >= 1 && K >= 64 && K % 64 == 0 && M <= (1ll << 30) && N <= (1ll << 30) &&
+         K <= (1ll << 30);
+}
+
+int int4_quantize_rows(const void* x, int64_t M, int64_t K, uint8_t* q, float* scale,
+                       ql_stream_t stream) {
+  if (!x || !q || !scale || M <= 0 || K <= 0) return QL_ERR_INVALID_ARG;
+  if (!int4_shape_ok(M, K, 1)) return fail_shape("int4: needs K >= 64 and K % 64 == 0");
+  if (!aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(scale) & 3u) != 0)
+    return QL_ERR_ALIGN;
+  int rc = check_device(nullptr);
+  if (rc != QL_OK) return rc;
+  cudaError_t e = ql::launch_int4_quantize(x, M, K, q, scale, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QL_OK : record(e, "int4_quantize_rows");
+}
+
+int int4_linear_gemm(const uint8_t* xq, const float* x_scale, int64_t M, int64_t K,
+                     const uint8_t* w, const float* w_scale, int64_t N, const float* bias,
+                     void* y, ql_stream_t stream) {
+  if (!xq || !x_scale || !w || !w_scale || !y || M <= 0 || N <= 0 || K <= 0)
+    return QL_ERR_INVALID_ARG;
+  if (!int4_shape_ok(M, K, N)) return fail_shape("int4: needs K >= 64 and K % 64 == 0");
+  if (!aligned16(xq) || !aligned16(w) || (reinterpret_cast<uintptr_t>(x_scale) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(w_scale) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(bias) & 3u) != 0 || (reinterpret_cast<uintptr_t>(y) & 1u) != 0)
+    return QL_ERR_ALIGN;
+  int rc = check_device(nullptr);
+  if (rc != QL_OK) return rc;
+  cudaError_t e = ql::launch_int4_gemm(xq, x_scale, M, K, w, w_scale, N, bias, y,
+                                       reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QL_OK : record(e, "int4_linear_gemm");
+}
+
+size_t int4_linear_workspace_size(int64_t M, int64_t K, int64_t N) {
+  if (!int4_shape_ok(M, K, N)) return 0;
+  return ql::align_up(static_cast<size_t>(M) * static_cast<size_t>(K / 2), 1024) +
+         ql::align_up(static_cast<size_t>(M) * static_cast<size_t>(K / 64) * 4, 1024);
+}
+
+int int4_linear(const void* x, int64_t M, int64_t K, const uint8_t* w, const float* w_scale,
+                int64_t N, const float* bias, void* y, void* workspace, size_t workspace_bytes,
+                ql_stream_t stream) {
+  if (!x || !w || !w_scale || !y || M <= 0 || N <= 0 || K <= 0) return QL_ERR_INVALID_ARG;
+  if (!int4_shape_ok(M, K, N)) return fail_shape("int4: needs K >= 64 and K % 64 == 0");
+  if (!workspace || workspace_bytes < int4_linear_workspace_size(M, K, N)) return QL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return QL_ERR_ALIGN;
+  uint8_t* xq = static_cast<uint8_t*>(workspace);
+  float* xs = reinterpret_cast<float*>(
+      xq + ql::align_up(static_cast<size_t>(M) * static_cast<size_t>(K / 2), 1024));
+  int rc = int4_quantize_rows(x, M, K, xq, xs, stream);
+  if (rc != QL_OK) return rc;
+  return int4_linear_gemm(xq, xs, M, K, w, w_scale, N, bias, y, stream);
+}
+
 // ------------------------------------------------------------------ diagnostics
 
 int ql_encode_e4m3(const float* in, uint8_t* out, int64_t n, ql_stream_t stream) {

@@ -86,6 +86,12 @@ cudaError_t launch_svdq_prologue(const void* x, int64_t M, int64_t K, const floa
 cudaError_t launch_w4a16_linear(const void* x, int64_t M, int64_t K, const uint8_t* w,
                                 const uint8_t* w_scale, int64_t N, const float* weight_scale_2,
                                 const float* bias, void* y, cudaStream_t s);
+// INT4 W4A4 (int4.cu): K % 64 == 0; x, q, w 16-byte aligned.
+cudaError_t launch_int4_quantize(const void* x, int64_t M, int64_t K, uint8_t* q, float* scale,
+                                 cudaStream_t s);
+cudaError_t launch_int4_gemm(const uint8_t* xq, const float* xs, int64_t M, int64_t K,
+                             const uint8_t* wq, const float* ws, int64_t N, const float* bias,
+                             void* y, cudaStream_t s);
 cudaError_t launch_fp8r_quantize_rows(const void* x, int64_t M, int64_t K, uint8_t* xq,
                                       float* x_scale, cudaStream_t s);
 cudaError_t launch_global_scale(const void* x, int64_t n, float* out, cudaStream_t s);

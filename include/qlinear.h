@@ -259,6 +259,48 @@ int nvfp4_linear_noalloc(const void* x, int64_t M, int64_t K,
                          const float* bias, void* y, ql_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* INT4 W4A4                                                                 */
+/* ------------------------------------------------------------------------ */
+
+/* INT4 quantization of rows: the INT4 variant of the 4-bit layer of the Diffusers
+ * page "Bringing Nunchaku 4-bit Diffusion Inference to Diffusers" (section
+ * "Introducing Nunchaku Lite": svdq_w4a4, "available in INT4 and NVFP4 variants").
+ * The page gives no format; this library's reading, per 64-element group along K:
+ *   scale = RN32(amax / 7); codes = clamp(round-half-even(RN32(x * RN32(1/scale))),
+ *   -8, 7); all codes 0 when scale == 0.
+ *   x      bf16 [M, K]
+ *   q      uint8 [M, K/2] signed 4-bit codes, element 2j in bits 3..0 of byte j
+ *   scale  fp32 [M, K/64] row-major group scales
+ * Used for activations (rows = tokens) and weights (rows = output channels).
+ * Requires K >= 64, K % 64 == 0; x and q 16-byte aligned. */
+int int4_quantize_rows(const void* x, int64_t M, int64_t K, uint8_t* q, float* scale,
+                       ql_stream_t stream);
+
+/* Bytes of workspace int4_linear needs (0 on bad sizes): the quantized rows of x. */
+size_t int4_linear_workspace_size(int64_t M, int64_t K, int64_t N);
+
+/* INT4 W4A4 linear forward (no low-rank branch):
+ *   Y[m, n] = bf16( sum_g x_scale[m,g] w_scale[n,g] sum_{k in g} qx[m,k] qw[n,k] + bias[n] )
+ * quantizing x at run time (int4_quantize_rows into the workspace), then a GEMM on
+ * warp-level 4-bit tensor-core MMAs with each group's integer sums scaled and added
+ * in fp32 (per-group fp32 scales have no block-scaled tcgen05 form).
+ *   x        bf16 [M, K]
+ *   w        uint8 [N, K/2] INT4 weight codes (as int4_quantize_rows writes them)
+ *   w_scale  fp32 [N, K/64] group scales
+ *   bias     fp32 [N] or NULL;  y  bf16 [M, N] (output)
+ *   workspace >= int4_linear_workspace_size(M, K, N) bytes, 16-byte aligned
+ * Requires K >= 64, K % 64 == 0; x, w 16-byte aligned. */
+int int4_linear(const void* x, int64_t M, int64_t K, const uint8_t* w, const float* w_scale,
+                int64_t N, const float* bias, void* y, void* workspace, size_t workspace_bytes,
+                ql_stream_t stream);
+
+/* The GEMM half of int4_linear, from activations quantized by int4_quantize_rows:
+ * xq uint8 [M, K/2], x_scale fp32 [M, K/64]. */
+int int4_linear_gemm(const uint8_t* xq, const float* x_scale, int64_t M, int64_t K,
+                     const uint8_t* w, const float* w_scale, int64_t N, const float* bias,
+                     void* y, ql_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* fp8r (FP8 row-wise)                                                       */
 /* ------------------------------------------------------------------------ */
 

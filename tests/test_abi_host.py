@@ -77,6 +77,10 @@ def test_argument_errors_before_device():
     assert lib.nvfp4_quantize_act(fake, M, 24, fake, fake, fake, None) == 2
     assert lib.nvfp4_quantize_act(odd, M, K, fake, fake, fake, None) == 3
     assert lib.ql_encode_e4m3(None, fake, 10, None) == 1
+    # int4: K % 64, null workspace
+    assert lib.int4_quantize_rows(fake, M, 96, fake, fake, None) == 2
+    assert lib.int4_linear(fake, M, K, fake, fake, N, None, fake, None, 1 << 20, None) == 5
+    assert lib.int4_linear_workspace_size(M, 96, N) == 0
     # w4a16: null weight, K % 32, misaligned x, odd w_scale
     assert lib.w4a16_linear(fake, 1, K, None, fake, N, fake, None, fake, None) == 1
     assert lib.w4a16_linear(fake, 1, 48, fake, fake, N, fake, None, fake, None) == 2

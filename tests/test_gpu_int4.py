@@ -1,0 +1,94 @@
+"""GPU parity of the INT4 W4A4 linear (the INT4 variant of the Nunchaku page's
+4-bit layer; reading: signed 4-bit codes, one fp32 scale = amax / 7 per 64-element
+group) against the oracle, through the C ABI: codes and group scales bit-exact; the
+linear within the acceptance bound of the other layers (per element 1e-3 * T plus
+one bf16 ulp, Frobenius 5e-3), small shapes in full with ragged M and N, the
+diffusion-transformer sizes on sampled rows."""
+import numpy as np
+import pytest
+import torch
+
+import fp8_rowwise_quantized_b200 as q
+import oracle
+from gpu_helpers import check_linear, sample_rows, to_dev
+from synthetic import make_linear_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+class Int4Case:
+    def __init__(self, M, K, N, seed=0, bias=False):
+        inp = make_linear_inputs(M, K, N, seed=seed, with_bias=bias)
+        self.M, self.K, self.N = M, K, N
+        self.x = inp.x
+        self.wq, self.ws = oracle.int4_quantize(inp.w)
+        self.bias = None if inp.bias is None else inp.bias.numpy()
+
+    def run(self):
+        y = torch.full((self.M, self.N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        q.int4_linear(to_dev(self.x), to_dev(self.wq), to_dev(self.ws),
+                      bias=None if self.bias is None else to_dev(self.bias), y=y)
+        torch.cuda.synchronize()
+        assert bool(torch.isfinite(y).all()), "unwritten or non-finite outputs"
+        assert q.read_device_status() == 0
+        return y
+
+    def reference(self, rows=None):
+        xq, xs = oracle.int4_quantize(self.x)
+        if rows is not None:
+            xq, xs = xq[rows], xs[rows]
+        return oracle.int4_linear(xq, xs, self.wq, self.ws, self.bias)
+
+
+@pytest.mark.parametrize("M,K", [(1, 64), (7, 128), (130, 3072), (513, 1024)])
+def test_int4_quantize_bit_exact(M, K):
+    g = torch.Generator().manual_seed(M + K)
+    x = torch.randn(M, K, generator=g)
+    x[:, ::37] *= 30.0
+    if M > 2:
+        x[1] = 0.0                      # a zero row: scale 0, codes 0
+        x[2, :64] = 0.0                 # a zero group
+    x = x.to(torch.bfloat16)
+    qg, sg = q.int4_quantize_rows(x.cuda())
+    torch.cuda.synchronize()
+    qo, so = oracle.int4_quantize(x)
+    np.testing.assert_array_equal(sg.cpu().numpy(), so)
+    np.testing.assert_array_equal(qg.cpu().numpy(), qo)
+
+
+@pytest.mark.parametrize("M,K,N,bias", [
+    (1, 64, 8, False),        # one group, one row
+    (17, 192, 130, True),     # ragged M and N, three groups
+    (130, 1024, 257, True),   # two row tiles, three column tiles
+    (256, 3072, 384, False),
+])
+def test_int4_linear_small_full(M, K, N, bias):
+    c = Int4Case(M, K, N, seed=M + N, bias=bias)
+    y = c.run()
+    _, y64, T = c.reference()
+    check_linear(y, y64, T, f"int4 {M}x{K}x{N}")
+
+
+@pytest.mark.parametrize("M,K,N,bias", [(4096, 3072, 3072, True), (4096, 3072, 12288, False)])
+def test_int4_linear_dit_sizes_sampled(M, K, N, bias):
+    c = Int4Case(M, K, N, seed=1, bias=bias)
+    y = c.run()
+    rows = sample_rows(M, 12, seed=2)
+    _, y64, T = c.reference(rows)
+    check_linear(y[torch.from_numpy(rows).cuda()], y64, T, f"int4 {M}x{K}x{N}")
+
+
+def test_int4_gemm_from_prequantized_matches_linear():
+    c = Int4Case(300, 1024, 520, seed=3, bias=True)
+    x = to_dev(c.x)
+    y1 = c.run()
+    xq, xs = q.int4_quantize_rows(x)
+    y2 = q.int4_linear_gemm(xq, xs, to_dev(c.wq), to_dev(c.ws), bias=to_dev(c.bias))
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+
+
+def test_int4_rejects_k_not_multiple_of_64():
+    x = torch.zeros((4, 96), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(q.QLinearError):
+        q.int4_quantize_rows(x)
