@@ -592,10 +592,11 @@ int int4_linear_gemm(const uint8_t* xq, const float* x_scale, int64_t M, int64_t
       (reinterpret_cast<uintptr_t>(w_scale) & 3u) != 0 ||
       (reinterpret_cast<uintptr_t>(bias) & 3u) != 0 || (reinterpret_cast<uintptr_t>(y) & 1u) != 0)
     return QL_ERR_ALIGN;
-  int rc = check_device(nullptr);
+  int dev = 0;
+  int rc = check_device(&dev);
   if (rc != QL_OK) return rc;
-  cudaError_t e = ql::launch_int4_gemm(xq, x_scale, M, K, w, w_scale, N, bias, y,
-                                       reinterpret_cast<cudaStream_t>(stream));
+  cudaError_t e = ql::launch_int4_gemm(xq, x_scale, M, K, w, w_scale, N, bias, y, status_ptr(dev),
+                                       timeout_ns(), reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? QL_OK : record(e, "int4_linear_gemm");
 }
 

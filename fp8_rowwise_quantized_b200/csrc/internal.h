@@ -91,7 +91,7 @@ cudaError_t launch_int4_quantize(const void* x, int64_t M, int64_t K, uint8_t* q
                                  cudaStream_t s);
 cudaError_t launch_int4_gemm(const uint8_t* xq, const float* xs, int64_t M, int64_t K,
                              const uint8_t* wq, const float* ws, int64_t N, const float* bias,
-                             void* y, cudaStream_t s);
+                             void* y, int* status, uint64_t timeout_ns, cudaStream_t s);
 cudaError_t launch_fp8r_quantize_rows(const void* x, int64_t M, int64_t K, uint8_t* xq,
                                       float* x_scale, cudaStream_t s);
 cudaError_t launch_global_scale(const void* x, int64_t n, float* out, cudaStream_t s);
