@@ -92,3 +92,31 @@ def test_int4_rejects_k_not_multiple_of_64():
     x = torch.zeros((4, 96), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(q.QLinearError):
         q.int4_quantize_rows(x)
+
+
+def test_int4_linear_odd_groups_ragged_tiles():
+    # nine 64-element groups (the last two-group pipeline stage holds one), three row
+    # tiles and five column tiles of 128, ragged in both
+    c = Int4Case(300, 576, 520, seed=5, bias=True)
+    y = c.run()
+    _, y64, T = c.reference()
+    check_linear(y, y64, T, "int4 300x576x520")
+
+
+def test_int4_gemm_unaligned_output_matches_aligned():
+    # an output that is not 16-byte aligned takes the element-wise store path; it must
+    # give the same bits and write nothing outside Y
+    M, K, N = 200, 320, 264
+    c = Int4Case(M, K, N, seed=6, bias=True)
+    xq, xs = q.int4_quantize_rows(to_dev(c.x))
+    w, ws, b = to_dev(c.wq), to_dev(c.ws), to_dev(c.bias)
+    y1 = q.int4_linear_gemm(xq, xs, w, ws, bias=b)
+    buf = torch.full((M * N + 8,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    y2 = buf[1:1 + M * N].view(M, N)
+    q.int4_linear_gemm(xq, xs, w, ws, bias=b, y=y2)
+    torch.cuda.synchronize()
+    assert y2.data_ptr() % 16 != 0
+    assert torch.equal(y1, y2)
+    assert bool(torch.isnan(buf[:1]).all()) and bool(torch.isnan(buf[1 + M * N:]).all())
+    _, y64, T = c.reference()
+    check_linear(y1, y64, T, "int4 200x320x264")
