@@ -281,9 +281,10 @@ size_t int4_linear_workspace_size(int64_t M, int64_t K, int64_t N);
 
 /* INT4 W4A4 linear forward (no low-rank branch):
  *   Y[m, n] = bf16( sum_g x_scale[m,g] w_scale[n,g] sum_{k in g} qx[m,k] qw[n,k] + bias[n] )
- * quantizing x at run time (int4_quantize_rows into the workspace), then a GEMM on
- * warp-level 4-bit tensor-core MMAs with each group's integer sums scaled and added
- * in fp32 (per-group fp32 scales have no block-scaled tcgen05 form).
+ * quantizing x at run time (int4_quantize_rows into the workspace), then a GEMM whose
+ * per-group integer sums come from tcgen05 int8 MMAs (the 4-bit codes widened to int8
+ * in shared memory) and are scaled and added in fp32 on the CUDA cores (per-group fp32
+ * scales have no block-scaled tcgen05 form).
  *   x        bf16 [M, K]
  *   w        uint8 [N, K/2] INT4 weight codes (as int4_quantize_rows writes them)
  *   w_scale  fp32 [N, K/64] group scales
@@ -295,7 +296,12 @@ int int4_linear(const void* x, int64_t M, int64_t K, const uint8_t* w, const flo
                 ql_stream_t stream);
 
 /* The GEMM half of int4_linear, from activations quantized by int4_quantize_rows:
- * xq uint8 [M, K/2], x_scale fp32 [M, K/64]. */
+ * xq uint8 [M, K/2], x_scale fp32 [M, K/64]; w, w_scale, bias and y as for int4_linear.
+ * Requires K >= 64, K % 64 == 0; xq and w 16-byte aligned, the scales and bias 4-byte,
+ * y 2-byte aligned (a 16-byte-aligned y with N % 8 == 0 takes 16-byte stores).
+ * Errors: QL_ERR_INVALID_ARG (null pointer, size <= 0), QL_ERR_SHAPE, QL_ERR_ALIGN,
+ * QL_ERR_DEVICE, QL_ERR_LAUNCH. Every wait inside the kernel is bounded; one that runs
+ * out sets the device status word (read with ql_read_device_status) to QL_ERR_TIMEOUT. */
 int int4_linear_gemm(const uint8_t* xq, const float* x_scale, int64_t M, int64_t K,
                      const uint8_t* w, const float* w_scale, int64_t N, const float* bias,
                      void* y, ql_stream_t stream);
