@@ -81,6 +81,20 @@ def test_argument_errors_before_device():
     assert lib.int4_quantize_rows(fake, M, 96, fake, fake, None) == 2
     assert lib.int4_linear(fake, M, K, fake, fake, N, None, fake, None, 1 << 20, None) == 5
     assert lib.int4_linear_workspace_size(M, 96, N) == 0
+    # workspace = activation codes then their group scales, each 1 KB-aligned
+    assert lib.int4_linear_workspace_size(M, K, N) == M * K // 2 + M * (K // 64) * 4
+    assert lib.int4_linear_workspace_size(3, 64, 1) == 1024 + 1024
+    assert lib.int4_linear(fake, M, K, fake, fake, N, None, fake, odd, 1 << 20, None) == 3
+    # int4_linear_gemm: null pointer, K % 64, misaligned codes / scales / bias / y
+    assert lib.int4_linear_gemm(None, fake, M, K, fake, fake, N, None, fake, None) == 1
+    assert lib.int4_linear_gemm(fake, fake, M, K, fake, fake, 0, None, fake, None) == 1
+    assert lib.int4_linear_gemm(fake, fake, M, 96, fake, fake, N, None, fake, None) == 2
+    assert lib.int4_linear_gemm(odd, fake, M, K, fake, fake, N, None, fake, None) == 3
+    assert lib.int4_linear_gemm(fake, fake, M, K, odd, fake, N, None, fake, None) == 3
+    assert lib.int4_linear_gemm(fake, fake + 2, M, K, fake, fake, N, None, fake, None) == 3
+    assert lib.int4_linear_gemm(fake, fake, M, K, fake, fake + 2, N, None, fake, None) == 3
+    assert lib.int4_linear_gemm(fake, fake, M, K, fake, fake, N, fake + 2, fake, None) == 3
+    assert lib.int4_linear_gemm(fake, fake, M, K, fake, fake, N, None, fake + 1, None) == 3
     # w4a16: null weight, K % 32, misaligned x, odd w_scale
     assert lib.w4a16_linear(fake, 1, K, None, fake, N, fake, None, fake, None) == 1
     assert lib.w4a16_linear(fake, 1, 48, fake, fake, N, fake, None, fake, None) == 2
