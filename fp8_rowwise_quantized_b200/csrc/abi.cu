@@ -36,8 +36,8 @@ int check_device(int* dev_out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return record(e, "cudaGetDevice");
-  static int cc_cache[64] = {};  // 0 = unknown, else major*10+minor
-  int cc = dev < 64 ? cc_cache[dev] : 0;
+  static std::atomic<int> cc_cache[64] = {};  // 0 = unknown, else major*10+minor
+  int cc = dev < 64 ? cc_cache[dev].load(std::memory_order_relaxed) : 0;
   if (cc == 0) {
     int major = 0, minor = 0;
     e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
@@ -45,7 +45,7 @@ int check_device(int* dev_out) {
     e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
     if (e != cudaSuccess) return record(e, "cudaDeviceGetAttribute");
     cc = major * 10 + minor;
-    if (dev < 64) cc_cache[dev] = cc;
+    if (dev < 64) cc_cache[dev].store(cc, std::memory_order_relaxed);
   }
   if (cc != 100) {
     std::snprintf(g_last_error, sizeof(g_last_error),

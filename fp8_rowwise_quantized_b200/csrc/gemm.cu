@@ -1244,9 +1244,9 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
   }
   // Persistent grid: as many CTA groups as can be resident at once (pairs need two
   // free SMs of one GPC, so fewer than SMs / 2 pairs may fit).
-  static int resident_groups[64] = {};
+  static std::atomic<int> resident_groups[64] = {};
   int max_groups = sms / CG;
-  if (dev < 64 && resident_groups[dev] == 0) {
+  if (dev < 64 && resident_groups[dev].load(std::memory_order_relaxed) == 0) {
     int n = max_groups;
     if (CG == 2) {
       cfg.gridDim = dim3(static_cast<unsigned>(max_groups * CG));
@@ -1257,9 +1257,9 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
         n = max_groups;
       }
     }
-    resident_groups[dev] = n < max_groups ? n : max_groups;
+    resident_groups[dev].store(n < max_groups ? n : max_groups, std::memory_order_relaxed);
   }
-  if (dev < 64) max_groups = resident_groups[dev];
+  if (dev < 64) max_groups = resident_groups[dev].load(std::memory_order_relaxed);
   const int groups = a.total_tiles < max_groups ? a.total_tiles : max_groups;
   cfg.gridDim = dim3(static_cast<unsigned>(groups * CG));
   if (p.pdl) {

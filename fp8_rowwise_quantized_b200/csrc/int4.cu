@@ -49,6 +49,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <mutex>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -551,19 +552,26 @@ cudaError_t launch_int4_quantize(const void* x, int64_t M, int64_t K, uint8_t* q
 cudaError_t launch_int4_gemm(const uint8_t* xq, const float* xs, int64_t M, int64_t K,
                              const uint8_t* wq, const float* ws, int64_t N, const float* bias,
                              void* y, int* status, uint64_t timeout_ns, cudaStream_t s) {
-  static int configured[64] = {};
+  // per device: the kernel's shared-memory limit (a per-device attribute) and the SM count
   static int sms[64] = {};
+  static std::mutex mu;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 64) return cudaErrorInvalidDevice;
-  if (!configured[dev]) {
-    e = cudaFuncSetAttribute(int4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kI4Smem);
-    if (e != cudaSuccess) return e;
-    e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
-    configured[dev] = 1;
+  int nsm = 0;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (sms[dev] == 0) {
+      e = cudaFuncSetAttribute(int4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kI4Smem);
+      if (e != cudaSuccess) return e;
+      int n = 0;
+      e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+      if (e != cudaSuccess) return e;
+      sms[dev] = n;
+    }
+    nsm = sms[dev];
   }
   const int64_t tm = (M + kI4Tile - 1) / kI4Tile, tn = (N + kI4Tile - 1) / kI4Tile;
   if (tm * tn > (1ll << 30)) return cudaErrorInvalidValue;
@@ -588,7 +596,7 @@ cudaError_t launch_int4_gemm(const uint8_t* xq, const float* xs, int64_t M, int6
   a.vec_store = (N % 8 == 0) && (reinterpret_cast<uintptr_t>(y) & 15u) == 0;
   a.status = status;
   a.timeout_ns = timeout_ns;
-  const int grid = a.total_tiles < sms[dev] ? a.total_tiles : sms[dev];
+  const int grid = a.total_tiles < nsm ? a.total_tiles : nsm;
   int4_gemm_kernel<<<grid, kI4Threads, kI4Smem, s>>>(ta, tb, a);
   return cudaGetLastError();
 }

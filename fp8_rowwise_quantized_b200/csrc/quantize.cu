@@ -10,6 +10,7 @@
 // nvfp4 and fp8r entries; "Kernels" table: run-time activation quantization).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <atomic>
 #include <cstdint>
 
 #include "internal.h"
@@ -316,8 +317,12 @@ cudaError_t launch_nvfp4_quantize_rowmajor(const void* x, int64_t M, int64_t K, 
                                            uint8_t* xq, uint8_t* xs, cudaStream_t s) {
   const int64_t segs = ceil_div64(K, 1024);
   const int64_t items = M * segs;
-  static int64_t wave = 0;
-  if (wave == 0) wave = resident_blocks(nvfp4_quantize_kernel<false>);
+  static std::atomic<int64_t> wave_cache{0};  // resident blocks of one wave (same on every B200)
+  int64_t wave = wave_cache.load(std::memory_order_relaxed);
+  if (wave == 0) {
+    wave = resident_blocks(nvfp4_quantize_kernel<false>);
+    wave_cache.store(wave, std::memory_order_relaxed);
+  }
   const int64_t need = ceil_div64(items, kQuantThreads / 32);
   const int64_t blocks = need < wave ? need : wave;
   nvfp4_quantize_kernel<false><<<static_cast<unsigned>(blocks), kQuantThreads, 0, s>>>(
@@ -336,8 +341,12 @@ cudaError_t launch_nvfp4_prologue(const void* x, int64_t M, int64_t K, const uin
   const int na = (bn + 127) / 128;
   const int64_t n_tiles = ceil_div64(N, bn);
   const int64_t w_jobs = n_tiles * na * ceil_div64(KG, kWsGroups);
-  static int64_t wave = 0;
-  if (wave == 0) wave = resident_blocks(nvfp4_prologue_kernel);
+  static std::atomic<int64_t> wave_cache{0};  // resident blocks of one wave (same on every B200)
+  int64_t wave = wave_cache.load(std::memory_order_relaxed);
+  if (wave == 0) {
+    wave = resident_blocks(nvfp4_prologue_kernel);
+    wave_cache.store(wave, std::memory_order_relaxed);
+  }
   int64_t need = ceil_div64(rows * segs, kQuantThreads / 32);
   if (need < w_jobs) need = w_jobs;
   const int64_t blocks = need < wave ? need : wave;
@@ -358,8 +367,12 @@ cudaError_t launch_nvfp4_weight_layout(const uint8_t* w_scale, int64_t M, int64_
   const int na = (bn + 127) / 128;
   const int64_t n_tiles = ceil_div64(N, bn);
   const int64_t w_jobs = n_tiles * na * ceil_div64(KG, kWsGroups);
-  static int64_t wave = 0;
-  if (wave == 0) wave = resident_blocks(nvfp4_prologue_kernel);
+  static std::atomic<int64_t> wave_cache{0};  // resident blocks of one wave (same on every B200)
+  int64_t wave = wave_cache.load(std::memory_order_relaxed);
+  if (wave == 0) {
+    wave = resident_blocks(nvfp4_prologue_kernel);
+    wave_cache.store(wave, std::memory_order_relaxed);
+  }
   const int64_t blocks = w_jobs < wave ? w_jobs : wave;
   nvfp4_prologue_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, 0, s>>>(
       nullptr, static_cast<int>(M), static_cast<int>(K), input_scale, workspace + L.codes_off,

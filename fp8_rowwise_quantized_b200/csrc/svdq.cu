@@ -31,6 +31,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <mutex>
 
 #include "internal.h"
 #include "layout.cuh"
@@ -381,13 +382,22 @@ svdq_prologue_kernel(const __grid_constant__ CUtensorMap tmap_x,
 template <int NB>
 cudaError_t launch_svdq_typed(const CUtensorMap& tx, const CUtensorMap& tws,
                               const SvdqPrologueArgs& args, unsigned grid, cudaStream_t s) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    const cudaError_t e = cudaFuncSetAttribute(svdq_prologue_kernel<NB>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               static_cast<int>(kSvSmemBytes));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
+  // the shared-memory limit is a per-device attribute of the kernel
+  static bool attr_set[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64) return cudaErrorInvalidDevice;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!attr_set[dev]) {
+      e = cudaFuncSetAttribute(svdq_prologue_kernel<NB>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kSvSmemBytes));
+      if (e != cudaSuccess) return e;
+      attr_set[dev] = true;
+    }
   }
   svdq_prologue_kernel<NB><<<grid, kSvThreads, kSvSmemBytes, s>>>(tx, tws, args);
   return cudaGetLastError();
