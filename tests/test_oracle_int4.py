@@ -7,7 +7,9 @@ reciprocal multiply), independent of the oracle's own code:
   * hand-worked ties round to even; zero groups give zero codes and scale 0;
   * sign symmetry; the clamp to [-8, 7] (only reachable through rounding up);
   * the linear equals exact rational arithmetic on tiny shapes (Fractions), a closed
-    form, and numpy's matmul of the dequantized operands.
+    form, and numpy's matmul of the dequantized operands;
+  * a row of three groups worked by hand (tests/golden/int4_worked_groups.txt): its
+    packed bytes, scales and the bf16 result of its linear with itself (a tie).
 """
 from fractions import Fraction
 
@@ -143,3 +145,42 @@ def test_linear_equals_numpy_matmul_of_dequantized_operands():
     # and the 4-bit result is a plausible approximation of the unquantized product
     full = bf16(x).double().numpy() @ bf16(w).double().numpy().T
     assert np.linalg.norm(y64 - full) / np.linalg.norm(full) < 0.3
+
+
+def _expand(tokens, conv):
+    out = []
+    for t in tokens:
+        if "*" in t:
+            v, n = t.split("*")
+            out += [conv(v)] * int(n)
+        else:
+            out.append(conv(t))
+    return out
+
+
+def test_hand_worked_groups_from_golden_file():
+    """tests/golden/int4_worked_groups.txt: codes, scales and one output worked by hand."""
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "int4_worked_groups.txt")
+    xs, fields = [], {}
+    for line in open(path):
+        line = line.split("#")[0].strip()
+        if not line:
+            continue
+        key, *rest = line.split()
+        if key == "x":
+            xs += _expand(rest, float)
+        else:
+            fields[key] = rest
+    assert len(xs) == 192
+    x = torch.tensor([xs], dtype=torch.float32).to(torch.bfloat16)
+    assert torch.equal(x.float(), torch.tensor([xs]))  # every value is exact in bf16
+    q, s = oracle.int4_quantize(x)
+    want_bytes = np.array(_expand(fields["bytes"], lambda v: int(v, 16)), np.uint8)
+    np.testing.assert_array_equal(q[0], want_bytes)
+    np.testing.assert_array_equal(s[0], np.array([float(v) for v in fields["scales"]], np.float32))
+    y, y64, _ = oracle.int4_linear(q, s, q, s)
+    assert y64[0, 0] == 251.5
+    want_y = float(fields["y"][0])
+    got = torch.tensor([int(y[0, 0])], dtype=torch.int32).to(torch.int16).view(torch.bfloat16)
+    assert float(got.float()[0]) == want_y
