@@ -11,6 +11,10 @@ The scheme (Diffusers page "BFL (fp8r / nvfp4)", scheme list):
     activations are quantized to NVFP4 at run time;
   * fp8r: E4M3 weight with one fp32 scale per row; activations are quantized per
     row to E4M3 at run time.
+
+Every tensor argument is checked (dtype, shape, contiguity) and must live on the
+device of the call (the device of its first tensor argument); the library call
+runs with that device current, on its current stream.
 """
 from typing import Optional, Tuple
 
@@ -40,27 +44,70 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
     return None if t is None else t.data_ptr()
 
 
-def _stream() -> int:
-    return torch.cuda.current_stream().cuda_stream
-
-
-def _need(t: torch.Tensor, name: str, dtype, ndim: Optional[int] = None):
+def _need(t: torch.Tensor, name: str, dtype, ndim: Optional[int] = None,
+          shape: Optional[tuple] = None, device: Optional[torch.device] = None):
+    """Checks a tensor argument: dtype, rank, shape, contiguity, and that it is a
+    CUDA tensor, on `device` (the device of the call) when one is given."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
-    if not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor")
     if t.dtype != dtype:
         raise ValueError(f"{name} must have dtype {dtype}, got {t.dtype}")
-    if not t.is_contiguous():
-        raise ValueError(f"{name} must be contiguous")
     if ndim is not None and t.dim() != ndim:
         raise ValueError(f"{name} must have {ndim} dims, got {t.dim()}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, but the call runs on {device}")
 
 
-def _scalar(t: torch.Tensor, name: str):
-    _need(t, name, torch.float32)
+def _scalar(t: torch.Tensor, name: str, device: Optional[torch.device] = None):
+    _need(t, name, torch.float32, device=device)
     if t.numel() != 1:
         raise ValueError(f"{name} must hold one fp32 value")
+
+
+def _out(y: Optional[torch.Tensor], M: int, N: int, device: torch.device) -> torch.Tensor:
+    """The bf16 [M, N] output: allocated when None, else checked."""
+    if y is None:
+        return torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    _need(y, "y", torch.bfloat16, 2, (M, N), device)
+    return y
+
+
+def _bias(bias: Optional[torch.Tensor], N: int, device: torch.device) -> None:
+    if bias is not None:
+        _need(bias, "bias", torch.float32, 1, (N,), device)
+
+
+def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]) -> torch.Tensor:
+    if workspace is None:
+        return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+    _need(workspace, "workspace", torch.uint8, device=device)
+    if workspace.numel() < nbytes:
+        raise ValueError(f"workspace holds {workspace.numel()} bytes, the call needs {nbytes}")
+    return workspace
+
+
+def _call(name: str, device: torch.device, *args) -> None:
+    """Runs the C entry point `name` with `device` current, on that device's current
+    stream (appended as the last argument); raises on a non-zero status."""
+    with torch.cuda.device(device):
+        stream = torch.cuda.current_stream(device).cuda_stream
+        _lib.check(name, getattr(_lib.load(), name)(*args, stream))
+
+
+def _nvfp4_weight(w: torch.Tensor, w_scale: torch.Tensor, K: int, dev) -> int:
+    """Checks an NVFP4 weight (codes uint8 [N, K/2], scales uint8 [N, K/16]); returns N."""
+    _need(w, "w", torch.uint8, 2, device=dev)
+    N = w.shape[0]
+    if w.shape[1] * 2 != K:
+        raise ValueError(f"w must have K/2 = {K // 2} bytes per row, got {w.shape[1]}")
+    _need(w_scale, "w_scale", torch.uint8, 2, (N, K // 16), dev)
+    return N
 
 
 # ----------------------------------------------------------------------------- NVFP4
@@ -70,14 +117,16 @@ def nvfp4_quantize_act(x: torch.Tensor, input_scale: torch.Tensor,
                        xs: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
     """bf16 [M, K] -> (packed E2M1 codes uint8 [M, K/2], E4M3 block scales uint8 [M, K/16])."""
     _need(x, "x", torch.bfloat16, 2)
-    _scalar(input_scale, "input_scale")
+    dev = x.device
+    _scalar(input_scale, "input_scale", dev)
     M, K = x.shape
     if xq is None:
-        xq = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device)
+        xq = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+    _need(xq, "xq", torch.uint8, 2, (M, K // 2), dev)
     if xs is None:
-        xs = torch.empty((M, K // 16), dtype=torch.uint8, device=x.device)
-    _lib.check("nvfp4_quantize_act", _lib.load().nvfp4_quantize_act(
-        _ptr(x), M, K, _ptr(input_scale), _ptr(xq), _ptr(xs), _stream()))
+        xs = torch.empty((M, K // 16), dtype=torch.uint8, device=dev)
+    _need(xs, "xs", torch.uint8, 2, (M, K // 16), dev)
+    _call("nvfp4_quantize_act", dev, _ptr(x), M, K, _ptr(input_scale), _ptr(xq), _ptr(xs))
     return xq, xs
 
 
@@ -92,13 +141,6 @@ def nvfp4_linear_workspace_layout(M: int, K: int, N: int) -> Tuple[int, int, int
     return a.value, b.value, c.value
 
 
-def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]) -> torch.Tensor:
-    if workspace is None:
-        return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
-    _need(workspace, "workspace", torch.uint8)
-    return workspace
-
-
 def nvfp4_linear(x: torch.Tensor, w: torch.Tensor, w_scale: torch.Tensor,
                  weight_scale_2: torch.Tensor, input_scale: torch.Tensor,
                  bias: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
@@ -108,22 +150,16 @@ def nvfp4_linear(x: torch.Tensor, w: torch.Tensor, w_scale: torch.Tensor,
     x bf16 [M, K]; w uint8 [N, K/2]; w_scale uint8 [N, K/16] (E4M3 codes);
     weight_scale_2 / input_scale fp32 scalars; bias fp32 [N] or None."""
     _need(x, "x", torch.bfloat16, 2)
-    _need(w, "w", torch.uint8, 2)
-    _need(w_scale, "w_scale", torch.uint8, 2)
-    _scalar(weight_scale_2, "weight_scale_2")
-    _scalar(input_scale, "input_scale")
+    dev = x.device
     M, K = x.shape
-    N = w.shape[0]
-    if w.shape[1] * 2 != K or tuple(w_scale.shape) != (N, K // 16):
-        raise ValueError("weight shapes do not match x")
-    if bias is not None:
-        _need(bias, "bias", torch.float32, 1)
-    if y is None:
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    ws = _workspace(nvfp4_linear_workspace_size(M, K, N), x.device, workspace)
-    _lib.check("nvfp4_linear", _lib.load().nvfp4_linear(
-        _ptr(x), M, K, _ptr(w), _ptr(w_scale), N, _ptr(weight_scale_2), _ptr(input_scale),
-        _ptr(bias), _ptr(y), _ptr(ws), ws.numel(), _stream()))
+    N = _nvfp4_weight(w, w_scale, K, dev)
+    _scalar(weight_scale_2, "weight_scale_2", dev)
+    _scalar(input_scale, "input_scale", dev)
+    _bias(bias, N, dev)
+    y = _out(y, M, N, dev)
+    ws = _workspace(nvfp4_linear_workspace_size(M, K, N), dev, workspace)
+    _call("nvfp4_linear", dev, _ptr(x), M, K, _ptr(w), _ptr(w_scale), N, _ptr(weight_scale_2),
+          _ptr(input_scale), _ptr(bias), _ptr(y), _ptr(ws), ws.numel())
     return y
 
 
@@ -135,22 +171,16 @@ def nvfp4_linear_single_launch(x: torch.Tensor, w: torch.Tensor, w_scale: torch.
     """nvfp4_linear as one kernel launch (quantization inside the GEMM launch, then a
     grid-wide barrier, then the GEMM); same bits as nvfp4_linear. Needs K % 256 == 0."""
     _need(x, "x", torch.bfloat16, 2)
-    _need(w, "w", torch.uint8, 2)
-    _need(w_scale, "w_scale", torch.uint8, 2)
-    _scalar(weight_scale_2, "weight_scale_2")
-    _scalar(input_scale, "input_scale")
+    dev = x.device
     M, K = x.shape
-    N = w.shape[0]
-    if w.shape[1] * 2 != K or tuple(w_scale.shape) != (N, K // 16):
-        raise ValueError("weight shapes do not match x")
-    if bias is not None:
-        _need(bias, "bias", torch.float32, 1)
-    if y is None:
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    ws = _workspace(nvfp4_linear_workspace_size(M, K, N), x.device, workspace)
-    _lib.check("nvfp4_linear_single_launch", _lib.load().nvfp4_linear_single_launch(
-        _ptr(x), M, K, _ptr(w), _ptr(w_scale), N, _ptr(weight_scale_2), _ptr(input_scale),
-        _ptr(bias), _ptr(y), _ptr(ws), ws.numel(), _stream()))
+    N = _nvfp4_weight(w, w_scale, K, dev)
+    _scalar(weight_scale_2, "weight_scale_2", dev)
+    _scalar(input_scale, "input_scale", dev)
+    _bias(bias, N, dev)
+    y = _out(y, M, N, dev)
+    ws = _workspace(nvfp4_linear_workspace_size(M, K, N), dev, workspace)
+    _call("nvfp4_linear_single_launch", dev, _ptr(x), M, K, _ptr(w), _ptr(w_scale), N,
+          _ptr(weight_scale_2), _ptr(input_scale), _ptr(bias), _ptr(y), _ptr(ws), ws.numel())
     return y
 
 
@@ -164,23 +194,18 @@ def nvfp4_linear_gelu_quantize(x: torch.Tensor, w: torch.Tensor, w_scale: torch.
     next_workspace, a uint8 buffer of nvfp4_linear_workspace_size(M, N, N_down)
     bytes, for nvfp4_linear_quantized_input. Needs N % 256 == 0."""
     _need(x, "x", torch.bfloat16, 2)
-    _need(w, "w", torch.uint8, 2)
-    _need(w_scale, "w_scale", torch.uint8, 2)
-    _need(next_workspace, "next_workspace", torch.uint8, 1)
-    _scalar(weight_scale_2, "weight_scale_2")
-    _scalar(input_scale, "input_scale")
-    _scalar(next_input_scale, "next_input_scale")
+    dev = x.device
     M, K = x.shape
-    N = w.shape[0]
-    if w.shape[1] * 2 != K or tuple(w_scale.shape) != (N, K // 16):
-        raise ValueError("weight shapes do not match x")
-    if bias is not None:
-        _need(bias, "bias", torch.float32, 1)
-    ws = _workspace(nvfp4_linear_workspace_size(M, K, N), x.device, workspace)
-    _lib.check("nvfp4_linear_gelu_quantize", _lib.load().nvfp4_linear_gelu_quantize(
-        _ptr(x), M, K, _ptr(w), _ptr(w_scale), N, _ptr(weight_scale_2), _ptr(input_scale),
-        _ptr(bias), _ptr(next_input_scale), _ptr(next_workspace), next_workspace.numel(),
-        _ptr(ws), ws.numel(), _stream()))
+    N = _nvfp4_weight(w, w_scale, K, dev)
+    _need(next_workspace, "next_workspace", torch.uint8, 1, device=dev)
+    _scalar(weight_scale_2, "weight_scale_2", dev)
+    _scalar(input_scale, "input_scale", dev)
+    _scalar(next_input_scale, "next_input_scale", dev)
+    _bias(bias, N, dev)
+    ws = _workspace(nvfp4_linear_workspace_size(M, K, N), dev, workspace)
+    _call("nvfp4_linear_gelu_quantize", dev, _ptr(x), M, K, _ptr(w), _ptr(w_scale), N,
+          _ptr(weight_scale_2), _ptr(input_scale), _ptr(bias), _ptr(next_input_scale),
+          _ptr(next_workspace), next_workspace.numel(), _ptr(ws), ws.numel())
 
 
 def nvfp4_linear_quantized_input(M: int, w: torch.Tensor, w_scale: torch.Tensor,
@@ -190,20 +215,17 @@ def nvfp4_linear_quantized_input(M: int, w: torch.Tensor, w_scale: torch.Tensor,
     """nvfp4_linear on activations already quantized into `workspace` (by
     nvfp4_linear_gelu_quantize): weight-scale layout, then the GEMM."""
     _need(w, "w", torch.uint8, 2)
-    _need(w_scale, "w_scale", torch.uint8, 2)
-    _need(workspace, "workspace", torch.uint8, 1)
-    _scalar(weight_scale_2, "weight_scale_2")
-    _scalar(input_scale, "input_scale")
-    N, K = w.shape[0], w.shape[1] * 2
-    if tuple(w_scale.shape) != (N, K // 16):
-        raise ValueError("weight scale shape does not match w")
-    if bias is not None:
-        _need(bias, "bias", torch.float32, 1)
-    if y is None:
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=w.device)
-    _lib.check("nvfp4_linear_quantized_input", _lib.load().nvfp4_linear_quantized_input(
-        M, K, _ptr(w), _ptr(w_scale), N, _ptr(weight_scale_2), _ptr(input_scale), _ptr(bias),
-        _ptr(y), _ptr(workspace), workspace.numel(), _stream()))
+    dev = w.device
+    K = w.shape[1] * 2
+    N = _nvfp4_weight(w, w_scale, K, dev)
+    _need(workspace, "workspace", torch.uint8, 1, device=dev)
+    _scalar(weight_scale_2, "weight_scale_2", dev)
+    _scalar(input_scale, "input_scale", dev)
+    _bias(bias, N, dev)
+    y = _out(y, M, N, dev)
+    _call("nvfp4_linear_quantized_input", dev, M, K, _ptr(w), _ptr(w_scale), N,
+          _ptr(weight_scale_2), _ptr(input_scale), _ptr(bias), _ptr(y), _ptr(workspace),
+          workspace.numel())
     return y
 
 
@@ -215,22 +237,20 @@ def nvfp4_linear_gemm_lowrank(M: int, w: torch.Tensor, weight_scale_2: torch.Ten
     """nvfp4_linear_gemm plus the low-rank branch alpha * lr_act @ lr_up^T: lr_act bf16
     [M, r] (the branch's activations divided by alpha), lr_up bf16 [N, r]."""
     _need(w, "w", torch.uint8, 2)
-    _need(workspace, "workspace", torch.uint8, 1)
-    _need(lr_act, "lr_act", torch.bfloat16, 2)
-    _need(lr_up, "lr_up", torch.bfloat16, 2)
-    _scalar(weight_scale_2, "weight_scale_2")
-    _scalar(input_scale, "input_scale")
+    dev = w.device
     N, K = w.shape[0], w.shape[1] * 2
+    _need(workspace, "workspace", torch.uint8, 1, device=dev)
+    _need(lr_act, "lr_act", torch.bfloat16, 2, device=dev)
     r = lr_act.shape[1]
-    if lr_act.shape[0] != M or tuple(lr_up.shape) != (N, r):
-        raise ValueError("low-rank operand shapes do not match")
-    if bias is not None:
-        _need(bias, "bias", torch.float32, 1)
-    if y is None:
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=w.device)
-    _lib.check("nvfp4_linear_gemm_lowrank", _lib.load().nvfp4_linear_gemm_lowrank(
-        M, K, _ptr(w), N, _ptr(weight_scale_2), _ptr(input_scale), _ptr(bias), _ptr(lr_act),
-        _ptr(lr_up), r, _ptr(y), _ptr(workspace), workspace.numel(), _stream()))
+    _need(lr_act, "lr_act", torch.bfloat16, 2, (M, r), dev)
+    _need(lr_up, "lr_up", torch.bfloat16, 2, (N, r), dev)
+    _scalar(weight_scale_2, "weight_scale_2", dev)
+    _scalar(input_scale, "input_scale", dev)
+    _bias(bias, N, dev)
+    y = _out(y, M, N, dev)
+    _call("nvfp4_linear_gemm_lowrank", dev, M, K, _ptr(w), N, _ptr(weight_scale_2),
+          _ptr(input_scale), _ptr(bias), _ptr(lr_act), _ptr(lr_up), r, _ptr(y),
+          _ptr(workspace), workspace.numel())
     return y
 
 
@@ -248,30 +268,23 @@ def svdq_nvfp4_linear(x: torch.Tensor, w: torch.Tensor, w_scale: torch.Tensor,
     + (xs lora_down^T) lora_up^T + bias), xs = bf16(x * smooth). lora_down bf16 [r, K],
     lora_up bf16 [N, r], smooth fp32 [K] or None; input_scale calibrated on xs."""
     _need(x, "x", torch.bfloat16, 2)
-    _need(w, "w", torch.uint8, 2)
-    _need(w_scale, "w_scale", torch.uint8, 2)
-    _need(lora_down, "lora_down", torch.bfloat16, 2)
-    _need(lora_up, "lora_up", torch.bfloat16, 2)
-    _scalar(weight_scale_2, "weight_scale_2")
-    _scalar(input_scale, "input_scale")
+    dev = x.device
     M, K = x.shape
-    N = w.shape[0]
+    N = _nvfp4_weight(w, w_scale, K, dev)
+    _need(lora_down, "lora_down", torch.bfloat16, 2, device=dev)
     r = lora_down.shape[0]
-    if w.shape[1] * 2 != K or tuple(w_scale.shape) != (N, K // 16):
-        raise ValueError("weight shapes do not match x")
-    if tuple(lora_down.shape) != (r, K) or tuple(lora_up.shape) != (N, r):
-        raise ValueError("low-rank shapes do not match")
+    _need(lora_down, "lora_down", torch.bfloat16, 2, (r, K), dev)
+    _need(lora_up, "lora_up", torch.bfloat16, 2, (N, r), dev)
+    _scalar(weight_scale_2, "weight_scale_2", dev)
+    _scalar(input_scale, "input_scale", dev)
     if smooth is not None:
-        _need(smooth, "smooth", torch.float32, 1)
-    if bias is not None:
-        _need(bias, "bias", torch.float32, 1)
-    if y is None:
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    ws = _workspace(svdq_nvfp4_linear_workspace_size(M, K, N, r), x.device, workspace)
-    _lib.check("svdq_nvfp4_linear", _lib.load().svdq_nvfp4_linear(
-        _ptr(x), M, K, _ptr(smooth), _ptr(lora_down), _ptr(lora_up), r, _ptr(w), _ptr(w_scale),
-        N, _ptr(weight_scale_2), _ptr(input_scale), _ptr(bias), _ptr(y), _ptr(ws), ws.numel(),
-        _stream()))
+        _need(smooth, "smooth", torch.float32, 1, (K,), dev)
+    _bias(bias, N, dev)
+    y = _out(y, M, N, dev)
+    ws = _workspace(svdq_nvfp4_linear_workspace_size(M, K, N, r), dev, workspace)
+    _call("svdq_nvfp4_linear", dev, _ptr(x), M, K, _ptr(smooth), _ptr(lora_down), _ptr(lora_up),
+          r, _ptr(w), _ptr(w_scale), N, _ptr(weight_scale_2), _ptr(input_scale), _ptr(bias),
+          _ptr(y), _ptr(ws), ws.numel())
     return y
 
 
@@ -284,20 +297,14 @@ def w4a16_linear(x: torch.Tensor, w: torch.Tensor, w_scale: torch.Tensor,
     x bf16 [M, K]; w uint8 [N, K/2]; w_scale uint8 [N, K/16]; weight_scale_2 fp32
     scalar; bias fp32 [N] or None."""
     _need(x, "x", torch.bfloat16, 2)
-    _need(w, "w", torch.uint8, 2)
-    _need(w_scale, "w_scale", torch.uint8, 2)
-    _scalar(weight_scale_2, "weight_scale_2")
+    dev = x.device
     M, K = x.shape
-    N = w.shape[0]
-    if w.shape[1] * 2 != K or tuple(w_scale.shape) != (N, K // 16):
-        raise ValueError("weight shapes do not match x")
-    if bias is not None:
-        _need(bias, "bias", torch.float32, 1)
-    if y is None:
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    _lib.check("w4a16_linear", _lib.load().w4a16_linear(
-        _ptr(x), M, K, _ptr(w), _ptr(w_scale), N, _ptr(weight_scale_2), _ptr(bias), _ptr(y),
-        _stream()))
+    N = _nvfp4_weight(w, w_scale, K, dev)
+    _scalar(weight_scale_2, "weight_scale_2", dev)
+    _bias(bias, N, dev)
+    y = _out(y, M, N, dev)
+    _call("w4a16_linear", dev, _ptr(x), M, K, _ptr(w), _ptr(w_scale), N, _ptr(weight_scale_2),
+          _ptr(bias), _ptr(y))
     return y
 
 
@@ -306,60 +313,65 @@ def nvfp4_linear_noalloc(x: torch.Tensor, w: torch.Tensor, w_scale: torch.Tensor
                          bias: Optional[torch.Tensor] = None,
                          y: Optional[torch.Tensor] = None) -> torch.Tensor:
     """nvfp4_linear without a workspace argument, for callers that cannot allocate
-    device memory: the library's fixed 32 MiB scratch array is used instead (see
-    include/qlinear.h). Pass ``y`` to avoid the output allocation here as well."""
+    device memory: the library's fixed 32 MiB scratch array of the call's device is
+    used instead (see include/qlinear.h). Pass ``y`` to avoid the output allocation
+    here as well; it is checked (bf16 [M, N], contiguous, on x's device)."""
     _need(x, "x", torch.bfloat16, 2)
-    _need(w, "w", torch.uint8, 2)
-    _need(w_scale, "w_scale", torch.uint8, 2)
-    _scalar(weight_scale_2, "weight_scale_2")
-    _scalar(input_scale, "input_scale")
+    dev = x.device
     M, K = x.shape
-    N = w.shape[0]
-    if w.shape[1] * 2 != K or tuple(w_scale.shape) != (N, K // 16):
-        raise ValueError("weight shapes do not match x")
-    if bias is not None:
-        _need(bias, "bias", torch.float32, 1)
-    if y is None:
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    _lib.check("nvfp4_linear_noalloc", _lib.load().nvfp4_linear_noalloc(
-        _ptr(x), M, K, _ptr(w), _ptr(w_scale), N, _ptr(weight_scale_2), _ptr(input_scale),
-        _ptr(bias), _ptr(y), _stream()))
+    N = _nvfp4_weight(w, w_scale, K, dev)
+    _scalar(weight_scale_2, "weight_scale_2", dev)
+    _scalar(input_scale, "input_scale", dev)
+    _bias(bias, N, dev)
+    y = _out(y, M, N, dev)
+    _call("nvfp4_linear_noalloc", dev, _ptr(x), M, K, _ptr(w), _ptr(w_scale), N,
+          _ptr(weight_scale_2), _ptr(input_scale), _ptr(bias), _ptr(y))
     return y
 
 
 def nvfp4_linear_prologue(x: torch.Tensor, w_scale: torch.Tensor, input_scale: torch.Tensor,
                           workspace: torch.Tensor) -> None:
+    """The first launch of nvfp4_linear: quantizes x and lays out the weight scales
+    into `workspace` (nvfp4_linear_workspace_size(M, K, N) bytes)."""
     _need(x, "x", torch.bfloat16, 2)
-    _need(w_scale, "w_scale", torch.uint8, 2)
-    _scalar(input_scale, "input_scale")
+    dev = x.device
     M, K = x.shape
+    _need(w_scale, "w_scale", torch.uint8, 2, device=dev)
     N = w_scale.shape[0]
-    _lib.check("nvfp4_linear_prologue", _lib.load().nvfp4_linear_prologue(
-        _ptr(x), M, K, _ptr(w_scale), N, _ptr(input_scale), _ptr(workspace), workspace.numel(),
-        _stream()))
+    _need(w_scale, "w_scale", torch.uint8, 2, (N, K // 16), dev)
+    _scalar(input_scale, "input_scale", dev)
+    ws = _workspace(nvfp4_linear_workspace_size(M, K, N), dev, workspace)
+    _call("nvfp4_linear_prologue", dev, _ptr(x), M, K, _ptr(w_scale), N, _ptr(input_scale),
+          _ptr(ws), ws.numel())
 
 
 def nvfp4_linear_gemm(M: int, w: torch.Tensor, weight_scale_2: torch.Tensor,
                       input_scale: torch.Tensor, workspace: torch.Tensor,
                       bias: Optional[torch.Tensor] = None,
                       y: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The second launch of nvfp4_linear: the GEMM on a workspace filled by
+    nvfp4_linear_prologue."""
     _need(w, "w", torch.uint8, 2)
+    dev = w.device
     N, K = w.shape[0], w.shape[1] * 2
-    if y is None:
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=w.device)
-    _lib.check("nvfp4_linear_gemm", _lib.load().nvfp4_linear_gemm(
-        M, K, _ptr(w), N, _ptr(weight_scale_2), _ptr(input_scale), _ptr(bias), _ptr(y),
-        _ptr(workspace), workspace.numel(), _stream()))
+    _scalar(weight_scale_2, "weight_scale_2", dev)
+    _scalar(input_scale, "input_scale", dev)
+    ws = _workspace(nvfp4_linear_workspace_size(M, K, N), dev, workspace)
+    _bias(bias, N, dev)
+    y = _out(y, M, N, dev)
+    _call("nvfp4_linear_gemm", dev, M, K, _ptr(w), N, _ptr(weight_scale_2), _ptr(input_scale),
+          _ptr(bias), _ptr(y), _ptr(ws), ws.numel())
     return y
 
 
 def nvfp4_global_scale(x: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Device fp32 scalar amax(|x|) / (6 * 448) (the calibration rule of the workloads)."""
     _need(x, "x", torch.bfloat16)
+    dev = x.device
     if out is None:
-        out = torch.empty((1,), dtype=torch.float32, device=x.device)
-    _lib.check("nvfp4_global_scale", _lib.load().nvfp4_global_scale(
-        _ptr(x), x.numel(), _ptr(out), _stream()))
+        out = torch.empty((1,), dtype=torch.float32, device=dev)
+    _scalar(out, "out", dev)
+    _call("nvfp4_global_scale", dev, _ptr(x), x.numel(), _ptr(out))
     return out
 
 
@@ -371,21 +383,21 @@ def prepare_nvfp4_weight(w: torch.Tensor):
     return wq, ws, g
 
 
-# ----------------------------------------------------------------------------- fp8r
-
 # ----------------------------------------------------------------------------- INT4
 
 def int4_quantize_rows(x: torch.Tensor, q: Optional[torch.Tensor] = None,
                        scale: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
     """bf16 [M, K] -> (INT4 codes uint8 [M, K/2], fp32 group scales [M, K/64])."""
     _need(x, "x", torch.bfloat16, 2)
+    dev = x.device
     M, K = x.shape
     if q is None:
-        q = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device)
+        q = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+    _need(q, "q", torch.uint8, 2, (M, K // 2), dev)
     if scale is None:
-        scale = torch.empty((M, K // 64), dtype=torch.float32, device=x.device)
-    _lib.check("int4_quantize_rows", _lib.load().int4_quantize_rows(
-        _ptr(x), M, K, _ptr(q), _ptr(scale), _stream()))
+        scale = torch.empty((M, K // 64), dtype=torch.float32, device=dev)
+    _need(scale, "scale", torch.float32, 2, (M, K // 64), dev)
+    _call("int4_quantize_rows", dev, _ptr(x), M, K, _ptr(q), _ptr(scale))
     return q, scale
 
 
@@ -398,56 +410,62 @@ def int4_linear_workspace_size(M: int, K: int, N: int) -> int:
     return int(_lib.load().int4_linear_workspace_size(M, K, N))
 
 
+def _int4_weight(w: torch.Tensor, w_scale: torch.Tensor, K: int, dev) -> int:
+    _need(w, "w", torch.uint8, 2, device=dev)
+    N = w.shape[0]
+    if w.shape[1] * 2 != K:
+        raise ValueError(f"w must have K/2 = {K // 2} bytes per row, got {w.shape[1]}")
+    _need(w_scale, "w_scale", torch.float32, 2, (N, K // 64), dev)
+    return N
+
+
 def int4_linear(x: torch.Tensor, w: torch.Tensor, w_scale: torch.Tensor,
                 bias: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
                 workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
     """INT4 W4A4 linear: Y = bf16(sum_g xs ws sum_k qx qw + bias), x quantized at run time."""
     _need(x, "x", torch.bfloat16, 2)
-    _need(w, "w", torch.uint8, 2)
-    _need(w_scale, "w_scale", torch.float32, 2)
+    dev = x.device
     M, K = x.shape
-    N = w.shape[0]
-    if w.shape[1] * 2 != K or tuple(w_scale.shape) != (N, K // 64):
-        raise ValueError("weight shapes do not match x")
-    if bias is not None:
-        _need(bias, "bias", torch.float32, 1)
-    if y is None:
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    ws = _workspace(int4_linear_workspace_size(M, K, N), x.device, workspace)
-    _lib.check("int4_linear", _lib.load().int4_linear(
-        _ptr(x), M, K, _ptr(w), _ptr(w_scale), N, _ptr(bias), _ptr(y), _ptr(ws), ws.numel(),
-        _stream()))
+    N = _int4_weight(w, w_scale, K, dev)
+    _bias(bias, N, dev)
+    y = _out(y, M, N, dev)
+    ws = _workspace(int4_linear_workspace_size(M, K, N), dev, workspace)
+    _call("int4_linear", dev, _ptr(x), M, K, _ptr(w), _ptr(w_scale), N, _ptr(bias), _ptr(y),
+          _ptr(ws), ws.numel())
     return y
 
 
 def int4_linear_gemm(xq: torch.Tensor, x_scale: torch.Tensor, w: torch.Tensor,
                      w_scale: torch.Tensor, bias: Optional[torch.Tensor] = None,
                      y: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The GEMM of int4_linear on activations quantized by int4_quantize_rows."""
     _need(xq, "xq", torch.uint8, 2)
-    _need(x_scale, "x_scale", torch.float32, 2)
-    _need(w, "w", torch.uint8, 2)
-    _need(w_scale, "w_scale", torch.float32, 2)
+    dev = xq.device
     M, K = xq.shape[0], xq.shape[1] * 2
-    N = w.shape[0]
-    if y is None:
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
-    _lib.check("int4_linear_gemm", _lib.load().int4_linear_gemm(
-        _ptr(xq), _ptr(x_scale), M, K, _ptr(w), _ptr(w_scale), N, _ptr(bias), _ptr(y),
-        _stream()))
+    _need(x_scale, "x_scale", torch.float32, 2, (M, K // 64), dev)
+    N = _int4_weight(w, w_scale, K, dev)
+    _bias(bias, N, dev)
+    y = _out(y, M, N, dev)
+    _call("int4_linear_gemm", dev, _ptr(xq), _ptr(x_scale), M, K, _ptr(w), _ptr(w_scale), N,
+          _ptr(bias), _ptr(y))
     return y
 
+
+# ----------------------------------------------------------------------------- fp8r
 
 def fp8r_quantize_rows(x: torch.Tensor, xq: Optional[torch.Tensor] = None,
                        x_scale: Optional[torch.Tensor] = None):
     """bf16 [M, K] -> (E4M3 codes uint8 [M, K], fp32 row scales [M])."""
     _need(x, "x", torch.bfloat16, 2)
+    dev = x.device
     M, K = x.shape
     if xq is None:
-        xq = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+        xq = torch.empty((M, K), dtype=torch.uint8, device=dev)
+    _need(xq, "xq", torch.uint8, 2, (M, K), dev)
     if x_scale is None:
-        x_scale = torch.empty((M,), dtype=torch.float32, device=x.device)
-    _lib.check("fp8r_quantize_rows", _lib.load().fp8r_quantize_rows(
-        _ptr(x), M, K, _ptr(xq), _ptr(x_scale), _stream()))
+        x_scale = torch.empty((M,), dtype=torch.float32, device=dev)
+    _need(x_scale, "x_scale", torch.float32, 1, (M,), dev)
+    _call("fp8r_quantize_rows", dev, _ptr(x), M, K, _ptr(xq), _ptr(x_scale))
     return xq, x_scale
 
 
@@ -460,40 +478,44 @@ def fp8r_linear_workspace_size(M: int, K: int, N: int) -> int:
     return int(_lib.load().fp8r_linear_workspace_size(M, K, N))
 
 
+def _fp8r_weight(w: torch.Tensor, w_scale: torch.Tensor, K: int, dev) -> int:
+    _need(w, "w", torch.uint8, 2, device=dev)
+    N = w.shape[0]
+    if w.shape[1] != K:
+        raise ValueError(f"w must have K = {K} bytes per row, got {w.shape[1]}")
+    _need(w_scale, "w_scale", torch.float32, 1, (N,), dev)
+    return N
+
+
 def fp8r_linear(x: torch.Tensor, w: torch.Tensor, w_scale: torch.Tensor,
                 bias: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
                 workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Y = bf16(x_scale[m] * w_scale[n] * (E4M3(x) @ E4M3(w)^T) + bias)."""
     _need(x, "x", torch.bfloat16, 2)
-    _need(w, "w", torch.uint8, 2)
-    _need(w_scale, "w_scale", torch.float32, 1)
+    dev = x.device
     M, K = x.shape
-    N = w.shape[0]
-    if w.shape[1] != K or w_scale.shape[0] != N:
-        raise ValueError("weight shapes do not match x")
-    if bias is not None:
-        _need(bias, "bias", torch.float32, 1)
-    if y is None:
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    ws = _workspace(fp8r_linear_workspace_size(M, K, N), x.device, workspace)
-    _lib.check("fp8r_linear", _lib.load().fp8r_linear(
-        _ptr(x), M, K, _ptr(w), _ptr(w_scale), N, _ptr(bias), _ptr(y), _ptr(ws), ws.numel(),
-        _stream()))
+    N = _fp8r_weight(w, w_scale, K, dev)
+    _bias(bias, N, dev)
+    y = _out(y, M, N, dev)
+    ws = _workspace(fp8r_linear_workspace_size(M, K, N), dev, workspace)
+    _call("fp8r_linear", dev, _ptr(x), M, K, _ptr(w), _ptr(w_scale), N, _ptr(bias), _ptr(y),
+          _ptr(ws), ws.numel())
     return y
 
 
 def fp8r_linear_gemm(xq: torch.Tensor, x_scale: torch.Tensor, w: torch.Tensor,
                      w_scale: torch.Tensor, bias: Optional[torch.Tensor] = None,
                      y: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The GEMM of fp8r_linear on activations quantized by fp8r_quantize_rows."""
     _need(xq, "xq", torch.uint8, 2)
-    _need(w, "w", torch.uint8, 2)
+    dev = xq.device
     M, K = xq.shape
-    N = w.shape[0]
-    if y is None:
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
-    _lib.check("fp8r_linear_gemm", _lib.load().fp8r_linear_gemm(
-        _ptr(xq), _ptr(x_scale), M, K, _ptr(w), _ptr(w_scale), N, _ptr(bias), _ptr(y),
-        _stream()))
+    _need(x_scale, "x_scale", torch.float32, 1, (M,), dev)
+    N = _fp8r_weight(w, w_scale, K, dev)
+    _bias(bias, N, dev)
+    y = _out(y, M, N, dev)
+    _call("fp8r_linear_gemm", dev, _ptr(xq), _ptr(x_scale), M, K, _ptr(w), _ptr(w_scale), N,
+          _ptr(bias), _ptr(y))
     return y
 
 
@@ -502,18 +524,20 @@ def fp8r_linear_gemm(xq: torch.Tensor, x_scale: torch.Tensor, w: torch.Tensor,
 def ql_encode_e4m3(v: torch.Tensor) -> torch.Tensor:
     _need(v, "v", torch.float32)
     out = torch.empty(v.shape, dtype=torch.uint8, device=v.device)
-    _lib.check("ql_encode_e4m3", _lib.load().ql_encode_e4m3(_ptr(v), _ptr(out), v.numel(), _stream()))
+    _call("ql_encode_e4m3", v.device, _ptr(v), _ptr(out), v.numel())
     return out
 
 
 def ql_encode_e2m1(v: torch.Tensor) -> torch.Tensor:
     _need(v, "v", torch.float32)
     out = torch.empty(v.shape, dtype=torch.uint8, device=v.device)
-    _lib.check("ql_encode_e2m1", _lib.load().ql_encode_e2m1(_ptr(v), _ptr(out), v.numel(), _stream()))
+    _call("ql_encode_e2m1", v.device, _ptr(v), _ptr(out), v.numel())
     return out
 
 
 def read_device_status() -> int:
+    """Reads and clears the current device's status word (0, or QL_ERR_TIMEOUT after a
+    kernel's bounded wait expired)."""
     st = _lib.C.c_int(0)
     _lib.check("ql_read_device_status", _lib.load().ql_read_device_status(_lib.C.byref(st)))
     return st.value

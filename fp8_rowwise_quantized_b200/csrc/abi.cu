@@ -101,6 +101,8 @@ bool fp8r_shape_ok(int64_t M, int64_t K, int64_t N) {
 
 }  // namespace
 
+int ql::check_current_device(int* dev) { return check_device(dev); }
+
 void ql::set_error_text(const char* text) {
   std::snprintf(g_last_error, sizeof(g_last_error), "%s", text);
 }

@@ -107,4 +107,8 @@ bool encode_2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, uin
 // Sets the text ql_last_error_message() returns on this thread.
 void set_error_text(const char* text);
 
+// QL_OK when the current device is an sm_100 part (its ordinal in *dev), else
+// QL_ERR_DEVICE or QL_ERR_LAUNCH with the error text set.
+int check_current_device(int* dev);
+
 }  // namespace ql

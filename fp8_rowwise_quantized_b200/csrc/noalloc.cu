@@ -42,6 +42,7 @@ uint8_t* scratch_on_current_device(int* status) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || p == nullptr) {
+      cudaGetLastError();  // leave no error pending for the caller's next check
       char msg[200];
       std::snprintf(msg, sizeof(msg), "nvfp4_linear_noalloc: cudaGetSymbolAddress failed: %s",
                     cudaGetErrorString(e));
@@ -77,7 +78,9 @@ extern "C" int nvfp4_linear_noalloc(const void* x, int64_t M, int64_t K, const u
     ql::set_error_text(msg);
     return QL_ERR_WORKSPACE;
   }
-  int status = QL_OK;
+  // an sm_100 device first: elsewhere the scratch lookup itself would fail
+  int status = ql::check_current_device(nullptr);
+  if (status != QL_OK) return status;
   uint8_t* scratch = scratch_on_current_device(&status);
   if (!scratch) return status;
   return nvfp4_linear(x, M, K, w, w_scale, N, weight_scale_2, input_scale, bias, y, scratch,

@@ -55,6 +55,15 @@ def test_workspace_sizes():
     assert a.value == 0 and b.value >= M * K // 2 and c.value > b.value and c.value < ws
 
 
+def test_every_dit_layer_fits_the_noalloc_scratch():
+    # nvfp4_linear_noalloc holds 32 MiB of scratch per device; every M = 4096
+    # diffusion-transformer layer of the workloads fits in it
+    lib = _lib.load()
+    for K, N in [(3072, 3072), (3072, 9216), (3072, 12288), (12288, 3072)]:
+        need = lib.nvfp4_linear_workspace_size(4096, K, N)
+        assert 0 < need <= (32 << 20), (K, N, need)
+
+
 def test_argument_errors_before_device():
     lib = _lib.load()
     fake = 1 << 20          # aligned, never dereferenced: validation fails first

@@ -48,6 +48,44 @@ def test_noalloc_matches_nvfp4_linear_on_two_calls_in_a_row():
     assert q.read_device_status() == 0
 
 
+def test_noalloc_on_a_side_stream_after_a_first_call():
+    # a first call on the default stream, then one on a side stream: the scratch
+    # path gives the same bits as nvfp4_linear issued on that same stream
+    c = Nvfp4Case(512, 1024, 640, seed=33, bias=True)
+    d = c.device_args()
+    q.nvfp4_linear_noalloc(d["x"], d["w"], d["w_scale"], d["weight_scale_2"], d["input_scale"],
+                           bias=d["bias"])
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        ref = q.nvfp4_linear(d["x"], d["w"], d["w_scale"], d["weight_scale_2"], d["input_scale"],
+                             bias=d["bias"])
+        out = q.nvfp4_linear_noalloc(d["x"], d["w"], d["w_scale"], d["weight_scale_2"],
+                                     d["input_scale"], bias=d["bias"], y=_nan_output(c.M, c.N))
+    side.synchronize()
+    assert torch.equal(out, ref)
+    _, y64, T = c.reference()
+    check_linear(out, y64, T, "nvfp4_linear_noalloc on a side stream")
+    assert q.read_device_status() == 0
+
+
+def test_noalloc_checks_the_output_and_bias():
+    c = Nvfp4Case(64, 256, 128, seed=34)
+    d = c.device_args()
+    wrong_y = torch.empty((c.M, c.N + 8), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ValueError):
+        q.nvfp4_linear_noalloc(d["x"], d["w"], d["w_scale"], d["weight_scale_2"],
+                               d["input_scale"], y=wrong_y)
+    with pytest.raises(ValueError):
+        q.nvfp4_linear_noalloc(d["x"], d["w"], d["w_scale"], d["weight_scale_2"],
+                               d["input_scale"],
+                               y=torch.empty((c.M, c.N), dtype=torch.float32, device="cuda"))
+    with pytest.raises(ValueError):
+        q.nvfp4_linear_noalloc(d["x"], d["w"], d["w_scale"], d["weight_scale_2"],
+                               d["input_scale"],
+                               bias=torch.zeros(c.N - 1, dtype=torch.float32, device="cuda"))
+
+
 def test_noalloc_rejects_problems_beyond_its_scratch():
     M, K, N = 16384, 12288, 3072  # needs about 130 MB of scratch
     assert q.nvfp4_linear_workspace_size(M, K, N) > (32 << 20)
