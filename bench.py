@@ -5,19 +5,22 @@ N = 12288, bf16 in / bf16 out, synthetic seeded inputs.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One step = one nvfp4_linear call (prologue kernel + GEMM kernel). Each timed step
-is bracketed by CUDA events on the launching stream; a 256 MB buffer is written
-between steps (outside the events) so every step starts with a cold L2. Several
-GPUs run independent replicas (weak scaling; the layer has no exchange step);
-the time is the max over ranks.
+One step = one nvfp4_linear call (prologue kernel + GEMM kernel). Consecutive
+steps cycle through buffer sets (x, weights, y, workspace) that together hold at
+least four times the L2, so every step reads its operands from HBM; each timed
+step is bracketed by CUDA events on the launching stream and the value comes from
+the median step. Several GPUs run independent replicas (weak scaling; the layer has
+no exchange step); the time is the max over ranks.
 
-Prints one JSON line (rank 0). Extra keys: roofline of the GEMM kernel,
-cpu_baseline (the CPU oracle on a bounded sample), e2e (host buffers, copies
-inside the timed region), clocks sampled during the timed region,
-l2_rotating_graph (the same step timed over buffer sets four times the L2, replayed
-from a CUDA graph), and under "variants" the other layer shapes (flushed L2), the
-skinny / batched NVFP4 sweep and the W4A16 modulation sweep (both rotating-graph
-timed, against the HBM and FP4 rooflines).
+Prints one JSON line (rank 0). Extra keys: step_stats (median / mean / min / max
+and the host's enqueue time per step), the same step with a 256 MB flush before
+every step (l2_flushed), with warm L2 (l2_warm) and as CUDA graphs over the
+rotating sets (l2_rotating_graph); roofline of the GEMM kernel (with the SM clock
+the GEMM ran at and the dense FP4 peak at that clock); cpu_baseline (the CPU oracle
+on a bounded sample, its CPU model, and one-thread figures); e2e (host buffers,
+copies inside the timed region); clocks sampled during the run; and under
+"variants" the other layer shapes, the skinny / batched NVFP4 sweep and the W4A16
+modulation sweep (rotating-graph timed, against the HBM and FP4 rooflines).
 """
 import argparse
 import hashlib
@@ -308,23 +311,26 @@ class MlpBlock:
 
 
 def time_events(fn, steps, warmup, flush, stream):
-    """Mean device time (ms) of fn over `steps` calls, each bracketed by CUDA events
-    on `stream`, with an L2 flush (outside the events) before every call."""
+    """Device time (ms) of fn over `steps` calls, each bracketed by CUDA events on
+    `stream`, with `flush()` (if given) before every call, outside the events.
+    Returns (median, per-call times)."""
     import torch
     for _ in range(warmup):
-        flush()
+        if flush:
+            flush()
         fn()
     torch.cuda.synchronize()
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     for i in range(steps):
-        flush()
+        if flush:
+            flush()
         starts[i].record(stream)
         fn()
         ends[i].record(stream)
     torch.cuda.synchronize()
     times = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    return statistics.fmean(times), times
+    return statistics.median(times), times
 
 
 L2_BYTES = 126 << 20
@@ -522,19 +528,95 @@ def skinny_sweep(device, stream, peaks, steps):
     return out
 
 
+class _QuietStdout:
+    """Sends file descriptor 1 to /dev/null inside the block (library code that prints
+    from native code would otherwise break the single JSON line on stdout)."""
+
+    def __enter__(self):
+        sys.stdout.flush()
+        self._saved = os.dup(1)
+        self._null = os.open(os.devnull, os.O_WRONLY)
+        os.dup2(self._null, 1)
+        return self
+
+    def __exit__(self, *exc):
+        sys.stdout.flush()
+        os.dup2(self._saved, 1)
+        os.close(self._saved)
+        os.close(self._null)
+
+
+def prior_art_flashinfer(M, K, N, device, stream):
+    """Context only: the kernels the BFL page names for nvfp4 (FlashInfer's
+    nvfp4_quantize and mm_fp4), timed on this GPU on the same shape, over rotating
+    operand copies larger than L2 (one CUDA graph per cycle). Library code; none of
+    it is on this library's path. Returns a dict, or the reason it could not run."""
+    import torch
+    try:
+        import flashinfer
+    except Exception as e:  # pragma: no cover - depends on the image
+        return {"unavailable": f"flashinfer import failed: {type(e).__name__}"}
+    from synthetic import make_linear_inputs
+    inp = make_linear_inputs(M, K, N, seed=0)
+    x = inp.x.to(device)
+    w = inp.w.to(device)
+    # FlashInfer takes the reciprocal global scale: 448 * 6 / amax
+    gx = ((448.0 * 6.0) / x.float().abs().amax()).reshape(1).float()
+    gw = ((448.0 * 6.0) / w.float().abs().amax()).reshape(1).float()
+    alpha = (1.0 / (gx * gw)).float()
+    out = {"how": "FlashInfer nvfp4_quantize + mm_fp4 on the same shape; rotating copies, "
+                  "one CUDA graph per cycle, mean per call"}
+    try:
+        xq, xs = flashinfer.nvfp4_quantize(x, gx)
+        wq, ws = flashinfer.nvfp4_quantize(w, gw)
+        per = xq.numel() + xs.numel() + wq.numel() + ws.numel() + 2 * M * N
+        R = max(2, -(-ROTATION_BYTES // per))
+        sets = [(xq.clone(), xs.clone(), wq.clone(), ws.clone(),
+                 torch.empty(M, N, dtype=torch.bfloat16, device=device)) for _ in range(R)]
+        idx = [0]
+        for backend in ("cudnn", "cutlass"):
+            def gemm(backend=backend):
+                a, asf, b, bsf, o = sets[idx[0]]
+                idx[0] = (idx[0] + 1) % R
+                flashinfer.mm_fp4(a, b.T, asf, bsf.T, alpha, torch.bfloat16, out=o,
+                                  backend=backend)
+            try:
+                ms = time_graph_rotation(gemm, R, 10, stream)
+                out[f"mm_fp4_{backend}_us"] = ms * 1e3
+                out[f"mm_fp4_{backend}_tflops"] = nvfp4_flops(M, K, N) / (ms / 1e3) / 1e12
+            except Exception as e:
+                out[f"mm_fp4_{backend}_error"] = f"{type(e).__name__}: {str(e)[:120]}"
+        del sets
+        xsets = [x.clone() for _ in range(max(2, -(-ROTATION_BYTES // (2 * M * K))))]
+        qi = [0]
+
+        def quant():
+            xx = xsets[qi[0]]
+            qi[0] = (qi[0] + 1) % len(xsets)
+            flashinfer.nvfp4_quantize(xx, gx)
+        out["nvfp4_quantize_us"] = time_graph_rotation(quant, len(xsets), 10, stream) * 1e3
+        del xsets
+    except Exception as e:
+        out["error"] = f"{type(e).__name__}: {str(e)[:160]}"
+    torch.cuda.empty_cache()
+    return out
+
+
 def traffic_from_profiles(kernel_key: str):
-    """Per-launch DRAM bytes of a kernel from the committed ncu summary, or None
-    when the kernel source changed since the capture."""
+    """(per-launch DRAM bytes of a kernel from the committed ncu capture, note): the
+    bytes are None, with a note saying so, when there is no capture or the kernel's
+    sources changed since it was taken (the counters would describe another kernel)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)[kernel_key]
     except (OSError, ValueError, KeyError):
-        return None
+        return None, "no capture recorded in profiles/traffic.json"
     src_hash = source_hash(rec.get("sources", []))
     if src_hash != rec.get("source_sha1"):
-        return None
-    return rec.get("bytes_per_launch")
+        return None, ("stale: the kernel's sources changed since the ncu capture in "
+                      "profiles/traffic.json")
+    return rec.get("bytes_per_launch"), rec.get("note", "")
 
 
 def source_hash(files):
@@ -570,6 +652,47 @@ def oracle_rows_for(seconds, x, gx, wq, ws, gw, M):
     fixed = max(t_a - a * per_row, 0.0)
     rows = int((seconds - fixed) / per_row) // th * th
     return int(max(1, min(M, max(rows, th))))
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def oracle_single_thread():
+    """The oracle on one thread for the tiny layer (all of it) and the attention
+    projection with bias (a 32-row sample, extrapolated to 4096 rows)."""
+    import oracle
+    from synthetic import make_linear_inputs
+    saved = oracle.get_threads()
+    oracle.set_threads(1)
+    out = {}
+    try:
+        for name, (M, K, N, bias, rows) in {
+                "tiny_128x256x256": (128, 256, 256, False, 128),
+                "attn_proj_4096x3072x3072_bias": (4096, 3072, 3072, True, 32)}.items():
+            inp = make_linear_inputs(M, K, N, seed=0, with_bias=bias)
+            gw = oracle.nvfp4_global_scale(inp.w)
+            wq, ws = oracle.nvfp4_quantize(inp.w, gw)
+            gx = oracle.nvfp4_global_scale(inp.x)
+            b = None if inp.bias is None else inp.bias.numpy()
+            t0 = time.perf_counter()
+            xq, xs = oracle.nvfp4_quantize(inp.x[:rows], gx)
+            oracle.nvfp4_linear(xq, xs, wq, ws, gx, gw, b)
+            t = time.perf_counter() - t0
+            out[name] = {"tflops": nvfp4_flops(rows, K, N) / t / 1e12,
+                         "seconds_full_layer": t * M / rows,
+                         "sample": f"{rows} of {M} rows" + ("" if rows == M else
+                                                             ", time extrapolated by rows")}
+    finally:
+        oracle.set_threads(saved)
+    return out
 
 
 def cpu_oracle_sample(M, K, N, target_s=15.0):
@@ -656,71 +779,105 @@ def run_ours(args):
     flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
 
     def flush():
+        # write 256 MB (twice the L2), then read it back: the read evicts the dirty
+        # lines of the write, so their write-back happens here, outside the events
         flush_buf.fill_(1)
+        flush_buf.view(torch.int32).max()
+
+    flops = nvfp4_flops(M, K, N)
+    fp4_peak = peaks["bf16_tflops"] * NOMINAL_FP4_OVER_BF16
 
     # --------------------------------------------------- headline: timed steps
-    for _ in range(args.warmup):
-        flush()
-        layer.step()
-    torch.cuda.synchronize()
-    barrier(device)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    # Inputs larger than L2: consecutive steps cycle through R buffer sets (x,
+    # weights, y, workspace) that together hold at least four times the L2, so each
+    # step reads its operands from HBM, as a stack of distinct layers would. Each
+    # step is bracketed by CUDA events on the launching stream; the value is the
+    # median step. The clock sampler runs over the warm-up and the timed steps.
+    rot = Nvfp4Rotation(layer)
+    with ClockSampler(local, period_s=0.002) as clk:
+        for _ in range(args.warmup):
+            rot.step()
+        torch.cuda.synchronize()
+        barrier(device)
+        torch.cuda.synchronize()
         starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
         ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        t_host = time.perf_counter()
         for i in range(args.steps):
-            flush()
             starts[i].record(stream)
-            layer.step()
+            rot.step()
             ends[i].record(stream)
+        host_s = time.perf_counter() - t_host
         torch.cuda.synchronize()
     barrier(device)
     torch.cuda.synchronize()
-    local_ms = statistics.fmean(s.elapsed_time(e) for s, e in zip(starts, ends))
-    flops = nvfp4_flops(M, K, N)
+    step_times = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    local_ms = statistics.median(step_times)
     ms, value_flops = aggregate(local_ms, flops, world, device)
     value = value_flops / 1e12
+    mean_ms, _ = aggregate(statistics.fmean(step_times), flops, world, device)
     status = q.read_device_status()
+    gemm_cycles, gemm_ns = q.read_gemm_clock()     # the last timed step's GEMM
+    step_sm_mhz = gemm_cycles / gemm_ns * 1e3 if gemm_ns else None
 
-    # the same step with inputs larger than L2 instead of a flush: consecutive
-    # steps cycle through buffer sets four times the L2, replayed from a CUDA graph
-    # (device time only, no host launch gaps)
-    rot = Nvfp4Rotation(layer)
-    rot_ms = time_graph_rotation(rot.step, rot.R, max(3, min(args.steps // rot.R, 50)), stream)
-    rot_ms, rot_val = aggregate(rot_ms, flops, world, device)
+    # the same step timed two more ways: a 256 MB flush before every step (the
+    # operands come from HBM, Y's lines start clean), and warm L2 (the same
+    # buffers every step, no flush)
+    n_alt = max(20, min(args.steps, 200))
+    fl_ms, _ = time_events(layer.step, n_alt, 3, flush, stream)
+    warm_ms, _ = time_events(layer.step, n_alt, 3, None, stream)
+    fl_ms, fl_val = aggregate(fl_ms, flops, world, device)
+    warm_ms, warm_val = aggregate(warm_ms, flops, world, device)
+    # and as one CUDA graph per cycle of buffer sets (no host launch gaps at all)
+    graph_ms = time_graph_rotation(rot.step, rot.R, max(3, min(args.steps // rot.R, 50)), stream)
+    graph_ms, graph_val = aggregate(graph_ms, flops, world, device)
 
     # --------------------------------------------------- roofline of the GEMM kernel
-    fp4_peak = peaks["bf16_tflops"] * NOMINAL_FP4_OVER_BF16
+    # the GEMM alone, the prologue alone and the activation quantizer alone, each
+    # over the rotating buffer sets, one CUDA graph per cycle of sets (a launch of
+    # the short kernels takes less device time than the host needs to issue it, so
+    # call-by-call events would time the host)
     tile_bn, tile_cg = q.tile_config(M, N, K)
-    roof_steps = max(20, min(args.steps, 200))
-    layer.prologue()
-    gemm_ms, _ = time_events(layer.gemm, roof_steps, 3, flush, stream)
-    prol_ms, _ = time_events(layer.prologue, roof_steps, 3, flush, stream)
-    xq_buf = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
-    xs_buf = torch.empty((M, K // 16), dtype=torch.uint8, device=device)
-    quant_ms, _ = time_events(lambda: q.nvfp4_quantize_act(layer.x, layer.gx, xq_buf, xs_buf),
-                              roof_steps, 3, flush, stream)
+    reps = max(3, min(args.steps // rot.R, 50))
+    rot.prologue_all()
+    torch.cuda.synchronize()
+    gemm_ms = time_graph_rotation(rot.gemm, rot.R, reps, stream)
+    g_cycles, g_ns = q.read_gemm_clock()
+    gemm_sm_mhz = g_cycles / g_ns * 1e3 if g_ns else None
+    prol_ms = time_graph_rotation(rot.prologue, rot.R, reps, stream)
+    quant_ms = time_graph_rotation(rot.quantize_act, rot.R, reps, stream)
     quant_bytes = 2 * M * K + M * K // 2 + M * K // 16
     gemm_tflops = flops / (gemm_ms / 1e3) / 1e12
     prologue_bytes = 2 * M * K + M * K // 2 + M * K // 16 + 2 * (N * K // 16)
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    # dense FP4 MMA rate: 32768 flops per SM per clock (9 PF nominal at 1.855 GHz)
+    clock_peak = (sms * 32768 * gemm_sm_mhz * 1e6 / 1e12) if gemm_sm_mhz else None
+    traffic, traffic_note = traffic_from_profiles("nvfp4_gemm_mlp_up")
     roofline = {
         "kernel": f"qgemm_kernel<FP4, BN={tile_bn}, {'CTA pair' if tile_cg == 2 else 'one CTA'}> "
                   "(tcgen05 block-scaled FP4 GEMM)",
         "bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
         "frac": gemm_tflops / fp4_peak,
-        "traffic": traffic_from_profiles("nvfp4_gemm_mlp_up"),
+        "traffic": traffic,
+        "traffic_note": traffic_note,
         "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {NOMINAL_FP4_OVER_BF16} "
-                       "(nominal dense FP4:bf16 ratio)",
+                       "(nominal dense FP4:bf16 ratio), of measured",
         "algorithmic": "2*M*K*N flops per launch",
         "gemm_us": gemm_ms * 1e3,
+        "gemm_sm_mhz": gemm_sm_mhz,
+        "clock_derived_fp4_peak": clock_peak,
+        "frac_of_clock_derived_peak": gemm_tflops / clock_peak if clock_peak else None,
+        "clock_derived_note": f"{sms} SMs x 32768 flop/clk x the SM clock CTA 0 of the GEMM "
+                              "measured over its own run (ql_read_gemm_clock)",
+        "frac_of_nominal_9pf": gemm_tflops / 9000.0,
         "prologue_us": prol_ms * 1e3,
         "prologue_gbs": prologue_bytes / (prol_ms / 1e3) / 1e9,
         "prologue_hbm_frac": prologue_bytes / (prol_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
         "quantize_act_us": quant_ms * 1e3,
         "quantize_act_gbs": quant_bytes / (quant_ms / 1e3) / 1e9,
         "quantize_act_hbm_frac": quant_bytes / (quant_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
-        "frac_of_nominal_9pf": gemm_tflops / 9000.0,
         "step_frac_of_fp4_peak": value / world / fp4_peak,
+        "step_frac_of_nominal_9pf": value / world / 9000.0,
     }
 
     # --------------------------------------------------- e2e through the public API
@@ -811,31 +968,50 @@ def run_ours(args):
         torch.cuda.empty_cache()
         variants["nvfp4_skinny_sweep_K3072"] = skinny_sweep(device, stream, peaks, v_steps)
         variants["w4a16_modulation_sweep"] = w4a16_sweep(device, stream, peaks, v_steps)
+    if not args.no_prior_art:
+        with _QuietStdout():
+            variants["prior_art_flashinfer_mlp_up"] = prior_art_flashinfer(M, K, N, device,
+                                                                          stream)
 
     # --------------------------------------------------- CPU oracle baseline (rank 0, N=1)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tfl, cores, rows, sec = cpu_oracle_sample(M, K, N)
         cpu = {"value": tfl, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "cpu_model": cpu_model(),
                "sample": f"{rows} of {M} activation rows, all N={N}, K={K} (quantize + fp64 "
-                         f"contraction), {sec:.1f} s"}
+                         f"contraction), {sec:.1f} s",
+               "single_thread": oracle_single_thread()}
 
+    clocks = clk.summary()
+    clocks["window"] = "NVML samples every 2 ms over the warm-up and the timed steps"
+    clocks["gemm_sm_mhz_in_kernel"] = step_sm_mhz
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "e2m1xe2m1->f32 (bf16 in/out)", "data": "synthetic",
         "config": {"workload": "nvfp4_mlp_up M4096 K3072 N12288", **WORKLOAD,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "flushed (256 MB write) before every step, outside the events"},
+                   "l2": f"inputs larger than L2: {rot.R} buffer sets of "
+                         f"{rot.bytes_per_set / 1e6:.0f} MB (x, weights, y, workspace) cycled, "
+                         "one per step; value from the median step",
+                   "timing": "CUDA events around each step on the launching stream"},
         "frac_of_fp4_peak": value / world / fp4_peak,
-        "l2_rotating_graph": {"value": rot_val / 1e12, "ms_per_step": rot_ms,
-                              "how": f"{rot.R} buffer sets of {rot.bytes_per_set / 1e6:.0f} MB (x, "
-                                     "weights, y, workspace) cycled, one per step, all steps of a "
-                                     "cycle in one CUDA graph; mean over replays"},
+        "step_stats": {"median_ms": ms, "mean_ms": mean_ms,
+                       "min_ms": min(step_times), "max_ms": max(step_times),
+                       "host_us_per_step": host_s / args.steps * 1e6},
+        "l2_flushed": {"value": fl_val / 1e12, "ms_per_step": fl_ms,
+                       "how": "256 MB written then read before every step, outside the events; "
+                              f"median of {n_alt} steps"},
+        "l2_warm": {"value": warm_val / 1e12, "ms_per_step": warm_ms,
+                    "how": f"the same buffers every step, no flush; median of {n_alt} steps"},
+        "l2_rotating_graph": {"value": graph_val / 1e12, "ms_per_step": graph_ms,
+                              "how": "the rotating buffer sets, one CUDA graph per cycle of "
+                                     "sets; mean over replays"},
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "clocks": clk.summary(),
+        "clocks": clocks,
         "gpu_launches": 2 * args.steps,
         "device_status": status,
         "variants": variants,
@@ -907,6 +1083,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-variants", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prior-art", action="store_true",
+                    help="skip timing FlashInfer's NVFP4 kernels (context only)")
     ap.add_argument("--profile", choices=["step", "prologue", "gemm", "quant", "mlp_fused", "svdq",
                                           "fp8r_step", "fp8r_quant", "fp8r_gemm", "w4a16", "int4",
                                           "skinny_16_3072", "skinny_16_12288",

@@ -32,7 +32,7 @@ __all__ = [
     "nvfp4_linear_workspace_size", "nvfp4_linear_workspace_layout", "nvfp4_global_scale",
     "fp8r_quantize_rows", "fp8r_linear", "fp8r_linear_gemm", "fp8r_linear_workspace_size",
     "ql_encode_e4m3", "ql_encode_e2m1", "read_device_status", "set_fault_injection",
-    "set_tile_override", "tile_config",
+    "set_tile_override", "tile_config", "read_gemm_clock",
     "prepare_nvfp4_weight", "prepare_fp8r_weight", "QLinearError", "library_path",
 ]
 
@@ -541,6 +541,15 @@ def read_device_status() -> int:
     st = _lib.C.c_int(0)
     _lib.check("ql_read_device_status", _lib.load().ql_read_device_status(_lib.C.byref(st)))
     return st.value
+
+
+def read_gemm_clock() -> Tuple[int, int]:
+    """(SM cycles, nanoseconds) of the first CTA of the last GEMM launch on the current
+    device; cycles / ns is the SM clock in GHz that launch ran at."""
+    c, t = _lib.C.c_int64(0), _lib.C.c_int64(0)
+    _lib.check("ql_read_gemm_clock", _lib.load().ql_read_gemm_clock(_lib.C.byref(c),
+                                                                      _lib.C.byref(t)))
+    return c.value, t.value
 
 
 def set_fault_injection(enable: bool, timeout_ms: int = 0) -> None:

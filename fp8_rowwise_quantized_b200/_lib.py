@@ -60,6 +60,7 @@ SIGNATURES = {
     "ql_encode_e4m3": (C.c_int, [_f32p, _u8p, _i64, _vp]),
     "ql_encode_e2m1": (C.c_int, [_f32p, _u8p, _i64, _vp]),
     "ql_read_device_status": (C.c_int, [C.POINTER(C.c_int)]),
+    "ql_read_gemm_clock": (C.c_int, [C.POINTER(C.c_int64), C.POINTER(C.c_int64)]),
     "ql_set_fault_injection": (None, [C.c_int, C.c_int]),
     "ql_set_tile_override": (C.c_int, [C.c_int, C.c_int]),
     "ql_tile_config": (C.c_int, [C.c_int, _i64, _i64, _i64, C.POINTER(C.c_int),

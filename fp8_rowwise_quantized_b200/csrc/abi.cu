@@ -130,6 +130,18 @@ void ql_set_fault_injection(int enable, int timeout_ms) {
   g_timeout_ms.store(timeout_ms > 0 ? timeout_ms : 2000);
 }
 
+int ql_read_gemm_clock(int64_t* cycles, int64_t* ns) {
+  if (!cycles || !ns) return QL_ERR_INVALID_ARG;
+  int rc = check_device(nullptr);
+  if (rc != QL_OK) return rc;
+  unsigned long long c = 0, t = 0;
+  cudaError_t e = ql::read_gemm_clock(&c, &t);
+  if (e != cudaSuccess) return record(e, "ql_read_gemm_clock");
+  *cycles = static_cast<int64_t>(c);
+  *ns = static_cast<int64_t>(t);
+  return QL_OK;
+}
+
 int ql_read_device_status(int* status) {
   if (!status) return QL_ERR_INVALID_ARG;
   int dev = 0;

@@ -39,6 +39,12 @@
 
 namespace ql {
 
+// SM clock seen by the GEMM: CTA 0 of every GEMM launch stores its elapsed SM
+// cycles (%clock64) and nanoseconds (%globaltimer) from set-up to teardown, so
+// the clock the tensor cores ran at under the kernel's own load can be read back
+// (it is below the idle boost clock when the part runs at its power limit).
+__device__ unsigned long long g_gemm_clock[2];
+
 namespace {
 
 constexpr int kRowsPerCta = 128;
@@ -508,6 +514,11 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
   const int group = (CG == 2) ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
   const int ngroups = (CG == 2) ? static_cast<int>(nclusters_x()) : static_cast<int>(gridDim.x);
   const uint64_t deadline = globaltimer_ns() + args.timeout_ns;
+  unsigned long long clk_cycles0 = 0, clk_ns0 = 0;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    asm volatile("mov.u64 %0, %%clock64;" : "=l"(clk_cycles0));
+    clk_ns0 = globaltimer_ns();
+  }
 
   if (threadIdx.x == 0) {
     prefetch_tmap(&tmap_a);
@@ -1057,6 +1068,12 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
   // ------------------------------------------------------------ teardown
   tc_fence_before();
   __syncthreads();
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    unsigned long long c1;
+    asm volatile("mov.u64 %0, %%clock64;" : "=l"(c1));
+    g_gemm_clock[0] = c1 - clk_cycles0;
+    g_gemm_clock[1] = globaltimer_ns() - clk_ns0;
+  }
   if constexpr (CG == 2) cluster_sync_all();  // no peer accesses this CTA's memory any more
   if constexpr (FUSED) {
     // this CTA is done with the sync words; the last CTA out resets them
@@ -1278,6 +1295,14 @@ namespace {
 std::atomic<int> g_force_bn{0};
 std::atomic<int> g_force_cg{0};
 }  // namespace
+
+cudaError_t read_gemm_clock(unsigned long long* cycles, unsigned long long* ns) {
+  unsigned long long v[2] = {0, 0};
+  const cudaError_t e = cudaMemcpyFromSymbol(v, g_gemm_clock, sizeof(v));
+  *cycles = v[0];
+  *ns = v[1];
+  return e;
+}
 
 bool set_tile_override(int bn, int cg) {
   if (bn == 0) {

@@ -61,6 +61,9 @@ struct GemmProblem {
 // a slab (the GELU-quantize epilogue).
 GemmConfig choose_config(bool fp4, int64_t M, int64_t N, int64_t K, bool whole_buffers = false);
 bool set_tile_override(int bn, int cg);  // bn == 0 restores the automatic choice
+// Elapsed SM cycles and nanoseconds of CTA 0 of the last GEMM launch on the current
+// device (synchronous copy from the device).
+cudaError_t read_gemm_clock(unsigned long long* cycles, unsigned long long* ns);
 cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream);
 
 cudaError_t launch_nvfp4_quantize_rowmajor(const void* x, int64_t M, int64_t K, const float* g,

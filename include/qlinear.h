@@ -357,6 +357,16 @@ int ql_encode_e2m1(const float* in, uint8_t* out, int64_t n, ql_stream_t stream)
  * ql_read_device_status stores the word in *status (host pointer) and clears it. */
 int ql_read_device_status(int* status);
 
+/* The SM clock a GEMM launch ran at: elapsed SM cycles (*cycles) and nanoseconds
+ * (*ns) of the first CTA of the most recent NVFP4 or fp8r GEMM launch on the
+ * current device (the INT4 GEMM does not record it), from its set-up to its
+ * teardown; cycles / ns is that CTA's mean SM clock in GHz. Host pointers;
+ * synchronises the device; both 0 before the first launch. No counterpart on the
+ * pages: a measurement aid (the part lowers its clock under a heavy tensor-core
+ * load, so the dense peak at that clock is the relevant one). QL_ERR_INVALID_ARG
+ * for null pointers. */
+int ql_read_gemm_clock(int64_t* cycles, int64_t* ns);
+
 /* Test hook: while set (nonzero), the next GEMM launches start with one wait on a
  * barrier that nothing completes, so the bounded-wait path runs and reports
  * QL_ERR_TIMEOUT through the status word. `timeout_ms` bounds every wait of the
