@@ -173,9 +173,11 @@ int nvfp4_quantize_act(const void* x, int64_t M, int64_t K, const float* input_s
 
 size_t nvfp4_linear_workspace_size(int64_t M, int64_t K, int64_t N) {
   if (!nvfp4_shape_ok(M, K, N)) return 0;
-  // large enough for the weight-scale layout of every tile width
+  // large enough for the weight-scale layout of every tile width the call may use
+  // (the narrow widths of the skinny kernels only when M <= 64)
   size_t need = 0;
-  for (int bn : {128, 192, 224, 256}) {
+  for (int bn : {64, 96, 128, 192, 224, 256}) {
+    if (bn < 128 && M > 64) continue;
     const size_t t = ql::nvfp4_workspace(M, K, N, bn).total;
     need = t > need ? t : need;
   }
@@ -227,7 +229,7 @@ static int nvfp4_gemm_impl(int64_t M, int64_t K, const uint8_t* w, int64_t N,
                            const float* bias, void* y, const void* workspace,
                            size_t workspace_bytes, ql_stream_t stream, bool pdl,
                            const void* lr_act = nullptr, const void* lr_up = nullptr,
-                           int lr_rank = 0) {
+                           int lr_rank = 0, const uint8_t* w_scale_rowmajor = nullptr) {
   if (!w || !weight_scale_2 || !input_scale || !y || M <= 0 || N <= 0 || K <= 0)
     return QL_ERR_INVALID_ARG;
   if (!nvfp4_shape_ok(M, K, N)) return fail_shape("nvfp4: needs K >= 32 and K % 32 == 0");
@@ -245,6 +247,7 @@ static int nvfp4_gemm_impl(int64_t M, int64_t K, const uint8_t* w, int64_t N,
   p.fp4 = true;
   p.bn = bn;
   p.cg = cfg.cg;
+  p.arows = cfg.arows;
   p.M = M;
   p.N = N;
   p.K = K;
@@ -263,6 +266,7 @@ static int nvfp4_gemm_impl(int64_t M, int64_t K, const uint8_t* w, int64_t N,
   p.lr_act = lr_act;
   p.lr_up = lr_up;
   p.lr_rank = lr_rank;
+  if (cfg.arows > 0) p.w_scale = w_scale_rowmajor;  // skinny: scales laid out in the GEMM
   cudaError_t e = ql::launch_gemm(p, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? QL_OK : record(e, "nvfp4 gemm launch");
 }
@@ -340,6 +344,19 @@ int nvfp4_linear(const void* x, int64_t M, int64_t K, const uint8_t* w, const ui
     return QL_ERR_ALIGN;
   if (!workspace || workspace_bytes < nvfp4_linear_workspace_size(M, K, N)) return QL_ERR_WORKSPACE;
   if (!aligned16(workspace)) return QL_ERR_ALIGN;
+  if (ql::choose_config(true, M, N, K).arows > 0) {
+    // skinny layer: the prologue quantizes the activations only and lets the GEMM
+    // launch at once; the GEMM streams the weights meanwhile and lays out their
+    // scales itself, then waits for the activations
+    int rc = check_device(nullptr);
+    if (rc != QL_OK) return rc;
+    const cudaError_t e = ql::launch_nvfp4_prologue(
+        x, M, K, w_scale, N, ql::choose_config(true, M, N, K).bn, input_scale,
+        static_cast<uint8_t*>(workspace), reinterpret_cast<cudaStream_t>(stream), false);
+    if (e != cudaSuccess) return record(e, "nvfp4_linear prologue");
+    return nvfp4_gemm_impl(M, K, w, N, weight_scale_2, input_scale, bias, y, workspace,
+                           workspace_bytes, stream, true, nullptr, nullptr, 0, w_scale);
+  }
   int rc = nvfp4_linear_prologue(x, M, K, w_scale, N, input_scale, workspace, workspace_bytes,
                                  stream);
   if (rc != QL_OK) return rc;
@@ -365,7 +382,7 @@ int nvfp4_linear_single_launch(const void* x, int64_t M, int64_t K, const uint8_
   int dev = 0;
   int rc = check_device(&dev);
   if (rc != QL_OK) return rc;
-  const ql::GemmConfig cfg = ql::choose_config(true, M, N, K);
+  const ql::GemmConfig cfg = ql::choose_config(true, M, N, K, false, false);
   const ql::Nvfp4Workspace L = ql::nvfp4_workspace(M, K, N, cfg.bn);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   ql::GemmProblem p{};

@@ -93,13 +93,23 @@ struct GemmArgs {
   // tile has fewer valid rows (rows past it keep stale shared memory, which only
   // reaches accumulator rows that are never stored; their scale atoms are zero)
   int a_box_rows;
+  // skinny kernels: weight scales taken row-major from w_scale ([N, K/16], ks_bytes
+  // per row; 16-byte loads when sfb_vec16) instead of atoms in the workspace
+  int sfb_rowmajor;
+  int ks_bytes;
+  int sfb_vec16;
 };
 
-template <bool FP4, int BN, int CG>
+// AROWS: rows of A a pipeline stage holds. 128 for every tile, or 16 / 32 / 64 for
+// the skinny kernels (M <= AROWS, one CTA per tile): the MMA still runs M = 128
+// and reads past the stage's rows into neighbouring shared memory, which only
+// reaches accumulator rows >= M (never stored); the stage being smaller, more
+// stages fit, so more weight bytes are in flight per SM.
+template <bool FP4, int BN, int CG, int AROWS = kRowsPerCta>
 struct Cfg {
   static constexpr int NA = (BN + 127) / 128;                        // 128-row scale atoms of B
   static constexpr int B_ROWS = BN / CG;                             // B rows held by one CTA
-  static constexpr int A_BYTES = kRowsPerCta * 128;
+  static constexpr int A_BYTES = AROWS * 128;
   static constexpr int B_BYTES = B_ROWS * 128;
   static constexpr int SFA_BYTES = FP4 ? 4 * kSfAtomBytes : 0;       // 4 K-groups x 1 atom
   static constexpr int SFB_BYTES = FP4 ? 4 * NA * kSfAtomBytes : 0;  // 4 K-groups x NA atoms
@@ -109,7 +119,8 @@ struct Cfg {
   static constexpr int COLVEC_BYTES = 2 * 2 * 256 * 4;  // bias + column scales, 2 tiles deep
   static constexpr int RESERVED = 1024 /*alignment*/ + 1024 /*barriers*/ + EPI_BYTES + COLVEC_BYTES;
   static constexpr int STAGES_FIT = (kSmemLimit - RESERVED) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+  static constexpr int MAX_STAGES = AROWS < kRowsPerCta ? 12 : 8;
+  static constexpr int STAGES = STAGES_FIT > MAX_STAGES ? MAX_STAGES : STAGES_FIT;
   static constexpr int SF_COLS = FP4 ? 16 + 4 * NA * 4 : 0;
   // Two accumulator buffers. When two full BN-column buffers and the scale columns
   // do not fit in TMEM (BN = 256 with scales), the second buffer starts 64 columns
@@ -138,6 +149,8 @@ struct Cfg {
   static constexpr int SLAB = (BN % 64 == 0) ? 64 : 32;
   static constexpr int NSLAB = BN / SLAB;
   static_assert(CG == 1 || CG == 2, "one SM or a CTA pair");
+  static_assert(AROWS == kRowsPerCta || (CG == 1 && AROWS % 16 == 0 && AROWS <= 64),
+                "skinny stages: one CTA per tile, 16 / 32 / 64 rows of A");
   static_assert(B_ROWS % 8 == 0, "B half must be whole 8-row core groups");
 };
 
@@ -466,23 +479,31 @@ constexpr int kModeGeluQuant = 2;
 // quadrant, taking alternate slabs).
 template <int MODE>
 constexpr int epi_warps() { return MODE == kModeGeluQuant ? 8 : 4; }
-template <int MODE>
+// The skinny kernels (AROWS < 128) add one warp after the epilogue warps: it lays out
+// the weight scales of each stage in shared memory from the row-major scales.
+template <int MODE, int AROWS = kRowsPerCta>
 constexpr int block_threads() {
-  return MODE == kModeSingleLaunch ? kThreadsFused : 64 + 32 * epi_warps<MODE>();
+  return MODE == kModeSingleLaunch ? kThreadsFused
+                                   : 64 + 32 * epi_warps<MODE>() + (AROWS < kRowsPerCta ? 32 : 0);
 }
 
-template <bool FP4, int BN, int CG, int MODE>
-__global__ void __launch_bounds__(block_threads<MODE>(), 1)
+template <bool FP4, int BN, int CG, int MODE, int AROWS = kRowsPerCta>
+__global__ void __launch_bounds__(block_threads<MODE, AROWS>(), 1)
 qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
              const __grid_constant__ CUtensorMap tmap_sfa,
              const __grid_constant__ CUtensorMap tmap_sfb,
              const __grid_constant__ CUtensorMap tmap_y,
              const __grid_constant__ CUtensorMap tmap_lra,
              const __grid_constant__ CUtensorMap tmap_lrb, const GemmArgs args) {
-  using C = Cfg<FP4, BN, CG>;
+  using C = Cfg<FP4, BN, CG, AROWS>;
   constexpr bool FUSED = MODE == kModeSingleLaunch;
   constexpr bool GQ = MODE == kModeGeluQuant;
+  constexpr bool SKINNY = AROWS < kRowsPerCta;
   constexpr int EPI_WARPS = epi_warps<MODE>();
+  constexpr int SF_WARP = 2 + EPI_WARPS;  // skinny kernels: the weight-scale warp
+  // skinny kernels given the row-major weight scales: SF_WARP writes each stage's
+  // scale atoms (no TMA load of them) and is a second arrival on the stage's barrier
+  const bool sfb_rm = SKINNY && args.sfb_rowmajor != 0;
   constexpr int EPI_THREADS = 32 * EPI_WARPS;
   constexpr int EPI_HALVES = EPI_WARPS / 4;  // warps per TMEM lane quadrant
   static_assert(!GQ || !C::OVERLAP, "two warps per quadrant need whole accumulator buffers");
@@ -525,7 +546,7 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     prefetch_tmap(&tmap_b);
     if constexpr (FP4) {
       prefetch_tmap(&tmap_sfa);
-      prefetch_tmap(&tmap_sfb);
+      if (!sfb_rm) prefetch_tmap(&tmap_sfb);
     }
     if (args.use_tma_store) prefetch_tmap(&tmap_y);
     if (args.lr_k16 > 0) {
@@ -533,7 +554,7 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
       prefetch_tmap(&tmap_lrb);
     }
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full_bar[s], 1);
+      mbar_init(&full_bar[s], sfb_rm ? 2 : 1);
       mbar_init(&empty_bar[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -549,6 +570,18 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
       }
     }
     fence_mbar_init();
+    if (SKINNY && args.wait_prior_grid && !args.inject_fault && group < args.total_tiles) {
+      // skinny kernels: the weight loads of the first stages go out now, before the
+      // TMEM allocation and the block's first barrier (the producer issues the rest)
+      int m_blk, n_blk;
+      tile_coords(group, args, m_blk, n_blk);
+      const int pre = args.num_k_tiles < C::STAGES ? args.num_k_tiles : C::STAGES;
+      const uint32_t kTx = C::A_BYTES + C::B_BYTES + C::SFA_BYTES + (sfb_rm ? 0u : C::SFB_BYTES);
+      for (int kt = 0; kt < pre; ++kt) {
+        mbar_arrive_expect_tx(&full_bar[kt], kTx);
+        tma_load_2d(smem_b + kt * C::B_BYTES, &tmap_b, &full_bar[kt], kt * 128, n_blk * BN);
+      }
+    }
   }
   if (warp == 1) {
     if constexpr (CG == 2) {
@@ -570,8 +603,11 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
       (CG == 2) ? map_to_cta(smem_u32(tempty_bar), 0) : smem_u32(tempty_bar);
 
   // Everything above overlaps the tail of the previous kernel on the stream;
-  // global inputs are read only after it has completed.
-  if (args.wait_prior_grid) grid_dependency_wait();
+  // global inputs are read only after it has completed. In the skinny kernels only
+  // the producer waits, and only after it has started the weight loads (the weights
+  // and their scales do not come from the previous kernel; the MMA and epilogue
+  // warps read nothing it writes).
+  if (args.wait_prior_grid && !SKINNY) grid_dependency_wait();
 
 
   bool run = true;
@@ -676,7 +712,106 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     if (!*s_barrier_ok) run = false;
   }
 
-  if (run && warp == 0) {
+  if (SKINNY && run && warp == 0) {
+    // ------------------------------------------------------------ TMA producer (skinny)
+    // As below, one CTA per tile; on the first tile the weight loads of the first
+    // stages go out before the wait for the kernel that writes the activations.
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    int issued = 0;
+    bool waited = !args.wait_prior_grid;
+    const uint32_t kTx = C::A_BYTES + C::B_BYTES + C::SFA_BYTES + (sfb_rm ? 0u : C::SFB_BYTES);
+    for (int tile = group; ok && tile < args.total_tiles; tile += ngroups) {
+      int m_blk, n_blk;
+      tile_coords(tile, args, m_blk, n_blk);
+      const int a_row = m_blk * C::TILE_M;
+      const int b_row = n_blk * BN;
+      int pre = 0;
+      if (!waited) {
+        // stages 0 .. pre-1 of a fresh pipeline: their weight loads went out during
+        // the set-up (thread 0); the rest of each stage follows the wait
+        pre = args.num_k_tiles < C::STAGES ? args.num_k_tiles : C::STAGES;
+        grid_dependency_wait();
+        waited = true;
+        for (int kt = 0; kt < pre; ++kt) {
+          if (elect_one()) {
+            tma_load_2d(smem_a + kt * C::A_BYTES, &tmap_a, &full_bar[kt], kt * 128, a_row);
+            if constexpr (FP4) {
+              tma_load_2d(smem_sfa + kt * C::SFA_BYTES, &tmap_sfa, &full_bar[kt], 0,
+                          static_cast<int>(static_cast<int64_t>(m_blk) * args.kg + kt * 4));
+              if (!sfb_rm)
+                tma_load_2d(smem_sfb + kt * C::SFB_BYTES, &tmap_sfb, &full_bar[kt], 0,
+                            static_cast<int>((static_cast<int64_t>(n_blk) * args.kg + kt * 4) *
+                                             C::NA));
+            }
+          }
+          __syncwarp();
+        }
+        issued = pre;
+        stage = pre == C::STAGES ? 0 : pre;
+        phase = pre == C::STAGES ? 1u : 0u;
+      }
+      for (int kt = pre; kt < args.num_k_tiles; ++kt) {
+        if (!warp_wait_bounded(&empty_bar[stage], phase ^ 1u, deadline)) {
+          ok = false;
+          break;
+        }
+        if (elect_one()) {
+          mbar_arrive_expect_tx(&full_bar[stage], kTx);
+          tma_load_2d(smem_a + stage * C::A_BYTES, &tmap_a, &full_bar[stage], kt * 128, a_row);
+          tma_load_2d(smem_b + stage * C::B_BYTES, &tmap_b, &full_bar[stage], kt * 128, b_row);
+          if constexpr (FP4) {
+            tma_load_2d(smem_sfa + stage * C::SFA_BYTES, &tmap_sfa, &full_bar[stage], 0,
+                        static_cast<int>(static_cast<int64_t>(m_blk) * args.kg + kt * 4));
+            if (!sfb_rm)
+              tma_load_2d(smem_sfb + stage * C::SFB_BYTES, &tmap_sfb, &full_bar[stage], 0,
+                          static_cast<int>((static_cast<int64_t>(n_blk) * args.kg + kt * 4) *
+                                           C::NA));
+          }
+        }
+        __syncwarp();
+        ++issued;
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (ok && args.lr_k16 > 0) {
+        // the low-rank branch's operands (AROWS rows of them), as in the kernels below
+        if (!warp_wait_bounded(&empty_bar[stage], phase ^ 1u, deadline)) {
+          ok = false;
+          break;
+        }
+        if (elect_one()) {
+          mbar_arrive_expect_tx(&full_bar[stage], C::A_BYTES + C::B_BYTES);
+          tma_load_2d(smem_a + stage * C::A_BYTES, &tmap_lra, &full_bar[stage], 0, a_row);
+          tma_load_2d(smem_b + stage * C::B_BYTES, &tmap_lrb, &full_bar[stage], 0, b_row);
+        }
+        __syncwarp();
+        ++issued;
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!waited) grid_dependency_wait();  // no tile: still ordered after the previous kernel
+    if (!ok) {
+      record_timeout(args.status);
+      const uint64_t drain_deadline = globaltimer_ns() + 100000000ull;
+      const int n = issued < C::STAGES ? issued : C::STAGES;
+      int st = stage;
+      uint32_t ph = phase;
+      for (int i = 0; i < n; ++i) {
+        if (--st < 0) {
+          st = C::STAGES - 1;
+          ph ^= 1u;
+        }
+        mbar_wait_bounded(&full_bar[st], ph, drain_deadline);
+      }
+    }
+  } else if (run && warp == 0) {
     // ------------------------------------------------------------ TMA producer
     int stage = 0;
     uint32_t phase = 0;
@@ -975,8 +1110,16 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
       if constexpr (!FP4) row_scale = (m < args.M) ? __ldg(args.scale_a + m) : 0.0f;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * C::ACC_STRIDE);
+      // a warp whose 32 rows all lie past M has nothing to store (the GELU-quantize
+      // epilogue still writes their zero scales): hand the buffer back at once
+      const bool rows_out = !GQ && row0 >= args.M;
+      if (rows_out) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(tempty_bar0 + bi * 8u);
+      }
 #pragma unroll 1
-      for (int it = 0; it < C::NSLAB; ++it) {
+      for (int it = 0; it < (rows_out ? 0 : C::NSLAB); ++it) {
         if (EPI_HALVES > 1 && it % EPI_HALVES != half) continue;  // warp-uniform
         // slab order: with shared slabs, buffer 0 drains its last slab (the shared
         // one) first; otherwise slabs go in order
@@ -1063,6 +1206,69 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
       if (C::OVERLAP || acc == 0) acc_phase ^= 1u;
     }
     if (lane == 0) bulk_wait_group_all();  // outstanding stores complete before exit
+  } else if (SKINNY && run && warp == SF_WARP && sfb_rm) {
+    // ------------------------------------------------------------ weight scales (skinny)
+    // Per stage: the 16 scales of each of the tile's BN weight rows for the stage's
+    // K tile (row-major [N, K/16], 16 bytes per row), rearranged into the 4 atoms
+    // the MMA's scale copies read (atom g, line l: group g of rows l, l+32, l+64,
+    // l+96); rows past the tile or N are zero. Lane l holds rows l + 32 j. The
+    // loads of a stage go out before the wait for its slot.
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    const int64_t ks = args.ks_bytes;
+    for (int tile = group; ok && tile < args.total_tiles; tile += ngroups) {
+      int m_blk, n_blk;
+      tile_coords(tile, args, m_blk, n_blk);
+      for (int kt = 0; kt < args.num_k_tiles; ++kt) {
+        uint4 v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int nn = lane + 32 * j;
+          const int64_t n = static_cast<int64_t>(n_blk) * BN + nn;
+          v[j] = make_uint4(0u, 0u, 0u, 0u);
+          if (nn < BN && n < args.N) {
+            const uint8_t* src = args.w_scale + n * ks + kt * 16;
+            if (args.sfb_vec16) {
+              v[j] = __ldg(reinterpret_cast<const uint4*>(src));
+            } else {
+              uint32_t w[4] = {0u, 0u, 0u, 0u};
+              for (int b = 0; b < 16; ++b)
+                if (kt * 16 + b < ks) w[b >> 2] |= static_cast<uint32_t>(__ldg(src + b)) << (8 * (b & 3));
+              v[j] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          }
+        }
+        if (!warp_wait_bounded(&empty_bar[stage], phase ^ 1u, deadline)) {
+          ok = false;
+          break;
+        }
+        uint8_t* ssb = smem_sfb + stage * C::SFB_BYTES;
+        *reinterpret_cast<uint4*>(ssb + 0 * kSfAtomBytes + lane * 16) = make_uint4(v[0].x, v[1].x, v[2].x, v[3].x);
+        *reinterpret_cast<uint4*>(ssb + 1 * kSfAtomBytes + lane * 16) = make_uint4(v[0].y, v[1].y, v[2].y, v[3].y);
+        *reinterpret_cast<uint4*>(ssb + 2 * kSfAtomBytes + lane * 16) = make_uint4(v[0].z, v[1].z, v[2].z, v[3].z);
+        *reinterpret_cast<uint4*>(ssb + 3 * kSfAtomBytes + lane * 16) = make_uint4(v[0].w, v[1].w, v[2].w, v[3].w);
+        fence_proxy_async_shared();  // the MMA thread's scale copies read these bytes
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full_bar[stage]);
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (ok && args.lr_k16 > 0) {  // the low-rank stage needs this warp's arrival too
+        if (!warp_wait_bounded(&empty_bar[stage], phase ^ 1u, deadline)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) mbar_arrive(&full_bar[stage]);
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok) record_timeout(args.status);
   }
 
   // ------------------------------------------------------------ teardown
@@ -1134,11 +1340,12 @@ bool encode_2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, uin
 
 namespace {
 
-template <bool FP4, int BN, int CG, int MODE>
+template <bool FP4, int BN, int CG, int MODE, int AROWS = kRowsPerCta>
 cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
-  using Cf = Cfg<FP4, BN, CG>;
+  using Cf = Cfg<FP4, BN, CG, AROWS>;
   constexpr bool FUSED = MODE == kModeSingleLaunch;
-  auto kern = qgemm_kernel<FP4, BN, CG, MODE>;
+  auto kern = qgemm_kernel<FP4, BN, CG, MODE, AROWS>;
+  if (AROWS < kRowsPerCta && p.M > AROWS) return cudaErrorInvalidValue;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -1165,7 +1372,8 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
   // A / B: uint8 rows of K* bytes, boxes of [rows, 128 bytes], 128-byte swizzle; a
   // lone CTA with fewer than 128 rows of A loads only those (whole 8-row swizzle
   // atoms), the plain FP4 mode only (its A scale atoms zero the rows past M)
-  const int a_box_rows = (CG == 1 && FP4 && MODE == kModePlain && p.M < kRowsPerCta)
+  const int a_box_rows = AROWS < kRowsPerCta ? AROWS
+                         : (CG == 1 && FP4 && MODE == kModePlain && p.M < kRowsPerCta)
                              ? static_cast<int>((p.M + 7) / 8 * 8)
                              : kRowsPerCta;
   if (!encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.a, k_bytes, p.M, k_bytes, 128,
@@ -1175,6 +1383,7 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
     return cudaErrorInvalidValue;
   const int64_t kg = sf_kgroups(p.K);
+  const bool sfb_rm = AROWS < kRowsPerCta && FP4 && MODE == kModePlain && p.w_scale != nullptr;
   if (FP4) {
     // scale atoms as rows of 128 32-bit words; one stage = 4 (A) or 4 * NA (B) atoms
     const int64_t a_atoms = ceil_div64(p.M, kRowsPerCta) * kg;
@@ -1182,9 +1391,10 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
     if (!encode_2d(&tsa, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.sfa, 128, a_atoms, kSfAtomBytes, 128, 4,
                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
       return cudaErrorInvalidValue;
-    if (!encode_2d(&tsb, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.sfb, 128, b_atoms, kSfAtomBytes,
-                          128, 4 * Cf::NA, CU_TENSOR_MAP_SWIZZLE_NONE,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B)) {
+    if (!sfb_rm &&
+        !encode_2d(&tsb, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.sfb, 128, b_atoms, kSfAtomBytes,
+                   128, 4 * Cf::NA, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B)) {
       return cudaErrorInvalidValue;
     }
   }
@@ -1201,7 +1411,7 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
     // bf16 [rows, r] with 128-byte boxes of 64 elements: columns r .. 63 read as zeros
     if (p.lr_rank > 64 || p.lr_rank % 8 != 0 || !p.lr_act || !p.lr_up ||
         !encode_2d(&tla, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.lr_act, p.lr_rank, p.M,
-                   p.lr_rank * 2, 64, kRowsPerCta, CU_TENSOR_MAP_SWIZZLE_128B,
+                   p.lr_rank * 2, 64, AROWS, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
         !encode_2d(&tlb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.lr_up, p.lr_rank, p.N,
                    p.lr_rank * 2, 64, Cf::B_ROWS, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -1211,6 +1421,12 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
 
   GemmArgs a{};
   a.a_box_rows = a_box_rows;
+  if (sfb_rm) {
+    a.sfb_rowmajor = 1;
+    a.w_scale = p.w_scale;
+    a.ks_bytes = static_cast<int>(p.K / 16);
+    a.sfb_vec16 = (p.K % 256 == 0 && (reinterpret_cast<uintptr_t>(p.w_scale) & 15) == 0) ? 1 : 0;
+  }
   a.lr_k16 = lowrank ? (p.lr_rank + 15) / 16 : 0;
   a.M = static_cast<int>(p.M);
   a.N = static_cast<int>(p.N);
@@ -1247,7 +1463,7 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
   }
 
   cudaLaunchConfig_t cfg{};
-  cfg.blockDim = dim3(block_threads<MODE>());
+  cfg.blockDim = dim3(block_threads<MODE, AROWS>());
   cfg.dynamicSmemBytes = Cf::SMEM;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
@@ -1310,19 +1526,49 @@ bool set_tile_override(int bn, int cg) {
     g_force_cg.store(0);
     return true;
   }
-  if ((bn != 128 && bn != 192 && bn != 224 && bn != 256) || (cg != 1 && cg != 2)) return false;
+  if ((bn != 64 && bn != 96 && bn != 128 && bn != 192 && bn != 224 && bn != 256) ||
+      (cg != 1 && cg != 2) || (bn < 128 && cg != 1))
+    return false;
   g_force_cg.store(cg);
   g_force_bn.store(bn);
   return true;
 }
 
-GemmConfig choose_config(bool fp4, int64_t M, int64_t N, int64_t K, bool whole_buffers) {
+// Rows of A per pipeline stage of the skinny FP4 kernels for M rows (0: none).
+static int skinny_rows(bool fp4, int64_t M, bool whole_buffers) {
+  if (!fp4 || whole_buffers || M > 64) return 0;
+  return M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+}
+
+GemmConfig choose_config(bool fp4, int64_t M, int64_t N, int64_t K, bool whole_buffers,
+                         bool allow_skinny) {
   GemmConfig c{};
+  const int sk = skinny_rows(fp4, M, whole_buffers || !allow_skinny);
   if (g_force_bn.load() != 0) {
     c.bn = g_force_bn.load();
     c.cg = g_force_cg.load();
     if (whole_buffers && c.bn == 256) c.bn = 224;
+    // skinny stages with one CTA per tile of at most 128 columns; narrower tiles
+    // exist only as skinny kernels
+    c.arows = (c.cg == 1 && c.bn <= 128) ? sk : 0;
+    if (c.bn < 128 && c.arows == 0) c.bn = 128;
     return c;
+  }
+  // Skinny layers (M <= 64, FP4): one CTA per tile with stages holding only 16 / 32 /
+  // 64 rows of A, and the narrowest tile width that keeps the tiles in one wave of
+  // 148 SMs (the weight streams through as many SMs as possible).
+  c.arows = sk;
+  if (c.arows > 0) {
+    c.cg = 1;
+    c.bn = 256;
+    for (int bn : {64, 96, 128, 192, 224, 256}) {
+      if (ceil_div64(N, bn) <= 148) {
+        c.bn = bn;
+        break;
+      }
+    }
+    if (c.bn > 128) c.arows = 0;  // wide tiles: the ordinary kernels
+    if (c.arows > 0) return c;
   }
   // CTA pairs once there are two 128-row blocks to pair. Tile width from a cost
   // model fitted to B200 measurements: waves over the resident groups x (K steps
@@ -1379,6 +1625,22 @@ cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream) {
     QL_FCASE(224, 2)
     QL_FCASE(256, 2)
 #undef QL_FCASE
+    return cudaErrorInvalidValue;
+  }
+  if (p.arows > 0) {
+    if (!p.fp4 || p.cg != 1) return cudaErrorInvalidValue;
+#define QL_SCASE(BN_, AR_) \
+  if (p.bn == BN_ && p.arows == AR_) return launch_typed<true, BN_, 1, kModePlain, AR_>(p, stream);
+    QL_SCASE(64, 16)
+    QL_SCASE(64, 32)
+    QL_SCASE(64, 64)
+    QL_SCASE(96, 16)
+    QL_SCASE(96, 32)
+    QL_SCASE(96, 64)
+    QL_SCASE(128, 16)
+    QL_SCASE(128, 32)
+    QL_SCASE(128, 64)
+#undef QL_SCASE
     return cudaErrorInvalidValue;
   }
 #define QL_CASE(FP4_, BN_, CG_) \

@@ -15,12 +15,14 @@ constexpr int QL_ERR_TIMEOUT_CODE = 7;  // same value as QL_ERR_TIMEOUT in qline
 struct GemmConfig {
   int bn;
   int cg;
+  int arows;  // rows of A per pipeline stage of a skinny kernel (16, 32, 64), or 0
 };
 
 struct GemmProblem {
   bool fp4;
   int bn;
   int cg;
+  int arows;  // GemmConfig::arows: 0, or the skinny kernel's rows of A per stage
   int64_t M, N, K;
   const void* a;
   const void* b;
@@ -39,7 +41,8 @@ struct GemmProblem {
   // tile width bn), then runs the GEMM on them
   bool fused;
   const void* x;             // bf16 [M, K]
-  const uint8_t* w_scale;    // E4M3 [N, K/16] row-major
+  const uint8_t* w_scale;    // E4M3 [N, K/16] row-major (also: a skinny plain GEMM given it
+                             // lays out the weight scales itself, per stage)
   uint64_t* sync;            // 8 words (64 bytes) in the workspace
   uint32_t tag;              // odd, different from the previous launch on this workspace
   // GELU-quantize epilogue (FP4, N % 256 == 0): instead of y, NVFP4 of GELU(Y) with
@@ -58,8 +61,11 @@ struct GemmProblem {
 };
 
 // whole_buffers: only tile widths whose two TMEM accumulator buffers do not share
-// a slab (the GELU-quantize epilogue).
-GemmConfig choose_config(bool fp4, int64_t M, int64_t N, int64_t K, bool whole_buffers = false);
+// a slab (the GELU-quantize epilogue). allow_skinny: M <= 64 may use the skinny
+// kernels (plain GEMM without the low-rank branch; the prologue that lays out the
+// weight scales must make the same choice).
+GemmConfig choose_config(bool fp4, int64_t M, int64_t N, int64_t K, bool whole_buffers = false,
+                         bool allow_skinny = true);
 bool set_tile_override(int bn, int cg);  // bn == 0 restores the automatic choice
 // Elapsed SM cycles and nanoseconds of CTA 0 of the last GEMM launch on the current
 // device (synchronous copy from the device).
@@ -68,9 +74,12 @@ cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream);
 
 cudaError_t launch_nvfp4_quantize_rowmajor(const void* x, int64_t M, int64_t K, const float* g,
                                            uint8_t* xq, uint8_t* xs, cudaStream_t s);
+// The prologue of nvfp4_linear: activations into codes + scale atoms, and (when
+// weight_layout) the weight scales into atoms for tiles of bn rows. Without the
+// weight layout it lets the next (skinny) GEMM launch at its start.
 cudaError_t launch_nvfp4_prologue(const void* x, int64_t M, int64_t K, const uint8_t* w_scale,
                                   int64_t N, int bn, const float* input_scale, uint8_t* workspace,
-                                  cudaStream_t s);
+                                  cudaStream_t s, bool weight_layout = true);
 // Weight-scale layout only (the activation part of the workspace is left as is).
 cudaError_t launch_nvfp4_weight_layout(const uint8_t* w_scale, int64_t M, int64_t K, int64_t N,
                                        int bn, const float* input_scale, uint8_t* workspace,

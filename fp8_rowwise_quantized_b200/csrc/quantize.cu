@@ -154,13 +154,18 @@ nvfp4_quantize_kernel(const uint16_t* __restrict__ x, int M, int K,
 // Each block allows the dependent GEMM launch once its own work is issued, so the
 // GEMM's set-up overlaps the prologue's tail (the GEMM reads the workspace only
 // after this grid has completed); triggering earlier would let resident GEMM CTAs
-// take the shared memory the prologue blocks need.
+// take the shared memory the prologue blocks need. EARLY: allow it at the start
+// instead (the small activation-only prologue of the skinny GEMMs, which stream
+// their weights while it runs; that instantiation asks for the largest shared-memory
+// split, so a GEMM CTA can join its blocks on an SM).
+template <bool EARLY>
 __global__ void __launch_bounds__(kQuantThreads)
 nvfp4_prologue_kernel(const uint16_t* __restrict__ x, int M, int K,
                       const float* __restrict__ g_ptr, uint8_t* __restrict__ xq,
                       uint8_t* __restrict__ xs, uint32_t rows_total, uint32_t segs, int KG,
                       const uint8_t* __restrict__ ws, int64_t N, int bn, int na, int64_t n_tiles,
                       int64_t w_jobs, uint8_t* __restrict__ wout) {
+  if constexpr (EARLY) grid_dependents_launch();
   __shared__ WsTile tile;
   // the block's first weight-scale job: its loads are in flight during the activation
   // items, so their latency is off the block's critical path
@@ -333,24 +338,40 @@ cudaError_t launch_nvfp4_quantize_rowmajor(const void* x, int64_t M, int64_t K, 
 
 cudaError_t launch_nvfp4_prologue(const void* x, int64_t M, int64_t K, const uint8_t* w_scale,
                                   int64_t N, int bn, const float* input_scale, uint8_t* workspace,
-                                  cudaStream_t s) {
+                                  cudaStream_t s, bool weight_layout) {
   const Nvfp4Workspace L = nvfp4_workspace(M, K, N, bn);
   const int64_t KG = sf_kgroups(K);
   const int64_t rows = ceil_div64(M, 128) * 128;
   const int64_t segs = ceil_div64(KG * 64, 1024);
   const int na = (bn + 127) / 128;
   const int64_t n_tiles = ceil_div64(N, bn);
-  const int64_t w_jobs = n_tiles * na * ceil_div64(KG, kWsGroups);
+  const int64_t w_jobs = weight_layout ? n_tiles * na * ceil_div64(KG, kWsGroups) : 0;
   static std::atomic<int64_t> wave_cache{0};  // resident blocks of one wave (same on every B200)
+  static std::atomic<int> carveout_set[64] = {};
   int64_t wave = wave_cache.load(std::memory_order_relaxed);
   if (wave == 0) {
-    wave = resident_blocks(nvfp4_prologue_kernel);
+    wave = resident_blocks(nvfp4_prologue_kernel<false>);
     wave_cache.store(wave, std::memory_order_relaxed);
+  }
+  if (!weight_layout) {
+    // An SM's split between L1 and shared memory follows the kernel whose blocks it
+    // runs: with the split chosen for this kernel's 9 KB, a GEMM CTA (about 200 KB)
+    // launched early could not join the prologue's blocks on an SM until they left.
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && carveout_set[dev].load(std::memory_order_relaxed) == 0) {
+      cudaError_t ce = cudaFuncSetAttribute(nvfp4_prologue_kernel<true>,
+                                            cudaFuncAttributePreferredSharedMemoryCarveout,
+                                            static_cast<int>(cudaSharedmemCarveoutMaxShared));
+      if (ce != cudaSuccess) return ce;
+      carveout_set[dev].store(1, std::memory_order_relaxed);
+    }
   }
   int64_t need = ceil_div64(rows * segs, kQuantThreads / 32);
   if (need < w_jobs) need = w_jobs;
   const int64_t blocks = need < wave ? need : wave;
-  nvfp4_prologue_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, 0, s>>>(
+  auto kern = weight_layout ? nvfp4_prologue_kernel<false> : nvfp4_prologue_kernel<true>;
+  kern<<<static_cast<unsigned>(blocks), kQuantThreads, 0, s>>>(
       static_cast<const uint16_t*>(x), static_cast<int>(M), static_cast<int>(K), input_scale,
       workspace + L.codes_off, workspace + L.act_sf_off, static_cast<uint32_t>(rows),
       static_cast<uint32_t>(segs), static_cast<int>(KG), w_scale, N, bn, na, n_tiles, w_jobs,
@@ -370,11 +391,11 @@ cudaError_t launch_nvfp4_weight_layout(const uint8_t* w_scale, int64_t M, int64_
   static std::atomic<int64_t> wave_cache{0};  // resident blocks of one wave (same on every B200)
   int64_t wave = wave_cache.load(std::memory_order_relaxed);
   if (wave == 0) {
-    wave = resident_blocks(nvfp4_prologue_kernel);
+    wave = resident_blocks(nvfp4_prologue_kernel<false>);
     wave_cache.store(wave, std::memory_order_relaxed);
   }
   const int64_t blocks = w_jobs < wave ? w_jobs : wave;
-  nvfp4_prologue_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, 0, s>>>(
+  nvfp4_prologue_kernel<false><<<static_cast<unsigned>(blocks), kQuantThreads, 0, s>>>(
       nullptr, static_cast<int>(M), static_cast<int>(K), input_scale, workspace + L.codes_off,
       workspace + L.act_sf_off, 0u, static_cast<uint32_t>(ceil_div64(KG * 64, 1024)),
       static_cast<int>(KG), w_scale, N, bn, na, n_tiles, w_jobs, workspace + L.wgt_sf_off);

@@ -86,6 +86,27 @@ def test_nvfp4_linear_batched_sampled(M, N):
     assert np.abs(yb).max() < 1e4 and (yb != 0).mean() > 0.99
 
 
+# Skinny kernels (M <= 64): stages hold only 16 / 32 / 64 rows of A, tiles of 64, 96
+# or 128 columns on one CTA; every combination through the tile override, with
+# ragged M, N and K and a bias.
+@pytest.mark.parametrize("bn", [64, 96, 128])
+@pytest.mark.parametrize("M", [1, 16, 17, 32, 40, 64])
+def test_nvfp4_linear_skinny_kernels_full(bn, M):
+    q.set_tile_override(bn, 1)
+    try:
+        assert q.tile_config(M, 1000, 800) == (bn, 1)
+        run_nvfp4(Nvfp4Case(M, 800, 1000, seed=M + bn, bias=True))
+    finally:
+        q.set_tile_override(0, 0)
+
+
+def test_skinny_choice_keeps_one_wave():
+    # the automatic choice for M <= 64: the narrowest width whose tiles fit 148 SMs
+    assert q.tile_config(16, 12288, 3072) == (96, 1)
+    assert q.tile_config(16, 3072, 3072) == (64, 1)
+    assert q.tile_config(64, 18432, 3072) == (128, 1)
+
+
 def test_nvfp4_mlp_down_from_gelu_of_up():
     # the down projection's input is GELU of the up projection's GPU output,
     # re-quantized at run time with a re-calibrated input scale
@@ -109,6 +130,25 @@ def test_nvfp4_linear_split_calls_match_fused():
                              bias=d["bias"])
     torch.cuda.synchronize()
     assert torch.equal(y1, y2)  # same kernels, same order: bit-identical
+
+
+@pytest.mark.parametrize("M", [16, 40])
+def test_skinny_linear_matches_split_calls(M):
+    # nvfp4_linear lays out the weight scales inside the skinny GEMM; the split
+    # prologue + GEMM calls take them from the workspace: same bits
+    c = Nvfp4Case(M, 3072, 3072, seed=M, bias=True)
+    d = c.device_args()
+    ws = torch.empty(q.nvfp4_linear_workspace_size(M, 3072, 3072), dtype=torch.uint8,
+                     device="cuda")
+    y1 = q.nvfp4_linear(d["x"], d["w"], d["w_scale"], d["weight_scale_2"], d["input_scale"],
+                        bias=d["bias"], workspace=ws)
+    q.nvfp4_linear_prologue(d["x"], d["w_scale"], d["input_scale"], ws)
+    y2 = q.nvfp4_linear_gemm(M, d["w"], d["weight_scale_2"], d["input_scale"], ws,
+                             bias=d["bias"])
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    _, y64, T = c.reference()
+    check_linear(y1, y64, T, "skinny nvfp4_linear")
 
 
 def test_nvfp4_linear_repeatable():
@@ -188,7 +228,6 @@ def test_fp8r_linear_every_tile_config(bn, cg):
 
 
 def test_tile_override_rejects_bad_values():
-    with pytest.raises(q.QLinearError):
-        q.set_tile_override(96, 1)
-    with pytest.raises(q.QLinearError):
-        q.set_tile_override(128, 3)
+    for bn, cg in [(80, 1), (96, 2), (64, 2), (128, 3), (320, 1)]:
+        with pytest.raises(q.QLinearError):
+            q.set_tile_override(bn, cg)

@@ -33,6 +33,7 @@ def lowrank_operands(K, N, r, seed):
 @pytest.mark.parametrize("M,K,N,r", [
     (600, 512, 520, 32),    # CTA pairs, ragged M and N
     (130, 1024, 1536, 32),  # single-CTA tiles
+    (40, 768, 1000, 32),    # skinny kernel (64 rows of A per stage)
     (512, 768, 1000, 64),   # the largest rank: all 4 bf16 MMAs
     (256, 256, 384, 8),     # the smallest rank
 ])
@@ -103,6 +104,7 @@ class SvdqCase:
     (600, 512, 520, 32),
     (130, 1024, 1536, 16),
     (1024, 3072, 3072, 32),
+    (24, 512, 640, 32),     # skinny kernel (32 rows of A per stage)
 ])
 def test_svdq_linear_end_to_end(M, K, N, r):
     from gpu_helpers import unpack_act_scale_atoms
