@@ -94,7 +94,7 @@ cudaError_t launch_svdq_prologue(const void* x, int64_t M, int64_t K, const floa
                                  int bn, const float* input_scale, const float* weight_scale_2,
                                  uint8_t* workspace, void* lr_act, int* status,
                                  uint64_t timeout_ns, cudaStream_t s);
-// W4A16 GEMV (w4a16.cu): K % 32 == 0, x / w 16-byte aligned, w_scale 2-byte aligned.
+// W4A16 linear (w4a16.cu): K % 32 == 0, x / w 16-byte aligned, w_scale 2-byte aligned.
 cudaError_t launch_w4a16_linear(const void* x, int64_t M, int64_t K, const uint8_t* w,
                                 const uint8_t* w_scale, int64_t N, const float* weight_scale_2,
                                 const float* bias, void* y, cudaStream_t s);

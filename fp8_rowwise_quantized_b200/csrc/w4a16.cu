@@ -10,21 +10,24 @@
 //   y[m, n]    = bf16(sum_k x[m, k] * what[n, k] + bias[n])
 // and the activations stay in bf16.
 //
-// These layers run on a few token rows (a batch of conditioning vectors), so the
-// kernel is a GEMV that streams the weight once from HBM: per byte of weight codes
-// it does a fixed amount of decode work and a few fp32 FMAs on the CUDA cores. A
-// tensor-core GEMM would waste the MMA on padding and add a shared-memory round
-// trip without moving the HBM bound.
-//
-// Work split: one warp owns kRows consecutive weight rows at a time; lane l reads
-// the 32-element chunks l, l + 32, ... of each of those rows (16 bytes of codes and
-// two scale bytes per chunk and row, the next chunk prefetched while the current
-// one is decoded), multiplies them with the same chunk of up to MR activation rows
-// (read through L1; every warp of the SM reads the same few KB), and accumulates
-// in fp32 (even and odd elements in the two halves of packed f32x2 FMAs). A warp
-// butterfly sums the lanes, and lane i writes one (row, column) output.
-// Grid: one wave of persistent CTAs (SM count x resident CTAs per SM) striding
-// over the row groups; grid.y walks the activation rows MR at a time.
+// These layers run on a few activation rows, so the weight is read once from HBM
+// and the time goes to streaming it and to the per-weight decode. Design:
+//   * one CTA of 16 warps per SM; a warp owns one item, a tile of 16 weight rows
+//     times one of S parts of K (S chosen so that the items fill one wave), and
+//     streams its codes and block scales straight into registers with 16-byte
+//     loads, four 128-element groups ahead (about 74 KB in flight per SM, what
+//     plain loads need to cover HBM latency; bulk copies into shared memory kept
+//     too few bytes in flight per SM and were slower);
+//   * the decode writes bf16 MMA fragments directly and mma.sync (m16n8k16, fp32
+//     accumulation) does the multiply-adds, one instruction per 256 weights, which
+//     leaves the issue slots to the decode. The tensor core is not here for FLOPs:
+//     the MMA's N = 8 columns hold up to 8 activation rows;
+//   * per weight pair: E2M1 pair -> f16 pair (exact), the products with the block
+//     scale straight into fp32 by mixed-precision fma (exact: at most 6 significant
+//     bits), one fp32 multiply by weight_scale_2 (the single RN32 rounding), and the
+//     bf16 pair;
+//   * the S partial sums of a tile meet in shared memory; bias, bf16 rounding and
+//     the stores follow.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cstdint>
@@ -35,211 +38,306 @@
 namespace ql {
 namespace {
 
-constexpr int kW4Threads = 256;
-constexpr int kW4Warps = kW4Threads / 32;
-constexpr int kRows = 4;  // weight rows per warp task
+constexpr int kWTileRows = 16;      // weight rows per tile (the MMA's M)
+constexpr int kWWarps = 16;         // warps per CTA, one item each
+constexpr int kWThreads = 32 * kWWarps;
+constexpr int kWGroup = 128;        // elements of a row per warp step: 4 lanes x 32
 
-// Packed fp32 pair (element 2i in the low word).
-__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-
-__device__ __forceinline__ void unpack_f32x2(uint64_t p, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(p));
-}
-
-// acc += a * b, both lanes of the packed pairs, each an fp32 fma (RN).
-__device__ __forceinline__ void fma_f32x2(uint64_t& acc, uint64_t a, uint64_t b) {
-  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
-}
-
-// Block scale code s -> (E4M3(s), E4M3(s)) as an f16x2 word (exact: every E4M3
-// value is an f16 value).
+// Two block-scale codes (bytes 0 and 1 of s) -> their E4M3 values as an f16 pair
+// (exact: every E4M3 value is an f16 value); byte 0 in the low half.
 __device__ __forceinline__ uint32_t scale_f16x2(uint32_t s) {
-  uint32_t r;
+  uint32_t h;
   asm("{\n\t.reg .b16 c;\n\t"
       "cvt.u16.u32 c, %1;\n\t"
       "cvt.rn.f16x2.e4m3x2 %0, c;\n\t}"
-      : "=r"(r)
-      : "r"(s | (s << 8)));
-  return r;
+      : "=r"(h)
+      : "r"(s));
+  return h;
 }
 
-// Two E2M1 codes (one byte of the packed weight: element 2j in the low nibble) ->
-// the two dequantized weights as bf16 bits in the high halves of two fp32 words:
-//   p = E2M1 * E4M3(s) in f16 (exact: at most 6 significant bits, 2^-10 <= |p| <=
-//       2688 or 0),
-//   RN32(p * g) (two fp32 lanes), then RN to bf16 (one cvt for the pair).
-// Returns the packed pair of fp32 values (element 2j in the low word).
-__device__ __forceinline__ uint64_t w4_decode2(uint32_t byte, uint32_t ss, uint64_t gg) {
-  uint64_t r;
-  asm("{\n\t"
-      ".reg .b8 c;\n\t"
-      ".reg .b16 lo16, hi16;\n\t"
-      ".reg .b32 h, f0, f1, b, w0, w1;\n\t"
-      ".reg .b64 p;\n\t"
-      "cvt.u8.u32 c, %1;\n\t"
-      "cvt.rn.f16x2.e2m1x2 h, c;\n\t"
-      "mul.rn.f16x2 h, h, %2;\n\t"
-      "mov.b32 {lo16, hi16}, h;\n\t"
-      "cvt.f32.f16 f0, lo16;\n\t"
-      "cvt.f32.f16 f1, hi16;\n\t"
-      "mov.b64 p, {f0, f1};\n\t"
-      "mul.rn.f32x2 p, p, %3;\n\t"
-      "mov.b64 {f0, f1}, p;\n\t"
-      "cvt.rn.bf16x2.f32 b, f1, f0;\n\t"
-      "shl.b32 w0, b, 16;\n\t"
-      "and.b32 w1, b, -65536;\n\t"
-      "mov.b64 %0, {w0, w1};\n\t}"
-      : "=l"(r)
-      : "r"(byte), "r"(ss), "l"(gg));
-  return r;
+// One 32-bit word of packed codes (element 2i in the low nibble of byte i) and
+// the block scale d (f16: the low half of dd when HI == 0, else the high half) ->
+// the four bf16 pairs of its eight dequantized weights (byte i -> r[i], element
+// 2i in the low half). Per byte: E2M1 pair -> f16 pair (exact); v * d exactly in
+// fp32 (mixed-precision fma with -0, so a -0 code stays -0); RN32(v * d * g) by
+// one fp32 multiply per element; RN to bf16.
+#define QL_W4_BYTE(C, R, D)                      \
+  "cvt.rn.f16x2.e2m1x2 h, " C ";\n\t"            \
+  "mov.b32 {v0, v1}, h;\n\t"                     \
+  "fma.rn.f32.f16 f0, v0, " D ", 0f80000000;\n\t" \
+  "fma.rn.f32.f16 f1, v1, " D ", 0f80000000;\n\t" \
+  "mov.b64 p, {f0, f1};\n\t"                     \
+  "mul.rn.f32x2 p, p, %6;\n\t"                   \
+  "mov.b64 {f0, f1}, p;\n\t"                     \
+  "cvt.rn.bf16x2.f32 " R ", f1, f0;\n\t"
+
+template <int HI>
+__device__ __forceinline__ void w4_word(uint32_t word, uint32_t dd, uint64_t gg, uint32_t (&r)[4]) {
+  if (HI == 0) {
+    asm("{\n\t"
+        ".reg .b8 c0, c1, c2, c3;\n\t"
+        ".reg .b16 v0, v1, d0, d1;\n\t"
+        ".reg .b32 h, f0, f1;\n\t"
+        ".reg .b64 p;\n\t"
+        "mov.b32 {c0, c1, c2, c3}, %4;\n\t"
+        "mov.b32 {d0, d1}, %5;\n\t"
+        QL_W4_BYTE("c0", "%0", "d0") QL_W4_BYTE("c1", "%1", "d0")
+        QL_W4_BYTE("c2", "%2", "d0") QL_W4_BYTE("c3", "%3", "d0")
+        "}"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+        : "r"(word), "r"(dd), "l"(gg));
+  } else {
+    asm("{\n\t"
+        ".reg .b8 c0, c1, c2, c3;\n\t"
+        ".reg .b16 v0, v1, d0, d1;\n\t"
+        ".reg .b32 h, f0, f1;\n\t"
+        ".reg .b64 p;\n\t"
+        "mov.b32 {c0, c1, c2, c3}, %4;\n\t"
+        "mov.b32 {d0, d1}, %5;\n\t"
+        QL_W4_BYTE("c0", "%0", "d1") QL_W4_BYTE("c1", "%1", "d1")
+        QL_W4_BYTE("c2", "%2", "d1") QL_W4_BYTE("c3", "%3", "d1")
+        "}"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+        : "r"(word), "r"(dd), "l"(gg));
+  }
+}
+#undef QL_W4_BYTE
+
+// D (16 x 8, fp32) += A (16 x 16, bf16, row-major) * B (16 x 8, bf16, column-major).
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// bf16 pair (one word, element 2i in the low half) -> packed fp32 pair.
-__device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t w) {
-  return pack_f32x2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
-}
+struct W4Args {
+  const uint16_t* x;
+  int64_t M, K, N;
+  const uint8_t* w;
+  const uint8_t* ws;
+  const float* g_ptr;
+  const float* bias;
+  uint16_t* y;
+  int parts;  // S: parts of K per tile, a power of two dividing kWWarps
+};
 
-template <int MR>
-__global__ void __launch_bounds__(kW4Threads)
-    w4a16_gemv_kernel(const uint16_t* __restrict__ x, int64_t M, int64_t K,
-                      const uint8_t* __restrict__ w, const uint8_t* __restrict__ ws, int64_t N,
-                      const float* __restrict__ g_ptr, const float* __restrict__ bias,
-                      uint16_t* __restrict__ y) {
-  const int lane = threadIdx.x & 31;
-  const int64_t warp_global = static_cast<int64_t>(blockIdx.x) * kW4Warps + (threadIdx.x >> 5);
-  const int64_t warp_stride = static_cast<int64_t>(gridDim.x) * kW4Warps;
-  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * MR;
-  const int64_t chunks = K / 32;        // 32 elements: 16 code bytes, 2 scale bytes
-  const int64_t row_code_bytes = K / 2;
-  const int64_t row_scale_bytes = K / 16;
-  const int64_t tasks = (N + kRows - 1) / kRows;
-  const float g = __ldg(g_ptr);
-  const uint64_t gg = pack_f32x2(g, g);
-  int mr_valid = static_cast<int>(M - m0 < MR ? M - m0 : MR);
 
-  for (int64_t task = warp_global; task < tasks; task += warp_stride) {
-    const int64_t n0 = task * kRows;
-    uint64_t acc[kRows][MR];
+// Decode one group's codes of this lane (16 bytes of rows gid and gid + 8, scale
+// pairs sa / sb) into bf16 fragments and run its 8 MMAs (per block of 8
+// activation rows), alternating between two accumulators.
+template <int MB>
+__device__ __forceinline__ void w4_group(float (&acc)[MB][2][4], const uint4& c0, const uint4& c1,
+                                         uint32_t sa, uint32_t sb, const uint4 (&xv)[MB][4],
+                                         uint64_t gg) {
+  const uint32_t da = scale_f16x2(sa), db = scale_f16x2(sb);
+  const uint32_t wa[4] = {c0.x, c0.y, c0.z, c0.w};
+  const uint32_t wb[4] = {c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-    for (int r = 0; r < kRows; ++r)
-#pragma unroll
-      for (int m = 0; m < MR; ++m) acc[r][m] = 0;
-
-    // software pipeline over this lane's chunks: codes and scales of chunk c + 32
-    // are in flight while chunk c is decoded
-    uint4 code[kRows];
-    uint32_t scl[kRows];
-    auto load_chunk = [&](int64_t c, uint4 (&cd)[kRows], uint32_t (&sc)[kRows]) {
-#pragma unroll
-      for (int r = 0; r < kRows; ++r) {
-        const int64_t n = n0 + r;
-        if (c < chunks && n < N) {
-          cd[r] = ld_stream16(w + n * row_code_bytes + c * 16);
-          sc[r] = __ldg(reinterpret_cast<const uint16_t*>(ws + n * row_scale_bytes + c * 2));
-        } else {
-          cd[r] = make_uint4(0, 0, 0, 0);
-          sc[r] = 0;
-        }
-      }
-    };
-    load_chunk(lane, code, scl);
-    for (int64_t c = lane; c < chunks; c += 32) {
-      uint4 next_code[kRows];
-      uint32_t next_scl[kRows];
-      load_chunk(c + 32, next_code, next_scl);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {  // 8 elements: k = 32 c + 8 i .. + 8
-        // activations of this word for every row of the pass, as fp32 pairs
-        uint64_t xv[MR][4];
-#pragma unroll
-        for (int m = 0; m < MR; ++m) {
-          uint4 u = make_uint4(0, 0, 0, 0);
-          if (m < mr_valid)
-            u = __ldg(reinterpret_cast<const uint4*>(x + (m0 + m) * K + c * 32 + i * 8));
-          xv[m][0] = bf16x2_to_f32x2(u.x);
-          xv[m][1] = bf16x2_to_f32x2(u.y);
-          xv[m][2] = bf16x2_to_f32x2(u.z);
-          xv[m][3] = bf16x2_to_f32x2(u.w);
-        }
-#pragma unroll
-        for (int r = 0; r < kRows; ++r) {
-          const uint32_t word = i == 0 ? code[r].x : i == 1 ? code[r].y : i == 2 ? code[r].z
-                                                                                 : code[r].w;
-          const uint32_t ss = scale_f16x2((scl[r] >> (8 * (i >> 1))) & 0xFFu);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint64_t wv = w4_decode2(word >> (8 * j), ss, gg);
-#pragma unroll
-            for (int m = 0; m < MR; ++m) fma_f32x2(acc[r][m], wv, xv[m][j]);
-          }
-        }
-      }
-#pragma unroll
-      for (int r = 0; r < kRows; ++r) {
-        code[r] = next_code[r];
-        scl[r] = next_scl[r];
-      }
+  for (int q = 0; q < 4; ++q) {  // code bytes 4q .. 4q + 3: MMAs 2q and 2q + 1
+    uint32_t ra_[4], rb_[4];
+    if (q < 2) {  // elements 0..15 of the chunk: the first scale byte
+      w4_word<0>(wa[q], da, gg, ra_);
+      w4_word<0>(wb[q], db, gg, rb_);
+    } else {      // elements 16..31: the second
+      w4_word<1>(wa[q], da, gg, ra_);
+      w4_word<1>(wb[q], db, gg, rb_);
     }
-
-    // lanes -> one sum per (row, activation row); lane r * MR + m writes it
-    float out = 0.0f;
 #pragma unroll
-    for (int r = 0; r < kRows; ++r) {
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t a0 = ra_[2 * h], a2 = ra_[2 * h + 1];
+      const uint32_t a1 = rb_[2 * h], a3 = rb_[2 * h + 1];
 #pragma unroll
-      for (int m = 0; m < MR; ++m) {
-        float lo, hi;
-        unpack_f32x2(acc[r][m], lo, hi);
-        float v = lo + hi;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
-        if (lane == r * MR + m) out = v;
-      }
-    }
-    if (lane < kRows * MR) {
-      const int r = lane / MR, m = lane % MR;
-      const int64_t n = n0 + r;
-      if (n < N && m < mr_valid) {
-        const float v = bias ? out + __ldg(bias + n) : out;
-        const __nv_bfloat16 b = __float2bfloat16_rn(v);
-        y[(m0 + m) * N + n] = *reinterpret_cast<const uint16_t*>(&b);
+      for (int mb = 0; mb < MB; ++mb) {
+        const uint32_t b0 = h == 0 ? xv[mb][q].x : xv[mb][q].z;
+        const uint32_t b1 = h == 0 ? xv[mb][q].y : xv[mb][q].w;
+        mma_bf16_16816(acc[mb][h], a0, a1, a2, a3, b0, b1);
       }
     }
   }
 }
 
-template <int MR>
-cudaError_t launch_mr(const void* x, int64_t M, int64_t K, const uint8_t* w, const uint8_t* ws,
-                      int64_t N, const float* g, const float* bias, void* y, cudaStream_t s) {
-  static int blocks_per_sm[64] = {};
+// 16-byte read-only load, not kept in L1; the L2::256B hint has L2 fetch the whole
+// aligned 256 bytes around it, so the next groups of the same row (64 bytes each)
+// are already on their way when their own loads are issued.
+__device__ __forceinline__ uint4 ld_codes16(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// One warp item: groups [g_begin, g_end) of the tile whose rows gid / gid + 8 are
+// ra / rb. FULL: both rows exist and every group lies inside K, so no load needs a
+// guard and the pointers advance by constants. The codes and scales of the next
+// P groups wait in registers while one is decoded. Activation rows past M are
+// read as row M - 1: they only feed MMA columns that are never stored.
+template <int MB, int P, bool FULL>
+__device__ __forceinline__ void w4_item(const W4Args& a, float (&acc)[MB][2][4], int64_t ra,
+                                        int64_t rb, int64_t g_begin, int64_t g_end, int64_t m0,
+                                        int gid, int tid, uint64_t gg) {
+  const int64_t code_row = a.K / 2, scale_row = a.K / 16;
+  const bool va = FULL || ra < a.N, vb = FULL || rb < a.N;
+  const int64_t e_first = g_begin * kWGroup + 32 * tid;
+  const uint8_t* pa = a.w + (va ? ra : 0) * code_row + e_first / 2;
+  const uint8_t* pb = a.w + (vb ? rb : 0) * code_row + e_first / 2;
+  const uint16_t* qa = reinterpret_cast<const uint16_t*>(a.ws + (va ? ra : 0) * scale_row) + e_first / 32;
+  const uint16_t* qb = reinterpret_cast<const uint16_t*>(a.ws + (vb ? rb : 0) * scale_row) + e_first / 32;
+  const uint4* px[MB];
+#pragma unroll
+  for (int mb = 0; mb < MB; ++mb) {
+    int64_t m = m0 + 8 * mb + gid;
+    if (m > a.M - 1) m = a.M - 1;
+    px[mb] = reinterpret_cast<const uint4*>(a.x + m * a.K + e_first);
+  }
+  // group g_begin + j sits j * 64 code bytes, 4 scale words and 16 activation
+  // vectors further on
+  auto load = [&](int64_t j, uint4& c0, uint4& c1, uint32_t& s0, uint32_t& s1) {
+    const int64_t gi = g_begin + j;
+    if (FULL) {
+      if (gi < g_end) {
+        c0 = ld_codes16(pa + 64 * j);
+        c1 = ld_codes16(pb + 64 * j);
+        s0 = __ldg(qa + 4 * j);
+        s1 = __ldg(qb + 4 * j);
+      }
+    } else {
+      c0 = c1 = make_uint4(0, 0, 0, 0);
+      s0 = s1 = 0;
+      const bool in_k = gi < g_end && gi * kWGroup + 32 * tid < a.K;
+      if (in_k && va) {
+        c0 = ld_codes16(pa + 64 * j);
+        s0 = __ldg(qa + 4 * j);
+      }
+      if (in_k && vb) {
+        c1 = ld_codes16(pb + 64 * j);
+        s1 = __ldg(qb + 4 * j);
+      }
+    }
+  };
+  uint4 ca[P], cb[P];
+  uint32_t sa[P], sb[P];
+#pragma unroll
+  for (int i = 0; i < P; ++i) load(i, ca[i], cb[i], sa[i], sb[i]);
+  const int64_t n_groups = g_end - g_begin;
+  for (int64_t base = 0; base < n_groups; base += P) {
+#pragma unroll
+    for (int i = 0; i < P; ++i) {
+      const int64_t j = base + i;
+      if (j >= n_groups) break;  // warp-uniform
+      uint4 xv[MB][4];
+      const bool x_in = FULL || (g_begin + j) * kWGroup + 32 * tid < a.K;
+#pragma unroll
+      for (int mb = 0; mb < MB; ++mb)
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          xv[mb][q] = x_in ? __ldg(px[mb] + 16 * j + q) : make_uint4(0, 0, 0, 0);
+      w4_group<MB>(acc, ca[i], cb[i], sa[i], sb[i], xv, gg);
+      // the slot just consumed takes the group P further on
+      load(j + P, ca[i], cb[i], sa[i], sb[i]);
+    }
+  }
+}
+
+// Fragment roles (mma.sync m16n8k16, lane = 4 * gid + tid): A registers a0 / a2 hold
+// row gid, a1 / a3 row gid + 8, at logical k (2 tid, 2 tid + 1) and (2 tid + 8,
+// 2 tid + 9); B registers b0 / b1 hold activation row gid at the same logical k.
+// Lane tid of a 128-element group owns the 32 elements [32 tid, 32 tid + 32) of
+// its two weight rows (16 code bytes each) and, in MMA j (0..7), feeds elements
+// 32 tid + 4 j + {0, 1} as logical (2 tid, 2 tid + 1) and 32 tid + 4 j + {2, 3} as
+// (2 tid + 8, 2 tid + 9). The map from logical to actual k depends on tid and j
+// only, so A and B agree for every row and the sum over the group is complete.
+template <int MB, int P>
+__global__ void __launch_bounds__(kWThreads, 1) w4a16_kernel(const W4Args a) {
+  __shared__ float4 red[kWWarps][MB][32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gid = lane >> 2, tid = lane & 3;
+  const int S = a.parts;
+  const int tiles_per_block = kWWarps / S;
+  const int64_t tiles = (a.N + kWTileRows - 1) / kWTileRows;
+  const int64_t blocks = (tiles + tiles_per_block - 1) / tiles_per_block;
+  const int64_t groups = (a.K + kWGroup - 1) / kWGroup;
+  const int64_t per_part = (groups + S - 1) / S;
+  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * (8 * MB);
+  const float g = __ldg(a.g_ptr);
+  uint64_t gg;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(gg) : "f"(g));
+
+  for (int64_t tb = blockIdx.x; tb < blocks; tb += gridDim.x) {
+    const int64_t tile = tb * tiles_per_block + warp / S;
+    const int64_t n0 = tile * kWTileRows;
+    const int64_t ra = n0 + gid, rb = n0 + gid + 8;
+    const int64_t g_begin = (warp % S) * per_part;
+    const int64_t g_end = g_begin + per_part < groups ? g_begin + per_part : groups;
+
+    float acc[MB][2][4];
+#pragma unroll
+    for (int mb = 0; mb < MB; ++mb)
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[mb][h][i] = 0.0f;
+
+    if (tile < tiles) {  // warp-uniform
+      const bool full = n0 + kWTileRows <= a.N && g_end * kWGroup <= a.K;
+      if (full)
+        w4_item<MB, P, true>(a, acc, ra, rb, g_begin, g_end, m0, gid, tid, gg);
+      else
+        w4_item<MB, P, false>(a, acc, ra, rb, g_begin, g_end, m0, gid, tid, gg);
+    }
+
+    // the S partial sums of each tile -> outputs
+#pragma unroll
+    for (int mb = 0; mb < MB; ++mb)
+      red[warp][mb][lane] = make_float4(acc[mb][0][0] + acc[mb][1][0], acc[mb][0][1] + acc[mb][1][1],
+                                        acc[mb][0][2] + acc[mb][1][2], acc[mb][0][3] + acc[mb][1][3]);
+    __syncthreads();
+    const float* redf = reinterpret_cast<const float*>(red);
+    for (int e = threadIdx.x; e < tiles_per_block * MB * 128; e += kWThreads) {
+      const int t = e / (MB * 128), rem = e % (MB * 128);
+      const int mb = rem >> 7, l = (rem & 127) >> 2, r = rem & 3;
+      float sum = 0.0f;  // from +0: a -0 weight gives +0, like an fp32 dot product
+      for (int p = 0; p < S; ++p) sum += redf[(((t * S + p) * MB + mb) * 32 + l) * 4 + r];
+      const int64_t n = (tb * tiles_per_block + t) * kWTileRows + (l >> 2) + 8 * (r >> 1);
+      const int64_t m = m0 + 8 * mb + 2 * (l & 3) + (r & 1);
+      if (n < a.N && m < a.M) {
+        const float v = a.bias ? sum + __ldg(a.bias + n) : sum;
+        const __nv_bfloat16 b = __float2bfloat16_rn(v);
+        a.y[m * a.N + n] = *reinterpret_cast<const uint16_t*>(&b);
+      }
+    }
+    __syncthreads();
+  }
+}
+
+template <int MB, int P>
+cudaError_t launch_mb(W4Args args, cudaStream_t s) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  int per_sm = dev < 64 ? blocks_per_sm[dev] : 0;
-  if (per_sm == 0) {
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, w4a16_gemv_kernel<MR>, kW4Threads, 0);
-    if (e != cudaSuccess) return e;
-    if (per_sm < 1) per_sm = 1;
-    if (dev < 64) blocks_per_sm[dev] = per_sm;
-  }
   int sms = 0;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  const int64_t tasks = (N + kRows - 1) / kRows;
-  const int64_t want = (tasks + kW4Warps - 1) / kW4Warps;
-  const int64_t wave = static_cast<int64_t>(sms) * per_sm;
-  const int64_t row_passes = (M + MR - 1) / MR;
-  // one wave in total over the row passes (at least one CTA per pass)
-  int64_t bx = wave / row_passes;
+  const int64_t tiles = (args.N + kWTileRows - 1) / kWTileRows;
+  const int64_t groups = (args.K + kWGroup - 1) / kWGroup;
+  const int64_t passes = (args.M + 8 * MB - 1) / (8 * MB);
+  if (passes > 65535) return cudaErrorInvalidValue;
+  // parts of K per tile: the largest power of two (<= 16, <= the groups) whose
+  // items still fit about one wave of warps over the activation-row passes
+  const int64_t wave_warps = static_cast<int64_t>(sms) * kWWarps / passes;
+  int S = 1;
+  while (S < kWWarps && 2 * S <= groups && tiles * 2 * S * 10 <= wave_warps * 11) S *= 2;
+  args.parts = S;
+  const int64_t blocks = (tiles + kWWarps / S - 1) / (kWWarps / S);
+  int64_t bx = sms / passes;
   if (bx < 1) bx = 1;
-  if (bx > want) bx = want;
-  if (row_passes > 65535) return cudaErrorInvalidValue;
-  dim3 grid(static_cast<unsigned>(bx), static_cast<unsigned>(row_passes));
-  w4a16_gemv_kernel<MR><<<grid, kW4Threads, 0, s>>>(
-      static_cast<const uint16_t*>(x), M, K, w, ws, N, g, bias, static_cast<uint16_t*>(y));
+  if (bx > blocks) bx = blocks;
+  dim3 grid(static_cast<unsigned>(bx), static_cast<unsigned>(passes));
+  w4a16_kernel<MB, P><<<grid, kWThreads, 0, s>>>(args);
   return cudaGetLastError();
 }
 
@@ -248,10 +346,19 @@ cudaError_t launch_mr(const void* x, int64_t M, int64_t K, const uint8_t* w, con
 cudaError_t launch_w4a16_linear(const void* x, int64_t M, int64_t K, const uint8_t* w,
                                 const uint8_t* w_scale, int64_t N, const float* weight_scale_2,
                                 const float* bias, void* y, cudaStream_t s) {
-  if (M == 1) return launch_mr<1>(x, M, K, w, w_scale, N, weight_scale_2, bias, y, s);
-  if (M == 2) return launch_mr<2>(x, M, K, w, w_scale, N, weight_scale_2, bias, y, s);
-  if (M <= 4) return launch_mr<4>(x, M, K, w, w_scale, N, weight_scale_2, bias, y, s);
-  return launch_mr<8>(x, M, K, w, w_scale, N, weight_scale_2, bias, y, s);
+  W4Args args;
+  args.x = static_cast<const uint16_t*>(x);
+  args.M = M;
+  args.K = K;
+  args.N = N;
+  args.w = w;
+  args.ws = w_scale;
+  args.g_ptr = weight_scale_2;
+  args.bias = bias;
+  args.y = static_cast<uint16_t*>(y);
+  args.parts = 1;
+  if (M <= 8) return launch_mb<1, 3>(args, s);
+  return launch_mb<2, 2>(args, s);
 }
 
 }  // namespace ql

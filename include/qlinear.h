@@ -133,8 +133,8 @@ int svdq_nvfp4_linear(const void* x, int64_t M, int64_t K, const float* smooth,
  *   weight_scale_2  device fp32 scalar
  *   bias            fp32 [N] or NULL
  *   y               bf16 [M, N] (output)
- * One launch, no workspace: a GEMV that streams the weight once per 8 rows of x
- * (made for M <= 8; larger M works and re-reads the weight, mostly from L2).
+ * One launch, no workspace: the weight streams once from HBM for up to 8 rows of x
+ * (made for M <= 8); larger M runs passes of 16 rows, each reading the weight again.
  * Requires K >= 32, K % 32 == 0; x, w, y 16-byte aligned, w_scale 2-byte aligned. */
 int w4a16_linear(const void* x, int64_t M, int64_t K, const uint8_t* w,
                  const uint8_t* w_scale, int64_t N, const float* weight_scale_2,
