@@ -435,9 +435,14 @@ def int4_linear(x: torch.Tensor, w: torch.Tensor, w_scale: torch.Tensor,
     return y
 
 
+def int4_linear_gemm_workspace_size(M: int, K: int, N: int) -> int:
+    return int(_lib.load().int4_linear_gemm_workspace_size(M, K, N))
+
+
 def int4_linear_gemm(xq: torch.Tensor, x_scale: torch.Tensor, w: torch.Tensor,
                      w_scale: torch.Tensor, bias: Optional[torch.Tensor] = None,
-                     y: Optional[torch.Tensor] = None) -> torch.Tensor:
+                     y: Optional[torch.Tensor] = None,
+                     workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
     """The GEMM of int4_linear on activations quantized by int4_quantize_rows."""
     _need(xq, "xq", torch.uint8, 2)
     dev = xq.device
@@ -446,8 +451,9 @@ def int4_linear_gemm(xq: torch.Tensor, x_scale: torch.Tensor, w: torch.Tensor,
     N = _int4_weight(w, w_scale, K, dev)
     _bias(bias, N, dev)
     y = _out(y, M, N, dev)
+    ws = _workspace(int4_linear_gemm_workspace_size(M, K, N), dev, workspace)
     _call("int4_linear_gemm", dev, _ptr(xq), _ptr(x_scale), M, K, _ptr(w), _ptr(w_scale), N,
-          _ptr(bias), _ptr(y))
+          _ptr(bias), _ptr(y), _ptr(ws), ws.numel())
     return y
 
 

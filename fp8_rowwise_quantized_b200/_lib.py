@@ -51,8 +51,9 @@ SIGNATURES = {
     "int4_quantize_rows": (C.c_int, [_vp, _i64, _i64, _u8p, _f32p, _vp]),
     "int4_linear_workspace_size": (C.c_size_t, [_i64, _i64, _i64]),
     "int4_linear": (C.c_int, [_vp, _i64, _i64, _u8p, _f32p, _i64, _f32p, _vp, _vp, _sz, _vp]),
+    "int4_linear_gemm_workspace_size": (C.c_size_t, [_i64, _i64, _i64]),
     "int4_linear_gemm": (C.c_int, [_u8p, _f32p, _i64, _i64, _u8p, _f32p, _i64, _f32p, _vp,
-                                   _vp]),
+                                   _vp, _sz, _vp]),
     "fp8r_quantize_rows": (C.c_int, [_vp, _i64, _i64, _u8p, _f32p, _vp]),
     "fp8r_linear_workspace_size": (C.c_size_t, [_i64, _i64, _i64]),
     "fp8r_linear": (C.c_int, [_vp, _i64, _i64, _u8p, _f32p, _i64, _f32p, _vp, _vp, _sz, _vp]),

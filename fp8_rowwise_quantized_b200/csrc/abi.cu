@@ -613,28 +613,72 @@ int int4_quantize_rows(const void* x, int64_t M, int64_t K, uint8_t* q, float* s
   return e == cudaSuccess ? QL_OK : record(e, "int4_quantize_rows");
 }
 
+size_t int4_linear_gemm_workspace_size(int64_t M, int64_t K, int64_t N) {
+  if (!int4_shape_ok(M, K, N)) return 0;
+  return ql::align_up(static_cast<size_t>(M) * static_cast<size_t>(K) * 2, 1024) +
+         ql::align_up(static_cast<size_t>(M) * 4, 1024) +
+         ql::align_up(static_cast<size_t>(N) * static_cast<size_t>(K) * 2, 1024) +
+         ql::align_up(static_cast<size_t>(N) * 4, 1024);
+}
+
 int int4_linear_gemm(const uint8_t* xq, const float* x_scale, int64_t M, int64_t K,
                      const uint8_t* w, const float* w_scale, int64_t N, const float* bias,
-                     void* y, ql_stream_t stream) {
+                     void* y, void* workspace, size_t workspace_bytes, ql_stream_t stream) {
   if (!xq || !x_scale || !w || !w_scale || !y || M <= 0 || N <= 0 || K <= 0)
     return QL_ERR_INVALID_ARG;
   if (!int4_shape_ok(M, K, N)) return fail_shape("int4: needs K >= 64 and K % 64 == 0");
-  if (!aligned16(xq) || !aligned16(w) || (reinterpret_cast<uintptr_t>(x_scale) & 3u) != 0 ||
+  if (!workspace || workspace_bytes < int4_linear_gemm_workspace_size(M, K, N))
+    return QL_ERR_WORKSPACE;
+  if (!aligned16(xq) || !aligned16(w) || !aligned16(workspace) ||
+      (reinterpret_cast<uintptr_t>(x_scale) & 3u) != 0 ||
       (reinterpret_cast<uintptr_t>(w_scale) & 3u) != 0 ||
       (reinterpret_cast<uintptr_t>(bias) & 3u) != 0 || (reinterpret_cast<uintptr_t>(y) & 1u) != 0)
     return QL_ERR_ALIGN;
   int dev = 0;
   int rc = check_device(&dev);
   if (rc != QL_OK) return rc;
-  cudaError_t e = ql::launch_int4_gemm(xq, x_scale, M, K, w, w_scale, N, bias, y, status_ptr(dev),
-                                       timeout_ns(), reinterpret_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? QL_OK : record(e, "int4_linear_gemm");
+  // workspace: f16 x [M, K] | x row factors [M] | f16 w [N, K] | w row factors [N]
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  void* xh = base;
+  base += ql::align_up(static_cast<size_t>(M) * static_cast<size_t>(K) * 2, 1024);
+  float* xf = reinterpret_cast<float*>(base);
+  base += ql::align_up(static_cast<size_t>(M) * 4, 1024);
+  void* wh = base;
+  base += ql::align_up(static_cast<size_t>(N) * static_cast<size_t>(K) * 2, 1024);
+  float* wf = reinterpret_cast<float*>(base);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = ql::launch_int4_dequant_f16(xq, x_scale, M, K, xh, xf, s);
+  if (e != cudaSuccess) return record(e, "int4 dequantize x");
+  e = ql::launch_int4_dequant_f16(w, w_scale, N, K, wh, wf, s);
+  if (e != cudaSuccess) return record(e, "int4 dequantize w");
+  ql::GemmProblem p{};
+  p.fp4 = false;
+  p.f16_operands = true;
+  const ql::GemmConfig cfg = ql::choose_config(false, M, N, K);
+  p.bn = cfg.bn;
+  p.cg = cfg.cg;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.a = xh;
+  p.b = wh;
+  p.scale_a = xf;
+  p.scale_b = wf;
+  p.bias = bias;
+  p.y = y;
+  p.status = status_ptr(dev);
+  p.timeout_ns = timeout_ns();
+  p.inject_fault = g_inject_fault.load();
+  p.pdl = true;
+  e = ql::launch_gemm(p, s);
+  return e == cudaSuccess ? QL_OK : record(e, "int4 f16 gemm launch");
 }
 
 size_t int4_linear_workspace_size(int64_t M, int64_t K, int64_t N) {
   if (!int4_shape_ok(M, K, N)) return 0;
   return ql::align_up(static_cast<size_t>(M) * static_cast<size_t>(K / 2), 1024) +
-         ql::align_up(static_cast<size_t>(M) * static_cast<size_t>(K / 64) * 4, 1024);
+         ql::align_up(static_cast<size_t>(M) * static_cast<size_t>(K / 64) * 4, 1024) +
+         int4_linear_gemm_workspace_size(M, K, N);
 }
 
 int int4_linear(const void* x, int64_t M, int64_t K, const uint8_t* w, const float* w_scale,
@@ -645,11 +689,13 @@ int int4_linear(const void* x, int64_t M, int64_t K, const uint8_t* w, const flo
   if (!workspace || workspace_bytes < int4_linear_workspace_size(M, K, N)) return QL_ERR_WORKSPACE;
   if (!aligned16(workspace)) return QL_ERR_ALIGN;
   uint8_t* xq = static_cast<uint8_t*>(workspace);
-  float* xs = reinterpret_cast<float*>(
-      xq + ql::align_up(static_cast<size_t>(M) * static_cast<size_t>(K / 2), 1024));
+  const size_t q_bytes = ql::align_up(static_cast<size_t>(M) * static_cast<size_t>(K / 2), 1024);
+  const size_t s_bytes = ql::align_up(static_cast<size_t>(M) * static_cast<size_t>(K / 64) * 4, 1024);
+  float* xs = reinterpret_cast<float*>(xq + q_bytes);
   int rc = int4_quantize_rows(x, M, K, xq, xs, stream);
   if (rc != QL_OK) return rc;
-  return int4_linear_gemm(xq, xs, M, K, w, w_scale, N, bias, y, stream);
+  return int4_linear_gemm(xq, xs, M, K, w, w_scale, N, bias, y, xq + q_bytes + s_bytes,
+                          workspace_bytes - q_bytes - s_bytes, stream);
 }
 
 // ------------------------------------------------------------------ diagnostics

@@ -61,6 +61,7 @@ constexpr int kEpiBufsPerWarp = 1;
 struct GemmArgs {
   int M, N, K;
   int tiles_m, tiles_n, num_k_tiles, total_tiles;
+  int f16_ops;              // FP8 path: the operands are f16 (kind::f16 MMAs)
   int64_t kg;               // FP4: 64-element scale groups per row (padded)
   const float* scale_a;     // FP4: input_scale (scalar)   FP8: x_scale [M]
   const float* scale_b;     // FP4: weight_scale_2 (scalar) FP8: w_scale [N]
@@ -972,15 +973,25 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                 mma_nvf4(d_tmem, ad, bd, C::IDESC, sfa, sfb, accum);
             }
           } else {
+            // 32 bytes of K per MMA: 32 E4M3 elements (kind::f8f6f4) or 16 f16
+            // elements (kind::f16); the instruction descriptor is the same word
+            // (E4M3 and f16 are both format 0 of their kinds)
 #pragma unroll
             for (int kb = 0; kb < 4; ++kb) {
               const uint64_t ad = smem_desc(a_addr + kb * 32, 16, 1024, 2);
               const uint64_t bd = smem_desc(b_addr + kb * 32, 16, 1024, 2);
               const uint32_t accum = (kt | kb) != 0 ? 1u : 0u;
-              if constexpr (CG == 2)
-                mma_f8f6f4_pair(d_tmem, ad, bd, C::IDESC, accum);
-              else
-                mma_f8f6f4(d_tmem, ad, bd, C::IDESC, accum);
+              if (args.f16_ops) {
+                if constexpr (CG == 2)
+                  mma_bf16_pair(d_tmem, ad, bd, C::IDESC, accum);
+                else
+                  mma_bf16(d_tmem, ad, bd, C::IDESC, accum);
+              } else {
+                if constexpr (CG == 2)
+                  mma_f8f6f4_pair(d_tmem, ad, bd, C::IDESC, accum);
+                else
+                  mma_f8f6f4(d_tmem, ad, bd, C::IDESC, accum);
+              }
             }
           }
           // frees the stage (in both CTAs of a pair) once these MMAs have read it
@@ -1362,7 +1373,8 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
 
-  const int64_t k_bytes = FP4 ? p.K / 2 : p.K;
+  if (p.f16_operands && (FP4 || MODE != kModePlain)) return cudaErrorInvalidValue;
+  const int64_t k_bytes = FP4 ? p.K / 2 : (p.f16_operands ? 2 * p.K : p.K);
   CUtensorMap ta, tb, tsa, tsb, ty, tla, tlb;
   std::memset(&tla, 0, sizeof(tla));
   std::memset(&tlb, 0, sizeof(tlb));
@@ -1433,7 +1445,9 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
   a.K = static_cast<int>(p.K);
   a.tiles_m = static_cast<int>(ceil_div64(p.M, Cf::TILE_M));
   a.tiles_n = static_cast<int>(ceil_div64(p.N, BN));
-  a.num_k_tiles = static_cast<int>(ceil_div64(p.K, FP4 ? kKTileFp4 : kKTileFp8));
+  // a K tile is 128 bytes of every row: 256 E2M1, 128 E4M3 or 64 f16 elements
+  a.num_k_tiles = static_cast<int>(ceil_div64(k_bytes, 128));
+  a.f16_ops = p.f16_operands ? 1 : 0;
   a.total_tiles = a.tiles_m * a.tiles_n;
   a.kg = kg;
   a.scale_a = p.scale_a;

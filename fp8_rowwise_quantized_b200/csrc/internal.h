@@ -58,6 +58,9 @@ struct GemmProblem {
   const void* lr_act;
   const void* lr_up;
   int lr_rank;
+  // FP8 path only: a and b hold f16 [rows, K] instead of E4M3 (kind::f16 MMAs, K
+  // tiles of 64 elements); scale_a [M] and scale_b [N] scale the rows and columns
+  bool f16_operands;
 };
 
 // whole_buffers: only tile widths whose two TMEM accumulator buffers do not share
@@ -101,9 +104,10 @@ cudaError_t launch_w4a16_linear(const void* x, int64_t M, int64_t K, const uint8
 // INT4 W4A4 (int4.cu): K % 64 == 0; x, q, w 16-byte aligned.
 cudaError_t launch_int4_quantize(const void* x, int64_t M, int64_t K, uint8_t* q, float* scale,
                                  cudaStream_t s);
-cudaError_t launch_int4_gemm(const uint8_t* xq, const float* xs, int64_t M, int64_t K,
-                             const uint8_t* wq, const float* ws, int64_t N, const float* bias,
-                             void* y, int* status, uint64_t timeout_ns, cudaStream_t s);
+// INT4 rows [rows, K/2] + group scales [rows, K/64] -> f16 [rows, K] (16-byte aligned)
+// and the row factors [rows] (out = RN16(RN32(q * s * 2^-e)), factor = 2^e).
+cudaError_t launch_int4_dequant_f16(const uint8_t* q, const float* scale, int64_t rows, int64_t K,
+                                    void* out, float* factor, cudaStream_t s);
 cudaError_t launch_fp8r_quantize_rows(const void* x, int64_t M, int64_t K, uint8_t* xq,
                                       float* x_scale, cudaStream_t s);
 cudaError_t launch_global_scale(const void* x, int64_t n, float* out, cudaStream_t s);

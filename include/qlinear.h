@@ -276,35 +276,48 @@ int nvfp4_linear_noalloc(const void* x, int64_t M, int64_t K,
 int int4_quantize_rows(const void* x, int64_t M, int64_t K, uint8_t* q, float* scale,
                        ql_stream_t stream);
 
-/* Bytes of workspace int4_linear needs (0 on bad sizes): the quantized rows of x. */
+/* Bytes of workspace int4_linear needs (0 on bad sizes): the quantized rows of x
+ * (codes, then scales, each part 1 KB aligned) followed by the workspace of
+ * int4_linear_gemm. */
 size_t int4_linear_workspace_size(int64_t M, int64_t K, int64_t N);
 
 /* INT4 W4A4 linear forward (no low-rank branch):
  *   Y[m, n] = bf16( sum_g x_scale[m,g] w_scale[n,g] sum_{k in g} qx[m,k] qw[n,k] + bias[n] )
- * quantizing x at run time (int4_quantize_rows into the workspace), then a GEMM whose
- * per-group integer sums come from tcgen05 int8 MMAs (the 4-bit codes widened to int8
- * in shared memory) and are scaled and added in fp32 on the CUDA cores (per-group fp32
- * scales have no block-scaled tcgen05 form).
+ * quantizing x at run time (int4_quantize_rows into the workspace), then
+ * int4_linear_gemm. Per-group fp32 scales have no block-scaled tcgen05 form, so the
+ * GEMM moves them into the operands: both INT4 operands are dequantized to f16 with
+ * one power-of-two factor per row, RN16(RN32(q * s * 2^-e)), and one f16 tensor-core
+ * GEMM (fp32 accumulation) applies the factors in its epilogue. Each product is
+ * within 2^-10 of its exact value, so |Y - exact| <= 2^-10 * sum |x w| plus the fp32
+ * accumulation's rounding (the INT4 codes and scales themselves are exact).
  *   x        bf16 [M, K]
  *   w        uint8 [N, K/2] INT4 weight codes (as int4_quantize_rows writes them)
  *   w_scale  fp32 [N, K/64] group scales
  *   bias     fp32 [N] or NULL;  y  bf16 [M, N] (output)
  *   workspace >= int4_linear_workspace_size(M, K, N) bytes, 16-byte aligned
- * Requires K >= 64, K % 64 == 0; x, w 16-byte aligned. */
+ * Requires K >= 64, K % 64 == 0; x, w 16-byte aligned. Four launches (quantize,
+ * two dequantizations, GEMM). */
 int int4_linear(const void* x, int64_t M, int64_t K, const uint8_t* w, const float* w_scale,
                 int64_t N, const float* bias, void* y, void* workspace, size_t workspace_bytes,
                 ql_stream_t stream);
 
+/* Bytes of workspace int4_linear_gemm needs (0 on bad sizes): f16 copies of both
+ * operands and their row factors, 2 * (M + N) * K + 4 * (M + N) bytes plus alignment. */
+size_t int4_linear_gemm_workspace_size(int64_t M, int64_t K, int64_t N);
+
 /* The GEMM half of int4_linear, from activations quantized by int4_quantize_rows:
- * xq uint8 [M, K/2], x_scale fp32 [M, K/64]; w, w_scale, bias and y as for int4_linear.
+ * xq uint8 [M, K/2], x_scale fp32 [M, K/64]; w, w_scale, bias and y as for int4_linear;
+ * workspace >= int4_linear_gemm_workspace_size(M, K, N) bytes, 16-byte aligned, for
+ * the f16 operands (owned by the caller, overwritten).
  * Requires K >= 64, K % 64 == 0; xq and w 16-byte aligned, the scales and bias 4-byte,
- * y 2-byte aligned (a 16-byte-aligned y with N % 8 == 0 takes 16-byte stores).
+ * y 2-byte aligned (a 16-byte-aligned y with N % 8 == 0 takes TMA stores).
  * Errors: QL_ERR_INVALID_ARG (null pointer, size <= 0), QL_ERR_SHAPE, QL_ERR_ALIGN,
- * QL_ERR_DEVICE, QL_ERR_LAUNCH. Every wait inside the kernel is bounded; one that runs
- * out sets the device status word (read with ql_read_device_status) to QL_ERR_TIMEOUT. */
+ * QL_ERR_WORKSPACE, QL_ERR_DEVICE, QL_ERR_LAUNCH. Every wait inside the GEMM is
+ * bounded; one that runs out sets the device status word (read with
+ * ql_read_device_status) to QL_ERR_TIMEOUT. */
 int int4_linear_gemm(const uint8_t* xq, const float* x_scale, int64_t M, int64_t K,
                      const uint8_t* w, const float* w_scale, int64_t N, const float* bias,
-                     void* y, ql_stream_t stream);
+                     void* y, void* workspace, size_t workspace_bytes, ql_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* fp8r (FP8 row-wise)                                                       */

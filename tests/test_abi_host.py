@@ -90,20 +90,30 @@ def test_argument_errors_before_device():
     assert lib.int4_quantize_rows(fake, M, 96, fake, fake, None) == 2
     assert lib.int4_linear(fake, M, K, fake, fake, N, None, fake, None, 1 << 20, None) == 5
     assert lib.int4_linear_workspace_size(M, 96, N) == 0
-    # workspace = activation codes then their group scales, each 1 KB-aligned
-    assert lib.int4_linear_workspace_size(M, K, N) == M * K // 2 + M * (K // 64) * 4
-    assert lib.int4_linear_workspace_size(3, 64, 1) == 1024 + 1024
-    assert lib.int4_linear(fake, M, K, fake, fake, N, None, fake, odd, 1 << 20, None) == 3
-    # int4_linear_gemm: null pointer, K % 64, misaligned codes / scales / bias / y
-    assert lib.int4_linear_gemm(None, fake, M, K, fake, fake, N, None, fake, None) == 1
-    assert lib.int4_linear_gemm(fake, fake, M, K, fake, fake, 0, None, fake, None) == 1
-    assert lib.int4_linear_gemm(fake, fake, M, 96, fake, fake, N, None, fake, None) == 2
-    assert lib.int4_linear_gemm(odd, fake, M, K, fake, fake, N, None, fake, None) == 3
-    assert lib.int4_linear_gemm(fake, fake, M, K, odd, fake, N, None, fake, None) == 3
-    assert lib.int4_linear_gemm(fake, fake + 2, M, K, fake, fake, N, None, fake, None) == 3
-    assert lib.int4_linear_gemm(fake, fake, M, K, fake, fake + 2, N, None, fake, None) == 3
-    assert lib.int4_linear_gemm(fake, fake, M, K, fake, fake, N, fake + 2, fake, None) == 3
-    assert lib.int4_linear_gemm(fake, fake, M, K, fake, fake, N, None, fake + 1, None) == 3
+    assert lib.int4_linear_gemm_workspace_size(M, 96, N) == 0
+    # GEMM workspace: f16 x [M, K], x row factors [M], f16 w [N, K], w row factors [N],
+    # each part 1 KB-aligned
+    al = lambda b: -(-b // 1024) * 1024
+    gws = al(2 * M * K) + al(4 * M) + al(2 * N * K) + al(4 * N)
+    assert lib.int4_linear_gemm_workspace_size(M, K, N) == gws
+    # int4_linear: activation codes, then their group scales, then the GEMM workspace
+    assert lib.int4_linear_workspace_size(M, K, N) == al(M * K // 2) + al(M * (K // 64) * 4) + gws
+    assert lib.int4_linear_workspace_size(3, 64, 1) == 1024 * 6
+    assert lib.int4_linear(fake, M, K, fake, fake, N, None, fake, odd, 1 << 30, None) == 3
+    # int4_linear_gemm: null pointer, K % 64, workspace, misaligned codes / scales / bias / y
+    big = 1 << 30
+    assert lib.int4_linear_gemm(None, fake, M, K, fake, fake, N, None, fake, fake, big, None) == 1
+    assert lib.int4_linear_gemm(fake, fake, M, K, fake, fake, 0, None, fake, fake, big, None) == 1
+    assert lib.int4_linear_gemm(fake, fake, M, 96, fake, fake, N, None, fake, fake, big, None) == 2
+    assert lib.int4_linear_gemm(fake, fake, M, K, fake, fake, N, None, fake, None, big, None) == 5
+    assert lib.int4_linear_gemm(fake, fake, M, K, fake, fake, N, None, fake, fake, gws - 1, None) == 5
+    assert lib.int4_linear_gemm(odd, fake, M, K, fake, fake, N, None, fake, fake, big, None) == 3
+    assert lib.int4_linear_gemm(fake, fake, M, K, odd, fake, N, None, fake, fake, big, None) == 3
+    assert lib.int4_linear_gemm(fake, fake + 2, M, K, fake, fake, N, None, fake, fake, big, None) == 3
+    assert lib.int4_linear_gemm(fake, fake, M, K, fake, fake + 2, N, None, fake, fake, big, None) == 3
+    assert lib.int4_linear_gemm(fake, fake, M, K, fake, fake, N, fake + 2, fake, fake, big, None) == 3
+    assert lib.int4_linear_gemm(fake, fake, M, K, fake, fake, N, None, fake + 1, fake, big, None) == 3
+    assert lib.int4_linear_gemm(fake, fake, M, K, fake, fake, N, None, fake, odd, big, None) == 3
     # w4a16: null weight, K % 32, misaligned x, odd w_scale
     assert lib.w4a16_linear(fake, 1, K, None, fake, N, fake, None, fake, None) == 1
     assert lib.w4a16_linear(fake, 1, 48, fake, fake, N, fake, None, fake, None) == 2

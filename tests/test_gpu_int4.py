@@ -120,3 +120,63 @@ def test_int4_gemm_unaligned_output_matches_aligned():
     assert bool(torch.isnan(buf[:1]).all()) and bool(torch.isnan(buf[1 + M * N:]).all())
     _, y64, T = c.reference()
     check_linear(y1, y64, T, "int4 200x320x264")
+
+
+def _f16_operand(codes, scales, K):
+    """numpy statement of the GEMM's f16 operand: per row e = E - 12 for the largest
+    group scale m 2^E (m in [0.5, 1)), values RN16(RN32(q * (s * 2^-e))), factor 2^e."""
+    rows = codes.shape[0]
+    lo = (codes.astype(np.int16) << 12).astype(np.int16) >> 12
+    hi = (codes.astype(np.int16) << 8).astype(np.int16) >> 12
+    qv = np.empty((rows, K), dtype=np.float32)
+    qv[:, 0::2] = lo
+    qv[:, 1::2] = hi
+    mx = np.abs(scales).max(axis=1)
+    e = np.where(mx > 0, np.frexp(mx)[1] - 12, 0).astype(np.int32)
+    s_scaled = np.ldexp(scales.astype(np.float64), -e[:, None]).astype(np.float32)
+    vals = (qv * np.repeat(s_scaled, 64, axis=1)).astype(np.float32).astype(np.float16)
+    return vals, np.ldexp(np.float32(1.0), e).astype(np.float32)
+
+
+def test_int4_gemm_f16_operands_bit_exact():
+    # the workspace of int4_linear_gemm holds f16 x [M, K], x factors [M], f16 w [N, K],
+    # w factors [N] (1 KB-aligned parts); both dequantizations match numpy bit for bit,
+    # including a zero row and a row whose groups span 2^30 in scale
+    M, K, N = 70, 320, 130
+    c = Int4Case(M, K, N, seed=8)
+    x = c.x.clone()
+    x[3] = 0
+    x[5] = x[5] * torch.logspace(-9, 0, K, base=10.0).to(torch.bfloat16)
+    x = x.to(torch.bfloat16)
+    xq, xs = q.int4_quantize_rows(to_dev(x))
+    ws = torch.empty(q.int4_linear_gemm_workspace_size(M, K, N), dtype=torch.uint8, device="cuda")
+    q.int4_linear_gemm(xq, xs, to_dev(c.wq), to_dev(c.ws), workspace=ws)
+    torch.cuda.synchronize()
+    al = lambda b: -(-b // 1024) * 1024
+    buf = ws.cpu().numpy()
+    o = 0
+    xh = buf[o:o + 2 * M * K].view(np.float16).reshape(M, K); o += al(2 * M * K)
+    xf = buf[o:o + 4 * M].view(np.float32); o += al(4 * M)
+    wh = buf[o:o + 2 * N * K].view(np.float16).reshape(N, K); o += al(2 * N * K)
+    wf = buf[o:o + 4 * N].view(np.float32)
+    ex, efx = _f16_operand(xq.cpu().numpy(), xs.cpu().numpy(), K)
+    ew, efw = _f16_operand(c.wq, c.ws, K)
+    np.testing.assert_array_equal(xh.view(np.uint16), ex.view(np.uint16))
+    np.testing.assert_array_equal(xf, efx)
+    np.testing.assert_array_equal(wh.view(np.uint16), ew.view(np.uint16))
+    np.testing.assert_array_equal(wf, efw)
+    assert np.abs(xh.astype(np.float32)).max() < 2.0 ** 15
+
+
+def test_int4_linear_same_sign_products():
+    # every product x w >= 0, so the operands' rounding errors cannot cancel in sign:
+    # the result still meets the linear's bound (each product within 2^-10 of exact)
+    M, K, N = 256, 3072, 256
+    g = torch.Generator().manual_seed(9)
+    c = Int4Case(M, K, N, seed=9)
+    c.x = (torch.rand(M, K, generator=g) * 4.0).to(torch.bfloat16)
+    w = (torch.rand(N, K, generator=g) * 0.05).to(torch.bfloat16)
+    c.wq, c.ws = oracle.int4_quantize(w)
+    y = c.run()
+    _, y64, T = c.reference()
+    check_linear(y, y64, T, "int4 same-sign 256x3072x256")
