@@ -61,7 +61,6 @@ constexpr int kEpiBufsPerWarp = 1;
 struct GemmArgs {
   int M, N, K;
   int tiles_m, tiles_n, num_k_tiles, total_tiles;
-  int f16_ops;              // FP8 path: the operands are f16 (kind::f16 MMAs)
   int64_t kg;               // FP4: 64-element scale groups per row (padded)
   const float* scale_a;     // FP4: input_scale (scalar)   FP8: x_scale [M]
   const float* scale_b;     // FP4: weight_scale_2 (scalar) FP8: w_scale [N]
@@ -488,7 +487,8 @@ constexpr int block_threads() {
                                    : 64 + 32 * epi_warps<MODE>() + (AROWS < kRowsPerCta ? 32 : 0);
 }
 
-template <bool FP4, int BN, int CG, int MODE, int AROWS = kRowsPerCta>
+// F16 (FP8 path, plain mode): the operands are f16 and the MMAs kind::f16.
+template <bool FP4, int BN, int CG, int MODE, int AROWS = kRowsPerCta, bool F16 = false>
 __global__ void __launch_bounds__(block_threads<MODE, AROWS>(), 1)
 qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
              const __grid_constant__ CUtensorMap tmap_sfa,
@@ -981,7 +981,7 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
               const uint64_t ad = smem_desc(a_addr + kb * 32, 16, 1024, 2);
               const uint64_t bd = smem_desc(b_addr + kb * 32, 16, 1024, 2);
               const uint32_t accum = (kt | kb) != 0 ? 1u : 0u;
-              if (args.f16_ops) {
+              if constexpr (F16) {
                 if constexpr (CG == 2)
                   mma_bf16_pair(d_tmem, ad, bd, C::IDESC, accum);
                 else
@@ -1351,11 +1351,13 @@ bool encode_2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, uin
 
 namespace {
 
-template <bool FP4, int BN, int CG, int MODE, int AROWS = kRowsPerCta>
+template <bool FP4, int BN, int CG, int MODE, int AROWS = kRowsPerCta, bool F16 = false>
 cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
   using Cf = Cfg<FP4, BN, CG, AROWS>;
   constexpr bool FUSED = MODE == kModeSingleLaunch;
-  auto kern = qgemm_kernel<FP4, BN, CG, MODE, AROWS>;
+  static_assert(!F16 || (!FP4 && MODE == kModePlain), "f16 operands: FP8 path, plain mode");
+  auto kern = qgemm_kernel<FP4, BN, CG, MODE, AROWS, F16>;
+  if (p.f16_operands != F16) return cudaErrorInvalidValue;
   if (AROWS < kRowsPerCta && p.M > AROWS) return cudaErrorInvalidValue;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -1373,8 +1375,7 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
 
-  if (p.f16_operands && (FP4 || MODE != kModePlain)) return cudaErrorInvalidValue;
-  const int64_t k_bytes = FP4 ? p.K / 2 : (p.f16_operands ? 2 * p.K : p.K);
+  const int64_t k_bytes = FP4 ? p.K / 2 : (F16 ? 2 * p.K : p.K);
   CUtensorMap ta, tb, tsa, tsb, ty, tla, tlb;
   std::memset(&tla, 0, sizeof(tla));
   std::memset(&tlb, 0, sizeof(tlb));
@@ -1447,7 +1448,6 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
   a.tiles_n = static_cast<int>(ceil_div64(p.N, BN));
   // a K tile is 128 bytes of every row: 256 E2M1, 128 E4M3 or 64 f16 elements
   a.num_k_tiles = static_cast<int>(ceil_div64(k_bytes, 128));
-  a.f16_ops = p.f16_operands ? 1 : 0;
   a.total_tiles = a.tiles_m * a.tiles_n;
   a.kg = kg;
   a.scale_a = p.scale_a;
@@ -1655,6 +1655,22 @@ cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream) {
     QL_SCASE(128, 32)
     QL_SCASE(128, 64)
 #undef QL_SCASE
+    return cudaErrorInvalidValue;
+  }
+  if (p.f16_operands) {
+    if (p.fp4) return cudaErrorInvalidValue;
+#define QL_HCASE(BN_, CG_) \
+  if (p.bn == BN_ && p.cg == CG_)    \
+    return launch_typed<false, BN_, CG_, kModePlain, kRowsPerCta, true>(p, stream);
+    QL_HCASE(128, 1)
+    QL_HCASE(192, 1)
+    QL_HCASE(256, 1)
+    QL_HCASE(224, 1)
+    QL_HCASE(224, 2)
+    QL_HCASE(128, 2)
+    QL_HCASE(192, 2)
+    QL_HCASE(256, 2)
+#undef QL_HCASE
     return cudaErrorInvalidValue;
   }
 #define QL_CASE(FP4_, BN_, CG_) \
