@@ -5,7 +5,10 @@ N = 12288, bf16 in / bf16 out, synthetic seeded inputs.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One step = one nvfp4_linear call (prologue kernel + GEMM kernel). Consecutive
+One step = one nvfp4_linear_laid_out call (the activations' quantization kernel +
+the GEMM kernel) on weight scales laid out once at set-up, like the weights' own
+quantization; the same step through nvfp4_linear, which lays the weight scales out
+in every call, is reported as per_call_weight_layout. Consecutive
 steps cycle through buffer sets (x, weights, y, workspace) that together hold at
 least four times the L2, so every step reads its operands from HBM; the K timed
 steps, each bracketed by CUDA event records, are captured in one CUDA graph and
@@ -189,10 +192,20 @@ class Nvfp4Layer:
         self.work = torch.empty(q.nvfp4_linear_workspace_size(M, K, N), dtype=torch.uint8,
                                 device=device)
         self.q = q
+        # the weight scales laid out once for the tile width a call of this size uses
+        # (a load-time step, like the weight's quantization above); skinny tile widths
+        # lay them out inside the GEMM and have no atoms
+        self.bn = q.tile_config(M, N, K)[0]
+        self.atoms = (q.nvfp4_layout_weight_scales(self.ws, self.bn)
+                      if self.bn in (128, 192, 224, 256) else None)
 
     def step(self):
         self.q.nvfp4_linear(self.x, self.wq, self.ws, self.gw, self.gx, bias=self.bias, y=self.y,
                             workspace=self.work)
+
+    def step_laid_out(self):
+        self.q.nvfp4_linear_laid_out(self.x, self.wq, self.atoms, self.bn, self.gw, self.gx,
+                                     bias=self.bias, y=self.y, workspace=self.work)
 
     def prologue(self):
         self.q.nvfp4_linear_prologue(self.x, self.ws, self.gx, self.work)
@@ -350,7 +363,7 @@ class Nvfp4Rotation:
         import torch
         self.L = layer
         per = sum(t.numel() * t.element_size() for t in
-                  (layer.x, layer.wq, layer.ws, layer.y, layer.work) if t is not None)
+                  (layer.x, layer.wq, layer.ws, layer.y, layer.work, layer.atoms) if t is not None)
         if layer.bias is not None:
             per += layer.bias.numel() * 4
         self.R = max(2, -(-min_bytes // per))
@@ -359,9 +372,11 @@ class Nvfp4Rotation:
         def clone(t):
             return None if t is None else t.clone()
         self.sets = [(layer.x, layer.wq, layer.ws, layer.bias, layer.y, layer.work)]
+        self.atoms = [layer.atoms]
         for _ in range(self.R - 1):
             self.sets.append((clone(layer.x), clone(layer.wq), clone(layer.ws), clone(layer.bias),
                               torch.empty_like(layer.y), torch.empty_like(layer.work)))
+            self.atoms.append(clone(layer.atoms))
         self.i = 0
 
     def _next(self):
@@ -372,6 +387,12 @@ class Nvfp4Rotation:
     def step(self):
         x, wq, ws, b, y, work = self._next()
         self.L.q.nvfp4_linear(x, wq, ws, self.L.gw, self.L.gx, bias=b, y=y, workspace=work)
+
+    def step_laid_out(self):
+        atoms = self.atoms[self.i]
+        x, wq, ws, b, y, work = self._next()
+        self.L.q.nvfp4_linear_laid_out(x, wq, atoms, self.L.bn, self.L.gw, self.L.gx, bias=b, y=y,
+                                       workspace=work)
 
     def prologue_all(self):
         for x, wq, ws, b, y, work in self.sets:
@@ -796,10 +817,13 @@ def run_ours(args):
     # timed steps, each bracketed by CUDA event records on the launching stream, are
     # captured in one CUDA graph and replayed once (so no host launch gap lands
     # inside a step); the value is the median step. The clock sampler runs over the
-    # warm-up and the timed steps.
+    # warm-up and the timed steps. A step is nvfp4_linear_laid_out: the activations'
+    # quantization and the GEMM, on weight scales laid out once at set-up (like the
+    # weights' own quantization); the same step laying them out every call is
+    # reported beside it (per_call_weight_layout).
     rot = Nvfp4Rotation(layer)
     for _ in range(rot.R):  # every set once before the capture (lazy set-up on the host)
-        rot.step()
+        rot.step_laid_out()
     torch.cuda.synchronize()
     starts = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(args.steps)]
@@ -811,13 +835,13 @@ def run_ours(args):
         with torch.cuda.graph(timed, stream=side):
             for i in range(args.steps):
                 starts[i].record(side)
-                rot.step()
+                rot.step_laid_out()
                 ends[i].record(side)
     stream.wait_stream(side)
     host_s = time.perf_counter() - t_host
     with ClockSampler(local, period_s=0.002) as clk:
         for _ in range(args.warmup):
-            rot.step()
+            rot.step_laid_out()
         torch.cuda.synchronize()
         barrier(device)
         torch.cuda.synchronize()
@@ -839,13 +863,17 @@ def run_ours(args):
     # operands come from HBM, Y's lines start clean), and warm L2 (the same
     # buffers every step, no flush)
     n_alt = max(20, min(args.steps, 200))
-    fl_ms, _ = time_events(layer.step, n_alt, 3, flush, stream)
-    warm_ms, _ = time_events(layer.step, n_alt, 3, None, stream)
+    fl_ms, _ = time_events(layer.step_laid_out, n_alt, 3, flush, stream)
+    warm_ms, _ = time_events(layer.step_laid_out, n_alt, 3, None, stream)
     fl_ms, fl_val = aggregate(fl_ms, flops, world, device)
     warm_ms, warm_val = aggregate(warm_ms, flops, world, device)
     # and as one CUDA graph per cycle of buffer sets (no host launch gaps at all)
-    graph_ms = time_graph_rotation(rot.step, rot.R, max(3, min(args.steps // rot.R, 50)), stream)
+    graph_ms = time_graph_rotation(rot.step_laid_out, rot.R, max(3, min(args.steps // rot.R, 50)),
+                                   stream)
     graph_ms, graph_val = aggregate(graph_ms, flops, world, device)
+    # nvfp4_linear, which lays the weight scales out inside every call
+    pc_ms = time_graph_rotation(rot.step, rot.R, max(3, min(args.steps // rot.R, 50)), stream)
+    pc_ms, pc_val = aggregate(pc_ms, flops, world, device)
 
     # --------------------------------------------------- roofline of the GEMM kernel
     # the GEMM alone, the prologue alone and the activation quantizer alone, each
@@ -904,8 +932,8 @@ def run_ours(args):
 
         def e2e_step():
             x_dev.copy_(x_pin, non_blocking=True)
-            q.nvfp4_linear(x_dev, layer.wq, layer.ws, layer.gw, layer.gx, y=layer.y,
-                           workspace=layer.work)
+            q.nvfp4_linear_laid_out(x_dev, layer.wq, layer.atoms, layer.bn, layer.gw, layer.gx,
+                                    y=layer.y, workspace=layer.work)
             y_pin.copy_(layer.y, non_blocking=True)
 
         e_steps = max(10, min(args.steps, 50))
@@ -1011,7 +1039,10 @@ def run_ours(args):
                          f"{rot.bytes_per_set / 1e6:.0f} MB (x, weights, y, workspace) cycled, "
                          "one per step; value from the median step",
                    "timing": "CUDA events around each step, recorded inside one CUDA graph "
-                             "of the K steps (no host launch gaps)"},
+                             "of the K steps (no host launch gaps)",
+                   "weight_scales": f"laid out once at set-up for {layer.bn}-row tiles "
+                                    "(nvfp4_layout_weight_scales), like the weights' own "
+                                    "quantization; a step is nvfp4_linear_laid_out"},
         "frac_of_fp4_peak": value / world / fp4_peak,
         "step_stats": {"median_ms": ms, "mean_ms": mean_ms,
                        "min_ms": min(step_times), "max_ms": max(step_times),
@@ -1026,6 +1057,9 @@ def run_ours(args):
         "l2_rotating_graph": {"value": graph_val / 1e12, "ms_per_step": graph_ms,
                               "how": "the rotating buffer sets, one CUDA graph per cycle of "
                                      "sets; mean over replays"},
+        "per_call_weight_layout": {"value": pc_val / 1e12, "ms_per_step": pc_ms,
+                                   "how": "nvfp4_linear (the weight scales laid out inside "
+                                          "every call), rotating graph as l2_rotating_graph"},
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
@@ -1044,7 +1078,8 @@ def run_ours(args):
 
 def run_profile(args):
     """Short fixed sequence for profilers: `--profile <piece>` runs `--steps` calls
-    of one piece of the headline workload (no flushes, no timing): `step`,
+    of one piece of the headline workload (no flushes, no timing): `step` (the
+    headline step, nvfp4_linear_laid_out), `step_per_call_layout` (nvfp4_linear),
     `prologue`, `gemm`, `quant` (activation quantization alone), `mlp_fused` (the MLP
     block with the GELU-quantize epilogue), `svdq` (the rank-32 svdq layer), `fp8r_step`,
     `fp8r_quant`, `fp8r_gemm`, `int4` (the INT4 W4A4 layer on the headline shape),
@@ -1081,7 +1116,8 @@ def run_profile(args):
         L.prologue()
         xq = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
         xs = torch.empty((M, K // 16), dtype=torch.uint8, device=device)
-        fn = {"step": L.step, "prologue": L.prologue, "gemm": L.gemm,
+        fn = {"step": L.step_laid_out, "step_per_call_layout": L.step, "prologue": L.prologue,
+              "gemm": L.gemm,
               "quant": lambda: L.q.nvfp4_quantize_act(L.x, L.gx, xq, xs)}[args.profile]
     for _ in range(args.steps):
         fn()
@@ -1103,7 +1139,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prior-art", action="store_true",
                     help="skip timing FlashInfer's NVFP4 kernels (context only)")
-    ap.add_argument("--profile", choices=["step", "prologue", "gemm", "quant", "mlp_fused", "svdq",
+    ap.add_argument("--profile", choices=["step", "step_per_call_layout", "prologue", "gemm",
+                                          "quant", "mlp_fused", "svdq",
                                           "fp8r_step", "fp8r_quant", "fp8r_gemm", "w4a16", "int4",
                                           "skinny_16_3072", "skinny_16_12288",
                                           "skinny_256_12288"], default=None,

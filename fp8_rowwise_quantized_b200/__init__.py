@@ -163,6 +163,55 @@ def nvfp4_linear(x: torch.Tensor, w: torch.Tensor, w_scale: torch.Tensor,
     return y
 
 
+def nvfp4_weight_scale_atoms_size(N: int, K: int, bn: int) -> int:
+    return int(_lib.load().nvfp4_weight_scale_atoms_size(N, K, bn))
+
+
+def nvfp4_layout_weight_scales(w_scale: torch.Tensor, bn: int,
+                               atoms: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The row-major E4M3 weight scales [N, K/16] laid out once for GEMM tiles of bn
+    rows (128, 192, 224 or 256): the atoms nvfp4_linear_laid_out reads."""
+    _need(w_scale, "w_scale", torch.uint8, 2)
+    dev = w_scale.device
+    N, K = w_scale.shape[0], w_scale.shape[1] * 16
+    size = nvfp4_weight_scale_atoms_size(N, K, bn)
+    if size == 0:
+        raise ValueError(f"no weight-scale layout for N={N}, K={K}, bn={bn}")
+    atoms = _workspace(size, dev, atoms)
+    _call("nvfp4_layout_weight_scales", dev, _ptr(w_scale), N, K, int(bn), _ptr(atoms),
+          atoms.numel())
+    return atoms
+
+
+def nvfp4_linear_laid_out(x: torch.Tensor, w: torch.Tensor, w_scale_atoms: torch.Tensor, bn: int,
+                          weight_scale_2: torch.Tensor, input_scale: torch.Tensor,
+                          bias: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
+                          workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """nvfp4_linear on weight scales laid out once by nvfp4_layout_weight_scales for
+    tiles of bn rows (the call runs its GEMM at that tile width)."""
+    _need(x, "x", torch.bfloat16, 2)
+    dev = x.device
+    M, K = x.shape
+    _need(w, "w", torch.uint8, 2, device=dev)
+    N = w.shape[0]
+    if w.shape[1] * 2 != K:
+        raise ValueError(f"w must have K/2 = {K // 2} bytes per row, got {w.shape[1]}")
+    size = nvfp4_weight_scale_atoms_size(N, K, bn)
+    if size == 0:
+        raise ValueError(f"no weight-scale layout for N={N}, K={K}, bn={bn}")
+    _need(w_scale_atoms, "w_scale_atoms", torch.uint8, 1, device=dev)
+    if w_scale_atoms.numel() < size:
+        raise ValueError(f"w_scale_atoms holds {w_scale_atoms.numel()} bytes, needs {size}")
+    _scalar(weight_scale_2, "weight_scale_2", dev)
+    _scalar(input_scale, "input_scale", dev)
+    _bias(bias, N, dev)
+    y = _out(y, M, N, dev)
+    ws = _workspace(nvfp4_linear_workspace_size(M, K, N), dev, workspace)
+    _call("nvfp4_linear_laid_out", dev, _ptr(x), M, K, _ptr(w), _ptr(w_scale_atoms), int(bn), N,
+          _ptr(weight_scale_2), _ptr(input_scale), _ptr(bias), _ptr(y), _ptr(ws), ws.numel())
+    return y
+
+
 def nvfp4_linear_single_launch(x: torch.Tensor, w: torch.Tensor, w_scale: torch.Tensor,
                                weight_scale_2: torch.Tensor, input_scale: torch.Tensor,
                                bias: Optional[torch.Tensor] = None,

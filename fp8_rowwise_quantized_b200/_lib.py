@@ -26,6 +26,10 @@ _vp, _i64, _sz, _u8p, _f32p, _ip = C.c_void_p, C.c_int64, C.c_size_t, C.c_void_p
 SIGNATURES = {
     "nvfp4_quantize_act": (C.c_int, [_vp, _i64, _i64, _f32p, _u8p, _u8p, _vp]),
     "nvfp4_linear_workspace_size": (C.c_size_t, [_i64, _i64, _i64]),
+    "nvfp4_weight_scale_atoms_size": (C.c_size_t, [_i64, _i64, C.c_int]),
+    "nvfp4_layout_weight_scales": (C.c_int, [_u8p, _i64, _i64, C.c_int, _u8p, _sz, _vp]),
+    "nvfp4_linear_laid_out": (C.c_int, [_vp, _i64, _i64, _u8p, _u8p, C.c_int, _i64, _f32p, _f32p,
+                                        _f32p, _vp, _vp, _sz, _vp]),
     "nvfp4_linear": (C.c_int, [_vp, _i64, _i64, _u8p, _u8p, _i64, _f32p, _f32p, _f32p, _vp, _vp,
                                _sz, _vp]),
     "nvfp4_linear_single_launch": (C.c_int, [_vp, _i64, _i64, _u8p, _u8p, _i64, _f32p, _f32p,

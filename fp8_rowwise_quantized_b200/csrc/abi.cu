@@ -364,6 +364,77 @@ int nvfp4_linear(const void* x, int64_t M, int64_t K, const uint8_t* w, const ui
                          workspace_bytes, stream, true);
 }
 
+static bool laid_out_width_ok(int bn) { return bn == 128 || bn == 192 || bn == 224 || bn == 256; }
+
+size_t nvfp4_weight_scale_atoms_size(int64_t N, int64_t K, int bn) {
+  if (!nvfp4_shape_ok(1, K, N) || !laid_out_width_ok(bn)) return 0;
+  const int64_t na = (bn + 127) / 128;
+  return static_cast<size_t>(ql::ceil_div64(N, bn) * ql::sf_kgroups(K) * na) * ql::kSfAtomBytes;
+}
+
+int nvfp4_layout_weight_scales(const uint8_t* w_scale, int64_t N, int64_t K, int bn,
+                               uint8_t* atoms, size_t atoms_bytes, ql_stream_t stream) {
+  if (!w_scale || !atoms || N <= 0 || K <= 0) return QL_ERR_INVALID_ARG;
+  if (!nvfp4_shape_ok(1, K, N)) return fail_shape("nvfp4: needs K >= 32 and K % 32 == 0");
+  if (!laid_out_width_ok(bn)) return fail_shape("weight-scale layout: bn must be 128, 192, 224 or 256");
+  if (atoms_bytes < nvfp4_weight_scale_atoms_size(N, K, bn)) return QL_ERR_WORKSPACE;
+  if (!aligned16(atoms)) return QL_ERR_ALIGN;
+  int rc = check_device(nullptr);
+  if (rc != QL_OK) return rc;
+  cudaError_t e = ql::launch_nvfp4_weight_atoms(w_scale, K, N, bn, atoms,
+                                                reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QL_OK : record(e, "nvfp4_layout_weight_scales");
+}
+
+int nvfp4_linear_laid_out(const void* x, int64_t M, int64_t K, const uint8_t* w,
+                          const uint8_t* w_scale_atoms, int bn, int64_t N,
+                          const float* weight_scale_2, const float* input_scale,
+                          const float* bias, void* y, void* workspace, size_t workspace_bytes,
+                          ql_stream_t stream) {
+  if (!x || !w || !w_scale_atoms || !weight_scale_2 || !input_scale || !y || M <= 0 || N <= 0 ||
+      K <= 0)
+    return QL_ERR_INVALID_ARG;
+  if (!nvfp4_shape_ok(M, K, N)) return fail_shape("nvfp4: needs K >= 32 and K % 32 == 0");
+  if (!laid_out_width_ok(bn)) return fail_shape("weight-scale layout: bn must be 128, 192, 224 or 256");
+  if (!aligned16(x) || !aligned16(w) || !aligned16(w_scale_atoms) || !aligned16(y) ||
+      (bias && !aligned16(bias)))
+    return QL_ERR_ALIGN;
+  if (!workspace || workspace_bytes < nvfp4_linear_workspace_size(M, K, N)) return QL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return QL_ERR_ALIGN;
+  int dev = 0;
+  int rc = check_device(&dev);
+  if (rc != QL_OK) return rc;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // the activations only (the ordinary prologue kernel, its weight jobs empty)
+  cudaError_t e = ql::launch_nvfp4_prologue(x, M, K, nullptr, N, bn, input_scale,
+                                            static_cast<uint8_t*>(workspace), s, false, false);
+  if (e != cudaSuccess) return record(e, "nvfp4_linear_laid_out prologue");
+  const ql::Nvfp4Workspace L = ql::nvfp4_workspace(M, K, N, bn);
+  const uint8_t* ws = static_cast<const uint8_t*>(workspace);
+  ql::GemmProblem p{};
+  p.fp4 = true;
+  p.bn = bn;
+  p.cg = M >= 512 ? 2 : 1;  // the automatic choice's rule for pairs
+  p.arows = 0;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.a = ws + L.codes_off;
+  p.b = w;
+  p.sfa = ws + L.act_sf_off;
+  p.sfb = w_scale_atoms;
+  p.scale_a = input_scale;
+  p.scale_b = weight_scale_2;
+  p.bias = bias;
+  p.y = y;
+  p.status = status_ptr(dev);
+  p.timeout_ns = timeout_ns();
+  p.inject_fault = g_inject_fault.load();
+  p.pdl = true;
+  e = ql::launch_gemm(p, s);
+  return e == cudaSuccess ? QL_OK : record(e, "nvfp4_linear_laid_out gemm");
+}
+
 int nvfp4_linear_single_launch(const void* x, int64_t M, int64_t K, const uint8_t* w,
                                const uint8_t* w_scale, int64_t N, const float* weight_scale_2,
                                const float* input_scale, const float* bias, void* y,

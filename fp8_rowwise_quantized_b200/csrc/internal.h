@@ -79,10 +79,14 @@ cudaError_t launch_nvfp4_quantize_rowmajor(const void* x, int64_t M, int64_t K, 
                                            uint8_t* xq, uint8_t* xs, cudaStream_t s);
 // The prologue of nvfp4_linear: activations into codes + scale atoms, and (when
 // weight_layout) the weight scales into atoms for tiles of bn rows. Without the
-// weight layout it lets the next (skinny) GEMM launch at its start.
+// weight layout and with early, it lets the next (skinny) GEMM launch at its start.
 cudaError_t launch_nvfp4_prologue(const void* x, int64_t M, int64_t K, const uint8_t* w_scale,
                                   int64_t N, int bn, const float* input_scale, uint8_t* workspace,
-                                  cudaStream_t s, bool weight_layout = true);
+                                  cudaStream_t s, bool weight_layout = true, bool early = true);
+// The weight scales [N, K/16] into the atoms for tiles of bn rows, at `atoms`
+// (the layout of the workspace's weight part).
+cudaError_t launch_nvfp4_weight_atoms(const uint8_t* w_scale, int64_t K, int64_t N, int bn,
+                                      uint8_t* atoms, cudaStream_t s);
 // Weight-scale layout only (the activation part of the workspace is left as is).
 cudaError_t launch_nvfp4_weight_layout(const uint8_t* w_scale, int64_t M, int64_t K, int64_t N,
                                        int bn, const float* input_scale, uint8_t* workspace,

@@ -338,7 +338,8 @@ cudaError_t launch_nvfp4_quantize_rowmajor(const void* x, int64_t M, int64_t K, 
 
 cudaError_t launch_nvfp4_prologue(const void* x, int64_t M, int64_t K, const uint8_t* w_scale,
                                   int64_t N, int bn, const float* input_scale, uint8_t* workspace,
-                                  cudaStream_t s, bool weight_layout) {
+                                  cudaStream_t s, bool weight_layout, bool early) {
+  const bool early_kernel = !weight_layout && early;
   const Nvfp4Workspace L = nvfp4_workspace(M, K, N, bn);
   const int64_t KG = sf_kgroups(K);
   const int64_t rows = ceil_div64(M, 128) * 128;
@@ -353,7 +354,7 @@ cudaError_t launch_nvfp4_prologue(const void* x, int64_t M, int64_t K, const uin
     wave = resident_blocks(nvfp4_prologue_kernel<false>);
     wave_cache.store(wave, std::memory_order_relaxed);
   }
-  if (!weight_layout) {
+  if (early_kernel) {
     // An SM's split between L1 and shared memory follows the kernel whose blocks it
     // runs: with the split chosen for this kernel's 9 KB, a GEMM CTA (about 200 KB)
     // launched early could not join the prologue's blocks on an SM until they left.
@@ -370,12 +371,34 @@ cudaError_t launch_nvfp4_prologue(const void* x, int64_t M, int64_t K, const uin
   int64_t need = ceil_div64(rows * segs, kQuantThreads / 32);
   if (need < w_jobs) need = w_jobs;
   const int64_t blocks = need < wave ? need : wave;
-  auto kern = weight_layout ? nvfp4_prologue_kernel<false> : nvfp4_prologue_kernel<true>;
+  auto kern = early_kernel ? nvfp4_prologue_kernel<true> : nvfp4_prologue_kernel<false>;
   kern<<<static_cast<unsigned>(blocks), kQuantThreads, 0, s>>>(
       static_cast<const uint16_t*>(x), static_cast<int>(M), static_cast<int>(K), input_scale,
       workspace + L.codes_off, workspace + L.act_sf_off, static_cast<uint32_t>(rows),
       static_cast<uint32_t>(segs), static_cast<int>(KG), w_scale, N, bn, na, n_tiles, w_jobs,
       workspace + L.wgt_sf_off);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_nvfp4_weight_atoms(const uint8_t* w_scale, int64_t K, int64_t N, int bn,
+                                      uint8_t* atoms, cudaStream_t s) {
+  // the prologue kernel with no activation rows writes only the weight-scale atoms;
+  // its scalar input is then unused (read, not applied): the atoms buffer stands in
+  const int64_t KG = sf_kgroups(K);
+  const int na = (bn + 127) / 128;
+  const int64_t n_tiles = ceil_div64(N, bn);
+  const int64_t w_jobs = n_tiles * na * ceil_div64(KG, kWsGroups);
+  static std::atomic<int64_t> wave_cache{0};  // resident blocks of one wave (same on every B200)
+  int64_t wave = wave_cache.load(std::memory_order_relaxed);
+  if (wave == 0) {
+    wave = resident_blocks(nvfp4_prologue_kernel<false>);
+    wave_cache.store(wave, std::memory_order_relaxed);
+  }
+  const int64_t blocks = w_jobs < wave ? w_jobs : wave;
+  nvfp4_prologue_kernel<false><<<static_cast<unsigned>(blocks), kQuantThreads, 0, s>>>(
+      nullptr, 0, static_cast<int>(K), reinterpret_cast<const float*>(atoms), atoms, atoms, 0u,
+      static_cast<uint32_t>(ceil_div64(KG * 64, 1024)), static_cast<int>(KG), w_scale, N, bn, na,
+      n_tiles, w_jobs, atoms);
   return cudaGetLastError();
 }
 

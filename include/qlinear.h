@@ -171,6 +171,33 @@ int nvfp4_linear_quantized_input(int64_t M, int64_t K, const uint8_t* w, const u
 /* Bytes of workspace nvfp4_linear needs for this problem size (0 on bad sizes). */
 size_t nvfp4_linear_workspace_size(int64_t M, int64_t K, int64_t N);
 
+/* Weight block scales laid out once, for weights that do not change between calls
+ * (a load-time step, like the weight's own quantization; the pages' mm_fp4 takes its
+ * weight block scales in a prepared layout the same way). The tensor-core layout of
+ * the scales depends on the GEMM's tile width bn (tiles of 224 rows do not align
+ * with the 128-row scale atoms), so the atoms are made for one bn:
+ *   nvfp4_weight_scale_atoms_size(N, K, bn)  bytes of the atoms (0 on bad sizes or
+ *                                           a bn outside {128, 192, 224, 256})
+ *   nvfp4_layout_weight_scales(w_scale, N, K, bn, atoms, atoms_bytes, stream)
+ *     w_scale uint8 [N, K/16] E4M3 row-major (as for nvfp4_linear); atoms: the caller's
+ *     device buffer (16-byte aligned), written on `stream`.
+ * ql_tile_config(1, M, N, K, ...) gives the bn nvfp4_linear itself would use for M. */
+size_t nvfp4_weight_scale_atoms_size(int64_t N, int64_t K, int bn);
+int nvfp4_layout_weight_scales(const uint8_t* w_scale, int64_t N, int64_t K, int bn,
+                               uint8_t* atoms, size_t atoms_bytes, ql_stream_t stream);
+
+/* nvfp4_linear on weight scales laid out by nvfp4_layout_weight_scales for tiles of
+ * bn rows: the prologue quantizes only the activations, and the GEMM runs at tile
+ * width bn (CTA pairs from M >= 512) reading the given atoms. Arguments as
+ * nvfp4_linear, with w_scale_atoms / bn instead of w_scale; the same workspace size.
+ * The result is bit for bit that of nvfp4_linear at the same tile width.
+ * Errors as nvfp4_linear; QL_ERR_SHAPE for a bn outside {128, 192, 224, 256}. */
+int nvfp4_linear_laid_out(const void* x, int64_t M, int64_t K, const uint8_t* w,
+                          const uint8_t* w_scale_atoms, int bn, int64_t N,
+                          const float* weight_scale_2, const float* input_scale,
+                          const float* bias, void* y, void* workspace, size_t workspace_bytes,
+                          ql_stream_t stream);
+
 /* NVFP4 W4A4 linear forward: quantizes x at run time with input_scale and
  * contracts it on the tensor cores against the pre-quantized weight.
  * Two launches on `stream`: nvfp4_linear_prologue, then nvfp4_linear_gemm

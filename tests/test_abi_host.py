@@ -114,6 +114,25 @@ def test_argument_errors_before_device():
     assert lib.int4_linear_gemm(fake, fake, M, K, fake, fake, N, fake + 2, fake, fake, big, None) == 3
     assert lib.int4_linear_gemm(fake, fake, M, K, fake, fake, N, None, fake + 1, fake, big, None) == 3
     assert lib.int4_linear_gemm(fake, fake, M, K, fake, fake, N, None, fake, odd, big, None) == 3
+    # weight scales laid out once: sizes, tile widths, workspace and alignment
+    assert lib.nvfp4_weight_scale_atoms_size(N, K, 96) == 0
+    assert lib.nvfp4_weight_scale_atoms_size(N, 40, 128) == 0
+    # atoms: ceil(N / bn) tiles x K/64 groups x ceil(bn / 128) atoms of 512 bytes
+    assert lib.nvfp4_weight_scale_atoms_size(N, K, 224) == -(-N // 224) * (K // 64) * 2 * 512
+    assert lib.nvfp4_weight_scale_atoms_size(N, K, 128) == -(-N // 128) * (K // 64) * 512
+    big = 1 << 30
+    assert lib.nvfp4_layout_weight_scales(None, N, K, 128, fake, big, None) == 1
+    assert lib.nvfp4_layout_weight_scales(fake, N, K, 96, fake, big, None) == 2
+    assert lib.nvfp4_layout_weight_scales(fake, N, K, 128, fake, 16, None) == 5
+    assert lib.nvfp4_layout_weight_scales(fake, N, K, 128, odd, big, None) == 3
+    assert lib.nvfp4_linear_laid_out(fake, M, K, fake, fake, 100, N, fake, fake, None, fake,
+                                     fake, big, None) == 2
+    assert lib.nvfp4_linear_laid_out(fake, M, K, fake, odd, 128, N, fake, fake, None, fake,
+                                     fake, big, None) == 3
+    assert lib.nvfp4_linear_laid_out(fake, M, K, fake, fake, 128, N, fake, fake, None, fake,
+                                     fake, 16, None) == 5
+    assert lib.nvfp4_linear_laid_out(fake, M, K, fake, None, 128, N, fake, fake, None, fake,
+                                     fake, big, None) == 1
     # w4a16: null weight, K % 32, misaligned x, odd w_scale
     assert lib.w4a16_linear(fake, 1, K, None, fake, N, fake, None, fake, None) == 1
     assert lib.w4a16_linear(fake, 1, 48, fake, fake, N, fake, None, fake, None) == 2

@@ -231,3 +231,61 @@ def test_tile_override_rejects_bad_values():
     for bn, cg in [(80, 1), (96, 2), (64, 2), (128, 3), (320, 1)]:
         with pytest.raises(q.QLinearError):
             q.set_tile_override(bn, cg)
+
+
+# ----------------------------------------------------------------------------- weight scales laid out once
+
+def _laid_out_vs_linear(M, K, N, bn, seed, bias):
+    c = Nvfp4Case(M, K, N, seed=seed, bias=bias)
+    d = c.device_args()
+    cg = 2 if M >= 512 else 1
+    q.set_tile_override(bn, cg)
+    try:
+        y_ref = q.nvfp4_linear(d["x"], d["w"], d["w_scale"], d["weight_scale_2"],
+                               d["input_scale"], bias=d["bias"])
+    finally:
+        q.set_tile_override(0, 0)
+    atoms = q.nvfp4_layout_weight_scales(d["w_scale"], bn)
+    y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    q.nvfp4_linear_laid_out(d["x"], d["w"], atoms, bn, d["weight_scale_2"], d["input_scale"],
+                            bias=d["bias"], y=y)
+    torch.cuda.synchronize()
+    assert q.read_device_status() == 0
+    return c, y, y_ref
+
+
+@pytest.mark.parametrize("bn", [128, 192, 224, 256])
+def test_laid_out_weight_scales_same_bits_as_nvfp4_linear(bn):
+    # CTA pairs, ragged M and N; the same tile width through nvfp4_linear (which lays
+    # the scales out per call) and through the atoms laid out once
+    c, y, y_ref = _laid_out_vs_linear(600, 768, 520, bn, seed=bn, bias=True)
+    assert torch.equal(y, y_ref)
+    _, y64, T = c.reference()
+    check_linear(y, y64, T, f"nvfp4_linear_laid_out bn={bn}")
+
+
+@pytest.mark.parametrize("M", [17, 300])
+def test_laid_out_single_cta_tiles(M):
+    # one CTA per tile (M < 512), including a lone tile with fewer than 128 rows
+    c, y, y_ref = _laid_out_vs_linear(M, 1024, 1000, 192, seed=M, bias=False)
+    assert torch.equal(y, y_ref)
+    _, y64, T = c.reference()
+    check_linear(y, y64, T, f"nvfp4_linear_laid_out M={M}")
+
+
+def test_laid_out_atoms_equal_the_workspace_atoms():
+    # the atoms laid out once are byte for byte the weight part nvfp4_linear_prologue
+    # writes into its workspace for the same tile width
+    M, K, N = 4096, 3072, 12288
+    c = Nvfp4Case(256, K, N, seed=4)
+    d = c.device_args()
+    bn, _ = q.tile_config(M, N, K)
+    x = torch.zeros((M, K), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(q.nvfp4_linear_workspace_size(M, K, N), dtype=torch.uint8, device="cuda")
+    q.nvfp4_linear_prologue(x, d["w_scale"], d["input_scale"], ws)
+    _, _, wgt_off = q.nvfp4_linear_workspace_layout(M, K, N)
+    atoms = q.nvfp4_layout_weight_scales(d["w_scale"], bn)
+    torch.cuda.synchronize()
+    n = q.nvfp4_weight_scale_atoms_size(N, K, bn)
+    assert atoms.numel() == n
+    assert torch.equal(ws[wgt_off:wgt_off + n], atoms)
