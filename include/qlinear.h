@@ -172,8 +172,9 @@ int nvfp4_linear_quantized_input(int64_t M, int64_t K, const uint8_t* w, const u
 size_t nvfp4_linear_workspace_size(int64_t M, int64_t K, int64_t N);
 
 /* Weight block scales laid out once, for weights that do not change between calls
- * (a load-time step, like the weight's own quantization; the pages' mm_fp4 takes its
- * weight block scales in a prepared layout the same way). The tensor-core layout of
+ * (a load-time step, like the weight's own quantization; FlashInfer's mm_fp4, the
+ * kernel the pages name, is likewise handed its weight block scales already in its
+ * own layout). The tensor-core layout of
  * the scales depends on the GEMM's tile width bn (tiles of 224 rows do not align
  * with the 128-row scale atoms), so the atoms are made for one bn:
  *   nvfp4_weight_scale_atoms_size(N, K, bn)  bytes of the atoms (0 on bad sizes or
