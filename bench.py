@@ -514,8 +514,9 @@ def nvfp4_gemm_alg_bytes(M, K, N):
 
 
 def skinny_sweep(device, stream, peaks, steps):
-    """Per shape: the nvfp4_linear step and its GEMM alone, timed over rotating
-    buffer sets, against the roofline max(FLOPs / FP4 peak, bytes / HBM peak)."""
+    """Per shape: the nvfp4_linear step, the step on weight scales laid out once
+    (nvfp4_linear_laid_out, where the tile width allows) and the GEMM alone, timed over
+    rotating buffer sets, against the roofline max(FLOPs / FP4 peak, bytes / HBM peak)."""
     import torch
     fp4_peak = peaks["bf16_tflops"] * NOMINAL_FP4_OVER_BF16
     hbm = peaks["hbm_gbs"]
@@ -527,6 +528,10 @@ def skinny_sweep(device, stream, peaks, steps):
             rot = Nvfp4Rotation(L)
             reps = max(3, min(steps // rot.R, 20))
             st_ms = time_graph_rotation(rot.step, rot.R, reps, stream)
+            # weight scales laid out once (tile widths from 128; the skinny widths lay
+            # them out inside the GEMM and have no laid-out call)
+            lo_ms = (time_graph_rotation(rot.step_laid_out, rot.R, reps, stream)
+                     if L.atoms is not None else None)
             rot.prologue_all()
             g_ms = time_graph_rotation(rot.gemm, rot.R, reps, stream)
             fl = nvfp4_flops(M, K, N)
@@ -546,6 +551,10 @@ def skinny_sweep(device, stream, peaks, steps):
                 "gemm_roofline_frac": max(t_fl, t_gemm_b) / (g_ms / 1e3),
                 "tile": f"{128 * cg}x{bn}", "rotation_sets": rot.R,
             }
+            if lo_ms is not None:
+                out[f"M{M}_N{N}"].update({
+                    "step_laid_out_us": lo_ms * 1e3,
+                    "step_laid_out_roofline_frac": max(t_fl, t_step_b) / (lo_ms / 1e3)})
             del rot, L
             torch.cuda.empty_cache()
     return out

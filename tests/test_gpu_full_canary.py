@@ -193,3 +193,41 @@ def test_noalloc_w4a16_int4_write_nothing_outside():
     wg.check("int4_linear workspace")
     assert bool(torch.isfinite(yi.t).all())
     assert q.read_device_status() == 0
+
+
+@pytest.mark.parametrize("M,K,N,bn", [(600, 512, 520, 224), (64, 3072, 200, 128), (17, 96, 136, 192)])
+def test_laid_out_weight_scales_write_nothing_outside(M, K, N, bn):
+    # the atoms exactly fill their reported size; the laid-out linear writes only Y and
+    # the workspace (ragged N, a lone CTA, N % 8 != 0)
+    c = Nvfp4Case(M, K, N, seed=M + bn, bias=True)
+    d = c.device_args()
+    n_atoms = q.nvfp4_weight_scale_atoms_size(N, K, bn)
+    ag = Guarded(n_atoms, fill=0x5A)
+    q.nvfp4_layout_weight_scales(d["w_scale"], bn, atoms=ag.t)
+    ag.check("nvfp4_layout_weight_scales atoms")
+    yg = guarded_y(M, N)
+    wg = Guarded(q.nvfp4_linear_workspace_size(M, K, N), fill=0x5A)
+    q.nvfp4_linear_laid_out(d["x"], d["w"], ag.t, bn, d["weight_scale_2"], d["input_scale"],
+                            bias=d["bias"], y=yg.t, workspace=wg.t)
+    yg.check("nvfp4_linear_laid_out y")
+    wg.check("nvfp4_linear_laid_out workspace")
+    ag.check("nvfp4_linear_laid_out atoms (read only)")
+    _, y64, T = c.reference()
+    check_linear(yg.t, y64, T, "nvfp4_linear_laid_out inside the canaries")
+    assert q.read_device_status() == 0
+
+
+def test_int4_gemm_workspace_write_nothing_outside():
+    # the f16 operands and row factors stay inside int4_linear_gemm's workspace
+    M, K, N = 130, 576, 200
+    x = torch.randn(M, K, generator=torch.Generator().manual_seed(31)).to(torch.bfloat16)
+    w = (torch.randn(N, K, generator=torch.Generator().manual_seed(32)) * 0.02).to(torch.bfloat16)
+    xq, xs = q.int4_quantize_rows(to_dev(x))
+    wq, ws = q.prepare_int4_weight(to_dev(w))
+    wg = Guarded(q.int4_linear_gemm_workspace_size(M, K, N), fill=0x5A)
+    yg = guarded_y(M, N)
+    q.int4_linear_gemm(xq, xs, wq, ws, y=yg.t, workspace=wg.t)
+    wg.check("int4_linear_gemm workspace")
+    yg.check("int4_linear_gemm y")
+    assert bool(torch.isfinite(yg.t).all())
+    assert q.read_device_status() == 0
