@@ -263,6 +263,7 @@ static int nvfp4_gemm_impl(int64_t M, int64_t K, const uint8_t* w, int64_t N,
   p.timeout_ns = timeout_ns();
   p.inject_fault = g_inject_fault.load();
   p.pdl = pdl;
+  p.b_ready = true;  // the kernel before is this library's prologue: it does not write w
   p.lr_act = lr_act;
   p.lr_up = lr_up;
   p.lr_rank = lr_rank;
@@ -431,6 +432,7 @@ int nvfp4_linear_laid_out(const void* x, int64_t M, int64_t K, const uint8_t* w,
   p.timeout_ns = timeout_ns();
   p.inject_fault = g_inject_fault.load();
   p.pdl = true;
+  p.b_ready = true;  // the kernel before is the activation prologue: it does not write w
   e = ql::launch_gemm(p, s);
   return e == cudaSuccess ? QL_OK : record(e, "nvfp4_linear_laid_out gemm");
 }
@@ -640,6 +642,7 @@ static int fp8r_gemm_impl(const uint8_t* xq, const float* x_scale, int64_t M, in
   p.timeout_ns = timeout_ns();
   p.inject_fault = g_inject_fault.load();
   p.pdl = pdl;
+  p.b_ready = true;  // the kernel before is fp8r_quantize_rows: it does not write w
   cudaError_t e = ql::launch_gemm(p, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? QL_OK : record(e, "fp8r gemm launch");
 }

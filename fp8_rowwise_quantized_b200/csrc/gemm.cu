@@ -70,6 +70,8 @@ struct GemmArgs {
   uint64_t timeout_ns;
   int inject_fault;
   int wait_prior_grid;
+  int b_ready;              // plain non-skinny mode: B is not written by the previous kernel, so
+                            // the producer starts its first stages' B loads before the wait
   int use_tma_store;        // Y written through shared memory + TMA (needs N % 8 == 0)
   int raster_n;             // tile order: 1 = N fastest (m_blk = tile / tiles_n), 0 = M fastest
   // in-launch activation quantization (FP4, K % 256 == 0)
@@ -608,7 +610,9 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
   // the producer waits, and only after it has started the weight loads (the weights
   // and their scales do not come from the previous kernel; the MMA and epilogue
   // warps read nothing it writes).
-  if (args.wait_prior_grid && !SKINNY) grid_dependency_wait();
+  // (Plain mode with b_ready: the same, the producer waits after its first B loads.)
+  if (args.wait_prior_grid && !SKINNY && !(MODE == kModePlain && args.b_ready))
+    grid_dependency_wait();
 
 
   bool run = true;
@@ -818,6 +822,32 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     uint32_t phase = 0;
     bool ok = true;
     int issued = 0;
+    // b_ready: the first tile's first `pre` stages get their byte counts and weight
+    // loads before the wait for the previous kernel (which writes A and its scales)
+    int pre = 0;
+    if (MODE == kModePlain && args.wait_prior_grid && args.b_ready) {
+      if (group < args.total_tiles) {
+        int m_blk0, n_blk0;
+        tile_coords(group, args, m_blk0, n_blk0);
+        const int b_row0 = n_blk0 * BN + static_cast<int>(rank) * C::B_ROWS;
+        pre = args.num_k_tiles < C::STAGES ? args.num_k_tiles : C::STAGES;
+        const uint32_t kTx0 = C::STAGE_BYTES - C::A_BYTES + args.a_box_rows * 128;
+        if (elect_one()) {
+          for (int kt = 0; kt < pre; ++kt) {
+            uint8_t* sb = smem_b + kt * C::B_BYTES;
+            if constexpr (CG == 2) {
+              if (leader) mbar_arrive_expect_tx(&full_bar[kt], CG * kTx0);
+              tma_load_2d_pair(sb, &tmap_b, full_bar0 + kt * 8u, kt * 128, b_row0);
+            } else {
+              mbar_arrive_expect_tx(&full_bar[kt], kTx0);
+              tma_load_2d(sb, &tmap_b, &full_bar[kt], kt * 128, b_row0);
+            }
+          }
+        }
+        __syncwarp();
+      }
+      grid_dependency_wait();
+    }
     for (int tile = group; ok && tile < args.total_tiles; tile += ngroups) {
       int m_blk, n_blk;
       tile_coords(tile, args, m_blk, n_blk);
@@ -841,18 +871,20 @@ qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
                                                 C::NA);
 
           const uint32_t kTx = C::STAGE_BYTES - C::A_BYTES + args.a_box_rows * 128;
+          // a prefetched stage already has its byte count and its B load
+          const bool fresh = !(tile == group && kt < pre);
           if constexpr (CG == 2) {
-            if (leader) mbar_arrive_expect_tx(&full_bar[stage], CG * kTx);
+            if (leader && fresh) mbar_arrive_expect_tx(&full_bar[stage], CG * kTx);
             tma_load_2d_pair(sa, &tmap_a, fb, kt * 128, a_row);
-            tma_load_2d_pair(sb, &tmap_b, fb, kt * 128, b_row);
+            if (fresh) tma_load_2d_pair(sb, &tmap_b, fb, kt * 128, b_row);
             if constexpr (FP4) {
               tma_load_2d_pair(ssa, &tmap_sfa, fb, 0, sfa_atom);
               tma_load_2d_pair(ssb, &tmap_sfb, fb, 0, sfb_atom);
             }
           } else {
-            mbar_arrive_expect_tx(&full_bar[stage], kTx);
+            if (fresh) mbar_arrive_expect_tx(&full_bar[stage], kTx);
             tma_load_2d(sa, &tmap_a, &full_bar[stage], kt * 128, a_row);
-            tma_load_2d(sb, &tmap_b, &full_bar[stage], kt * 128, b_row);
+            if (fresh) tma_load_2d(sb, &tmap_b, &full_bar[stage], kt * 128, b_row);
             if constexpr (FP4) {
               tma_load_2d(ssa, &tmap_sfa, &full_bar[stage], 0, sfa_atom);
               tma_load_2d(ssb, &tmap_sfb, &full_bar[stage], 0, sfb_atom);
@@ -1458,6 +1490,7 @@ cudaError_t launch_typed(const GemmProblem& p, cudaStream_t stream) {
   a.timeout_ns = p.timeout_ns;
   a.inject_fault = p.inject_fault;
   a.wait_prior_grid = p.pdl ? 1 : 0;
+  a.b_ready = (MODE == kModePlain && p.b_ready) ? 1 : 0;
   a.use_tma_store = tma_store ? 1 : 0;
   a.raster_n = 0;
   if (MODE == kModeGeluQuant) {

@@ -36,6 +36,8 @@ struct GemmProblem {
   uint64_t timeout_ns;
   int inject_fault;
   bool pdl;              // launched right after its producer kernel (programmatic dependency)
+  bool b_ready;          // with pdl: B (the weight codes) is not written by that kernel, so the
+                         // GEMM may start loading it before the wait (plain mode)
   // fused (FP4, K % 256 == 0): the launch first quantizes x into a (codes) and
   // sfa (scale atoms) and lays out the row-major weight scales into sfb (atoms for
   // tile width bn), then runs the GEMM on them
