@@ -151,6 +151,41 @@ def test_skinny_linear_matches_split_calls(M):
     check_linear(y1, y64, T, "skinny nvfp4_linear")
 
 
+@pytest.mark.parametrize("M,K,bn", [(1, 800, 64), (17, 800, 96), (40, 3072, 128),
+                                    (64, 800, 128), (16, 3072, 0)])
+def test_skinny_linear_leaves_the_quantized_activations(M, K, bn):
+    # the skinny layer quantizes its activations inside the GEMM (one launch); the
+    # CTAs of the first column of tiles leave the codes and scale atoms in the
+    # workspace: the codes are the oracle's, and codes and atoms are byte for byte
+    # what nvfp4_linear_prologue writes (ragged K: 800 is not a multiple of 256)
+    N = 1000
+    if bn:
+        q.set_tile_override(bn, 1)
+    try:
+        c = Nvfp4Case(M, K, N, seed=M + K, bias=True)
+        d = c.device_args()
+        n = q.nvfp4_linear_workspace_size(M, K, N)
+        codes_off, sf_off, wgt_off = q.nvfp4_linear_workspace_layout(M, K, N)
+        ws1 = torch.full((n,), 0xA5, dtype=torch.uint8, device="cuda")
+        ws2 = ws1.clone()
+        y = q.nvfp4_linear(d["x"], d["w"], d["w_scale"], d["weight_scale_2"], d["input_scale"],
+                           bias=d["bias"], workspace=ws1)
+        q.nvfp4_linear_prologue(d["x"], d["w_scale"], d["input_scale"], ws2)
+        torch.cuda.synchronize()
+    finally:
+        q.set_tile_override(0, 0)
+    xq, _ = c.oracle_act()
+    n_codes = M * (K // 2)
+    assert np.array_equal(ws1[codes_off:codes_off + n_codes].cpu().numpy(), xq.reshape(-1))
+    kg = (K + 255) // 256 * 4
+    n_atoms = (M + 127) // 128 * kg * 512
+    assert sf_off + n_atoms <= wgt_off
+    assert torch.equal(ws1[sf_off:sf_off + n_atoms], ws2[sf_off:sf_off + n_atoms])
+    assert torch.equal(ws1[codes_off:codes_off + n_codes], ws2[codes_off:codes_off + n_codes])
+    _, y64, T = c.reference()
+    check_linear(y, y64, T, "skinny nvfp4_linear, one launch")
+
+
 def test_nvfp4_linear_repeatable():
     c = Nvfp4Case(1024, 3072, 3072, seed=6)
     d = c.device_args()
