@@ -166,6 +166,10 @@ nvfp4_prologue_kernel(const uint16_t* __restrict__ x, int M, int K,
                       const uint8_t* __restrict__ ws, int64_t N, int bn, int na, int64_t n_tiles,
                       int64_t w_jobs, uint8_t* __restrict__ wout) {
   if constexpr (EARLY) grid_dependents_launch();
+  // launched as a programmatic dependent of the kernel before it (the previous layer's
+  // GEMM lets it be scheduled at its own start): nothing is read before that kernel
+  // has completed and its writes are visible
+  grid_dependency_wait();
   __shared__ WsTile tile;
   // the block's first weight-scale job: its loads are in flight during the activation
   // items, so their latency is off the block's critical path
@@ -372,12 +376,23 @@ cudaError_t launch_nvfp4_prologue(const void* x, int64_t M, int64_t K, const uin
   if (need < w_jobs) need = w_jobs;
   const int64_t blocks = need < wave ? need : wave;
   auto kern = early_kernel ? nvfp4_prologue_kernel<true> : nvfp4_prologue_kernel<false>;
-  kern<<<static_cast<unsigned>(blocks), kQuantThreads, 0, s>>>(
-      static_cast<const uint16_t*>(x), static_cast<int>(M), static_cast<int>(K), input_scale,
-      workspace + L.codes_off, workspace + L.act_sf_off, static_cast<uint32_t>(rows),
-      static_cast<uint32_t>(segs), static_cast<int>(KG), w_scale, N, bn, na, n_tiles, w_jobs,
-      workspace + L.wgt_sf_off);
-  return cudaGetLastError();
+  // a programmatic dependent of the kernel before it: its blocks may be resident and
+  // waiting while that kernel finishes (the kernel waits before any memory access)
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+  cfg.blockDim = dim3(kQuantThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<const uint16_t*>(x), static_cast<int>(M),
+                            static_cast<int>(K), input_scale, workspace + L.codes_off,
+                            workspace + L.act_sf_off, static_cast<uint32_t>(rows),
+                            static_cast<uint32_t>(segs), static_cast<int>(KG), w_scale, N, bn, na,
+                            n_tiles, w_jobs, workspace + L.wgt_sf_off);
 }
 
 cudaError_t launch_nvfp4_weight_atoms(const uint8_t* w_scale, int64_t K, int64_t N, int bn,
