@@ -153,6 +153,27 @@ def test_no_device_reports_error_instead_of_crashing():
     assert lib.ql_read_device_status(C.byref(st)) in (4, 6)
 
 
+def test_tile_choice_of_the_dit_layers():
+    # the cost model's picks for the benchmarked layers (host logic, no device):
+    # 256 x 224 CTA-pair tiles for the MLP up projection and the fused QKV, 256 x 256 for
+    # the MLP down projection, 256 x 192 for the attention projection; below 512 rows
+    # one CTA per 128-row tile; at most 64 rows the skinny kernels with the narrowest
+    # width whose tiles fit one wave of 148 SMs
+    import fp8_rowwise_quantized_b200 as q
+    assert q.tile_config(4096, 12288, 3072) == (224, 2)
+    assert q.tile_config(4096, 9216, 3072) == (224, 2)
+    assert q.tile_config(4096, 3072, 12288) == (256, 2)
+    assert q.tile_config(4096, 3072, 3072) == (192, 2)
+    assert q.tile_config(256, 12288, 3072) == (192, 1)
+    assert q.tile_config(16, 12288, 3072) == (96, 1)     # 128 tiles
+    assert q.tile_config(16, 3072, 3072) == (64, 1)      # 48 tiles
+    assert q.tile_config(64, 18432, 3072) == (128, 1)    # 144 tiles
+    assert q.tile_config(65, 3072, 3072)[0] >= 128       # 65 rows: no skinny kernel
+    for M, N in [(1, 3072), (16, 12288), (64, 18432)]:
+        bn, cg = q.tile_config(M, N, 3072)
+        assert cg == 1 and -(-N // bn) <= 148
+
+
 def test_tile_config_is_host_only_and_follows_override():
     import fp8_rowwise_quantized_b200 as q
     bn, cg = q.tile_config(4096, 12288, 3072)
