@@ -81,3 +81,34 @@ def test_reference_arm_prints_one_json_line():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_traffic_record_describes_the_current_gemm():
+    # the DRAM bytes bench.py reports as roofline.traffic come from an ncu capture keyed
+    # on the GEMM's sources: they must match the sources as committed
+    sys.path.insert(0, ROOT)
+    import bench
+    nbytes, note = bench.traffic_from_profiles("nvfp4_gemm_mlp_up")
+    assert nbytes is not None, note
+    # at least the operands read once, at most the algorithmic bytes of the launch
+    M, K, N = 4096, 3072, 12288
+    operands = M * K // 2 + M * K // 16 + N * K // 2 + N * K // 16
+    assert operands <= nbytes <= operands + 2 * M * N
+
+
+def test_traffic_record_goes_stale_when_a_source_changes(tmp_path, monkeypatch):
+    sys.path.insert(0, ROOT)
+    import json
+    import bench
+    src = tmp_path / "k.cu"
+    src.write_text("kernel v1\n")
+    (tmp_path / "profiles").mkdir()
+    rec = {"bytes_per_launch": 123, "note": "n", "sources": ["k.cu"]}
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    rec["source_sha1"] = bench.source_hash(rec["sources"])
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps({"k": rec}))
+    assert bench.traffic_from_profiles("k") == (123, "n")
+    src.write_text("kernel v2\n")
+    nbytes, note = bench.traffic_from_profiles("k")
+    assert nbytes is None and "stale" in note
+    assert bench.traffic_from_profiles("missing")[0] is None
