@@ -181,6 +181,24 @@ def test_fp8r_representable_rows_are_exact():
     assert np.array_equal(np.vectorize(oracle.e4m3_decode)(q), vals / scale)
 
 
+def test_fp8r_worked_row_golden():
+    # one row worked by exact rational arithmetic (the fixture's header): the scale bits,
+    # the reciprocal-multiply reading (it differs from a division on four elements), a
+    # subnormal code, zero and a negative value
+    rows = {}
+    with open(os.path.join(GOLDEN, "fp8r_worked_row.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                key, *vals = line.split()
+                rows[key] = [int(v, 16) for v in vals]
+    bits = np.array(rows["x_bits"], np.uint16)
+    x = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).reshape(1, -1)
+    q, s = oracle.fp8r_quantize_rows(x)
+    assert int(s.view(np.uint32)[0]) == rows["scale_bits"][0]
+    assert list(q[0]) == rows["codes"]
+
+
 def test_nvfp4_scale_constant_rounding_order_golden():
     rows = {}
     with open(os.path.join(GOLDEN, "nvfp4_rounding_order.txt")) as f:
