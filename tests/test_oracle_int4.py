@@ -184,3 +184,23 @@ def test_hand_worked_groups_from_golden_file():
     want_y = float(fields["y"][0])
     got = torch.tensor([int(y[0, 0])], dtype=torch.int32).to(torch.int16).view(torch.bfloat16)
     assert float(got.float()[0]) == want_y
+
+
+def test_reciprocal_group_golden():
+    """tests/golden/int4_reciprocal_group.txt: a group whose codes differ between
+    x * RN32(1/scale) (the reading) and x / scale (a tie there), worked by exact
+    arithmetic."""
+    import os
+    rows = {}
+    path = os.path.join(os.path.dirname(__file__), "golden", "int4_reciprocal_group.txt")
+    with open(path) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                key, *vals = line.split()
+                rows[key] = [int(v, 16) for v in vals]
+    b = np.array(rows["x_bits"], np.uint16)
+    x = torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).reshape(1, -1)
+    q, s = oracle.int4_quantize(x)
+    assert int(s.view(np.uint32)[0, 0]) == rows["scale_bits"][0]
+    assert list(q[0]) == rows["bytes"]

@@ -199,6 +199,32 @@ def test_fp8r_worked_row_golden():
     assert list(q[0]) == rows["codes"]
 
 
+def _golden_hex(name):
+    rows = {}
+    with open(os.path.join(os.path.dirname(__file__), "golden", name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                key, *vals = line.split()
+                rows[key] = [int(v, 16) for v in vals]
+    return rows
+
+
+def _bf16_row(bits):
+    b = np.array(bits, np.uint16)
+    return torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).reshape(1, -1)
+
+
+def test_nvfp4_reciprocal_block_golden():
+    # a block worked by exact arithmetic whose codes differ on five elements between
+    # x * RN32(1/d) (the reading) and x / d (ties there)
+    rows = _golden_hex("nvfp4_reciprocal_block.txt")
+    g = float(np.array(rows["g_bits"], np.uint32).view(np.float32)[0])
+    q, s = oracle.nvfp4_quantize(_bf16_row(rows["x_bits"]), g)
+    assert list(s[0]) == rows["scales"]
+    assert list(q[0]) == rows["bytes"]
+
+
 def test_nvfp4_scale_constant_rounding_order_golden():
     rows = {}
     with open(os.path.join(GOLDEN, "nvfp4_rounding_order.txt")) as f:

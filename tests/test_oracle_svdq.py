@@ -83,3 +83,23 @@ def test_zero_residual_closed_form_and_linearity():
     up2 = _bits(torch.from_numpy(2 * ui).to(torch.bfloat16))
     _, y64b, _, _ = oracle.svdq_nvfp4_linear(xq, xs, wq, ws, 1.0, 1.0, Di.astype(float), up2, bias)
     assert np.array_equal(y64b - bias, 2 * (y64 - bias))
+
+
+def test_smoothing_rounds_to_fp32_first_golden():
+    """tests/golden/svdq_smoothing_rounding.txt: the fp32 product lands exactly on a
+    bf16 midpoint (a tie to even), where one rounding of the exact product would go the
+    other way."""
+    import os
+    rows = {}
+    path = os.path.join(os.path.dirname(__file__), "golden", "svdq_smoothing_rounding.txt")
+    with open(path) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                key, *vals = line.split()
+                rows[key] = [int(v, 16) for v in vals]
+    x = torch.from_numpy(np.array(rows["x_bits"], np.uint16).view(np.int16)).view(
+        torch.bfloat16).reshape(1, 1)
+    smooth = np.array(rows["smooth_bits"], np.uint32).view(np.float32)
+    out = oracle.smooth_bf16(x, smooth)
+    assert int(out[0, 0]) == rows["xs_bits"][0]
