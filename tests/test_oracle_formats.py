@@ -171,3 +171,21 @@ def test_bf16_from_double_single_rounding():
     got = oracle.bf16_from_double(np.array([1 + 2.0 ** -8, 1 + 2.0 ** -8 + 2.0 ** -40,
                                             -(1 + 3 * 2.0 ** -8)]))
     assert list(got) == [0x3F80, 0x3F81, 0xBF82]
+
+
+def test_bf16_from_double_subnormals_vs_torch():
+    # the fp32 subnormal range, where bf16 keeps a quantum of 2^-133: one rounding from
+    # fp64 equals torch's fp32 -> bf16 round-to-nearest-even cast
+    pos = np.arange(1, 0x800000, 13, dtype=np.uint32)
+    f = np.concatenate([pos, pos | np.uint32(0x80000000)]).view(np.float32)
+    ref = torch.from_numpy(f).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = oracle.bf16_from_double(f.astype(np.float64))
+    bad = np.nonzero(got != ref)[0]
+    assert bad.size == 0, [(float(f[i]), hex(got[i]), hex(ref[i])) for i in bad[:10]]
+
+
+def test_e4m3_encode_nan_is_a_nan_code():
+    # E4M3 (OCP) has no infinity; its NaN is S.1111.111
+    codes = oracle.e4m3_encode(np.float32([np.nan, -np.nan]))
+    assert all(c & 0x7F == 0x7F for c in codes)
+    assert all(np.isnan(oracle.e4m3_decode(int(c))) for c in codes)

@@ -130,6 +130,18 @@ def test_nvfp4_sign_symmetry_and_zero_block():
     assert not qz.any() and not sz.any()
 
 
+def test_nvfp4_block_whose_scale_rounds_to_zero_encodes_zeros():
+    # tiny values of either sign: the block scale rounds to E4M3 zero, so d = 0 and the
+    # whole block is encoded as +0 codes (no -0 nibbles)
+    x = torch.full((1, 32), -(2.0 ** -30), dtype=torch.bfloat16)
+    x[0, 1::2] = 2.0 ** -31
+    x[0, 16:] = 1.0                             # the second block is ordinary
+    q, s = oracle.nvfp4_quantize(x, 1.0)
+    assert s[0, 0] == 0 and s[0, 1] != 0
+    assert not q[0, :8].any()
+    assert q[0, 8:].all()
+
+
 def test_nvfp4_saturation_when_input_scale_too_small():
     inp = make_linear_inputs(4, 256, 1, seed=6)
     g = oracle.nvfp4_global_scale(inp.x) / 4   # activations exceed the calibration

@@ -103,3 +103,32 @@ def test_smoothing_rounds_to_fp32_first_golden():
     smooth = np.array(rows["smooth_bits"], np.uint32).view(np.float32)
     out = oracle.smooth_bf16(x, smooth)
     assert int(out[0, 0]) == rows["xs_bits"][0]
+
+
+def test_low_rank_term_is_not_scaled_by_the_global_scales():
+    # with a zero 4-bit residual, Y = D up^T + bias whatever input_scale and
+    # weight_scale_2 are: only the 4-bit product carries them
+    M, K, N, r = 4, 64, 6, 3
+    rng = np.random.default_rng(5)
+    xq = np.zeros((M, K // 2), dtype=np.uint8)
+    xs = np.full((M, K // 16), 0x38, dtype=np.uint8)
+    wq = np.zeros((N, K // 2), dtype=np.uint8)
+    ws = np.full((N, K // 16), 0x38, dtype=np.uint8)
+    Di = rng.integers(-5, 6, size=(M, r))
+    ui = rng.integers(-5, 6, size=(N, r))
+    up = _bits(torch.from_numpy(ui).to(torch.bfloat16))
+    bias = np.arange(N, dtype=np.float32)
+    _, y64, _, _ = oracle.svdq_nvfp4_linear(xq, xs, wq, ws, 0.5, 0.25, Di.astype(float), up, bias)
+    assert np.array_equal(y64, (Di @ ui.T).astype(np.float64) + bias)
+
+
+def test_lowrank_down_is_exact_under_cancellation():
+    # 2^24 + 1 - 2^24: an fp32 accumulation loses the 1, the exact contraction keeps it
+    K = 16
+    xi = np.zeros((2, K))
+    xi[0, :3] = [2.0 ** 24, 1.0, -(2.0 ** 24)]
+    xi[1, :4] = [2.0 ** 30, 3.0, -(2.0 ** 30), 0.5]
+    xs = _bits(torch.from_numpy(xi).to(torch.bfloat16))
+    down = _bits(torch.ones(1, K, dtype=torch.bfloat16))
+    D = oracle.lowrank_down(xs, down)
+    assert D[0, 0] == 1.0 and D[1, 0] == 3.5
