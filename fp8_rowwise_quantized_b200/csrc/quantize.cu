@@ -166,9 +166,9 @@ nvfp4_prologue_kernel(const uint16_t* __restrict__ x, int M, int K,
                       const uint8_t* __restrict__ ws, int64_t N, int bn, int na, int64_t n_tiles,
                       int64_t w_jobs, uint8_t* __restrict__ wout) {
   if constexpr (EARLY) grid_dependents_launch();
-  // launched as a programmatic dependent of the kernel before it (the previous layer's
-  // GEMM lets it be scheduled at its own start): nothing is read before that kernel
-  // has completed and its writes are visible
+  // launched as a programmatic dependent of the kernel before it (a skinny GEMM of the
+  // previous layer lets it be scheduled at that GEMM's start): nothing is read or
+  // written before that kernel has completed and its writes are visible
   grid_dependency_wait();
   __shared__ WsTile tile;
   // the block's first weight-scale job: its loads are in flight during the activation
