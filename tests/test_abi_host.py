@@ -140,6 +140,76 @@ def test_argument_errors_before_device():
     assert lib.w4a16_linear(fake, 1, K, fake, fake + 1, N, fake, None, fake, None) == 3
 
 
+def test_argument_errors_of_the_split_fused_and_extension_calls():
+    # every check runs before the device is touched: null pointers (1), shapes (2),
+    # alignment (3), workspace (5), in the order each entry point documents
+    lib = _lib.load()
+    fake, odd, big = 1 << 20, (1 << 20) + 8, 1 << 30
+    M, K, N = 128, 256, 256
+    al = lambda b: -(-b // 1024) * 1024
+    # nvfp4_linear_prologue(x, M, K, w_scale, N, input_scale, workspace, bytes, stream)
+    assert lib.nvfp4_linear_prologue(None, M, K, fake, N, fake, fake, big, None) == 1
+    assert lib.nvfp4_linear_prologue(fake, M, 40, fake, N, fake, fake, big, None) == 2
+    assert lib.nvfp4_linear_prologue(odd, M, K, fake, N, fake, fake, big, None) == 3
+    assert lib.nvfp4_linear_prologue(fake, M, K, fake, N, fake, fake, 16, None) == 5
+    assert lib.nvfp4_linear_prologue(fake, M, K, fake, N, fake, odd, big, None) == 3
+    # nvfp4_linear_gemm(M, K, w, N, weight_scale_2, input_scale, bias, y, workspace, bytes, s)
+    assert lib.nvfp4_linear_gemm(M, K, None, N, fake, fake, None, fake, fake, big, None) == 1
+    assert lib.nvfp4_linear_gemm(M, K, fake, N, fake, fake, None, odd, fake, big, None) == 3
+    assert lib.nvfp4_linear_gemm(M, K, fake, N, fake, fake, odd, fake, fake, big, None) == 3
+    assert lib.nvfp4_linear_gemm(M, K, fake, N, fake, fake, None, fake, None, big, None) == 5
+    # nvfp4_linear_gemm_lowrank(..., bias, lr_act, lr_up, rank, y, workspace, bytes, s)
+    lr = lambda act, rank: lib.nvfp4_linear_gemm_lowrank(M, K, fake, N, fake, fake, None, act,
+                                                         fake, rank, fake, fake, big, None)
+    assert lr(None, 32) == 1
+    assert lr(fake, 12) == 2 and lr(fake, 72) == 2 and lr(fake, 0) == 2
+    assert lr(odd, 32) == 3
+    # nvfp4_linear_single_launch: K % 256 == 0 and a 16-byte aligned w_scale as well
+    sl = lambda k, w_scale, nbytes: lib.nvfp4_linear_single_launch(
+        fake, M, k, fake, w_scale, N, fake, fake, None, fake, fake, nbytes, None)
+    assert sl(288, fake, big) == 2
+    assert sl(K, odd, big) == 3
+    assert sl(K, fake, 16) == 5
+    # nvfp4_linear_gelu_quantize(x, M, K, w, w_scale, N, ws2, is, bias, next_is,
+    #                            next_workspace, next_bytes, workspace, bytes, s)
+    gq = lambda n, next_is, next_ws, next_bytes, ws: lib.nvfp4_linear_gelu_quantize(
+        fake, M, K, fake, fake, n, fake, fake, None, next_is, next_ws, next_bytes, ws, big, None)
+    assert gq(N, None, fake, big, fake) == 1
+    assert gq(200, fake, fake, big, fake) == 2             # N % 256 != 0
+    assert gq(N, fake, odd, big, fake) == 3
+    assert gq(N, fake, fake, 16, fake) == 5
+    assert gq(N, fake, fake, big, None) == 5
+    # nvfp4_linear_quantized_input(M, K, w, w_scale, N, ws2, is, bias, y, workspace, bytes, s)
+    qi = lambda k, ws, nbytes: lib.nvfp4_linear_quantized_input(
+        M, k, fake, fake, N, fake, fake, None, fake, ws, nbytes, None)
+    assert qi(K, None, big) == 1
+    assert qi(48, fake, big) == 2
+    assert qi(K, fake, 16) == 5
+    assert qi(K, odd, big) == 3
+    # svdq_nvfp4_linear(x, M, K, smooth, down, up, rank, w, w_scale, N, ws2, is, bias, y,
+    #                   workspace, bytes, s); its workspace adds lr_act bf16 [M, rank]
+    need = lib.svdq_nvfp4_linear_workspace_size(M, K, N, 32)
+    assert need == lib.nvfp4_linear_workspace_size(M, K, N) + al(M * 32 * 2)
+    assert lib.svdq_nvfp4_linear_workspace_size(M, K, N, 4) == 0
+    assert lib.svdq_nvfp4_linear_workspace_size(M, K, N, 72) == 0
+    sv = lambda smooth, down, rank, nbytes: lib.svdq_nvfp4_linear(
+        fake, M, K, smooth, down, fake, rank, fake, fake, N, fake, fake, None, fake, fake, nbytes,
+        None)
+    assert sv(None, None, 32, big) == 1
+    assert sv(None, fake, 30, big) == 2
+    assert sv(odd, fake, 32, big) == 3                     # the smoothing vector
+    assert sv(None, fake, 32, need - 1) == 5
+    # fp8r_linear_gemm(xq, x_scale, M, K, w, w_scale, N, bias, y, s)
+    assert lib.fp8r_linear_gemm(None, fake, M, K, fake, fake, N, None, fake, None) == 1
+    assert lib.fp8r_linear_gemm(fake, fake, M, 40, fake, fake, N, None, fake, None) == 2
+    assert lib.fp8r_linear_gemm(odd, fake, M, K, fake, fake, N, None, fake, None) == 3
+    # calibration and the element encoders
+    assert lib.nvfp4_global_scale(None, 10, fake, None) == 1
+    assert lib.nvfp4_global_scale(fake, 0, fake, None) == 1
+    assert lib.ql_encode_e2m1(fake, None, 10, None) == 1
+    assert lib.ql_encode_e2m1(fake, fake, 0, None) == 1
+
+
 def test_no_device_reports_error_instead_of_crashing():
     import torch
     if torch.cuda.is_available():
