@@ -257,3 +257,43 @@ def test_tile_config_is_host_only_and_follows_override():
     assert q.tile_config(4096, 12288, 3072) == (bn, cg)
     lib = _lib.load()
     assert lib.ql_tile_config(1, 0, 1, 1, None, None) == _lib.QL_ERR_INVALID_ARG
+
+
+def test_binding_rejects_host_tensors_without_computing():
+    # there is no CPU path: every compute call given host tensors raises before any
+    # work is done, instead of falling back to another implementation
+    import torch
+    import fp8_rowwise_quantized_b200 as q
+    M, K, N = 16, 256, 128
+    x = torch.zeros((M, K), dtype=torch.bfloat16)
+    w4 = torch.zeros((N, K // 2), dtype=torch.uint8)
+    s4 = torch.zeros((N, K // 16), dtype=torch.uint8)
+    one = torch.ones(1, dtype=torch.float32)
+    w8 = torch.zeros((N, K), dtype=torch.uint8)
+    rows = torch.ones(N, dtype=torch.float32)
+    i4s = torch.ones((N, K // 64), dtype=torch.float32)
+    down = torch.zeros((32, K), dtype=torch.bfloat16)
+    up = torch.zeros((N, 32), dtype=torch.bfloat16)
+    nws = torch.zeros(1 << 20, dtype=torch.uint8)
+    calls = {
+        "nvfp4_quantize_act": lambda: q.nvfp4_quantize_act(x, one),
+        "nvfp4_global_scale": lambda: q.nvfp4_global_scale(x),
+        "nvfp4_linear": lambda: q.nvfp4_linear(x, w4, s4, one, one),
+        "nvfp4_layout_weight_scales": lambda: q.nvfp4_layout_weight_scales(s4, 128),
+        "nvfp4_linear_laid_out": lambda: q.nvfp4_linear_laid_out(x, w4, nws, 128, one, one),
+        "nvfp4_linear_single_launch": lambda: q.nvfp4_linear_single_launch(x, w4, s4, one, one),
+        "nvfp4_linear_noalloc": lambda: q.nvfp4_linear_noalloc(x, w4, s4, one, one),
+        "nvfp4_linear_gelu_quantize": lambda: q.nvfp4_linear_gelu_quantize(
+            x, w4, s4, one, one, one, nws),
+        "nvfp4_linear_quantized_input": lambda: q.nvfp4_linear_quantized_input(
+            M, w4, s4, one, one, nws),
+        "svdq_nvfp4_linear": lambda: q.svdq_nvfp4_linear(x, w4, s4, one, one, down, up),
+        "w4a16_linear": lambda: q.w4a16_linear(x, w4, s4, one),
+        "fp8r_quantize_rows": lambda: q.fp8r_quantize_rows(x),
+        "fp8r_linear": lambda: q.fp8r_linear(x, w8, rows),
+        "int4_quantize_rows": lambda: q.int4_quantize_rows(x),
+        "int4_linear": lambda: q.int4_linear(x, w4, i4s),
+    }
+    for name, call in calls.items():
+        with pytest.raises(ValueError, match="CUDA tensor"):
+            call()
