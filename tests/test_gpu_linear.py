@@ -186,6 +186,43 @@ def test_skinny_linear_leaves_the_quantized_activations(M, K, bn):
     check_linear(y, y64, T, "skinny nvfp4_linear, one launch")
 
 
+def test_skinny_layer_output_feeds_the_next_layer_at_once():
+    # a skinny GEMM lets the next kernel on the stream launch at its start; the next
+    # layer's prologue must still read this layer's finished output. Two skinny layers
+    # back to back, no synchronisation between them, the first output starting as NaN.
+    from synthetic import make_linear_inputs
+    M, K1, N1, N2 = 16, 256, 512, 256
+    assert q.tile_config(M, N1, K1)[0] < 128 and q.tile_config(M, N2, N1)[0] < 128
+    inp1 = make_linear_inputs(M, K1, N1, seed=21)
+    inp2 = make_linear_inputs(M, N1, N2, seed=22)
+    g1 = oracle.nvfp4_global_scale(inp1.w)
+    w1q, w1s = oracle.nvfp4_quantize(inp1.w, g1)
+    g2 = oracle.nvfp4_global_scale(inp2.w)
+    w2q, w2s = oracle.nvfp4_quantize(inp2.w, g2)
+    gx1 = oracle.nvfp4_global_scale(inp1.x)
+    # the second layer's input scale: calibrated on the oracle's first-layer output
+    xq1, xs1 = oracle.nvfp4_quantize(inp1.x, gx1)
+    y1_ref, _, _ = oracle.nvfp4_linear(xq1, xs1, w1q, w1s, gx1, g1)
+    gx2 = oracle.nvfp4_global_scale(torch.from_numpy(y1_ref.view(np.int16)).view(torch.bfloat16))
+    x1 = to_dev(inp1.x)
+    d1 = dict(w=to_dev(w1q), w_scale=to_dev(w1s), weight_scale_2=scalar_dev(g1),
+              input_scale=scalar_dev(float(gx1)))
+    d2 = dict(w=to_dev(w2q), w_scale=to_dev(w2s), weight_scale_2=scalar_dev(g2),
+              input_scale=scalar_dev(float(gx2)))
+    for _ in range(3):
+        y1 = nan_output(M, N1)
+        y2 = nan_output(M, N2)
+        q.nvfp4_linear(x1, d1["w"], d1["w_scale"], d1["weight_scale_2"], d1["input_scale"], y=y1)
+        q.nvfp4_linear(y1, d2["w"], d2["w_scale"], d2["weight_scale_2"], d2["input_scale"], y=y2)
+        torch.cuda.synchronize()
+        assert bool(torch.isfinite(y1).all()) and bool(torch.isfinite(y2).all())
+        # the second layer against the oracle on the first layer's actual output
+        xq2, xs2 = oracle.nvfp4_quantize(y1.cpu(), gx2)
+        _, y64, T = oracle.nvfp4_linear(xq2, xs2, w2q, w2s, gx2, g2)
+        check_linear(y2, y64, T, "second skinny layer")
+    assert q.read_device_status() == 0
+
+
 def test_nvfp4_linear_repeatable():
     c = Nvfp4Case(1024, 3072, 3072, seed=6)
     d = c.device_args()
