@@ -202,7 +202,14 @@ int nvfp4_linear_laid_out(const void* x, int64_t M, int64_t K, const uint8_t* w,
 /* NVFP4 W4A4 linear forward: quantizes x at run time with input_scale and
  * contracts it on the tensor cores against the pre-quantized weight.
  * Two launches on `stream`: nvfp4_linear_prologue, then nvfp4_linear_gemm
- * (started early through programmatic dependent launch).
+ * (started early through programmatic dependent launch). The prologue is itself
+ * launched as a programmatic dependent of whatever precedes it on `stream`, and
+ * waits for that kernel to complete before it reads or writes memory. For M <= 64
+ * (the skinny kernels) the GEMM lets the next kernel on `stream` start early: a
+ * kernel the caller launches next with the programmatic-stream-serialization
+ * attribute must wait for its prerequisite grid (griddepcontrol.wait /
+ * cudaGridDependencySynchronize) before it reads y. Kernels launched without that
+ * attribute are ordered as usual.
  *   x              bf16 [M, K]
  *   w              uint8 [N, K/2]  packed E2M1 weight codes
  *   w_scale        uint8 [N, K/16] E4M3 weight block scales (row-major, as stored
